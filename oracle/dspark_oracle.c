@@ -1,0 +1,469 @@
+/*
+ * dspark_oracle.c -- plain, slow, single-threaded fp64 restatement of the
+ * per-round token path of DSpark (arXiv:2607.05147).
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the oracle that the CUDA path is
+ * checked against.  Only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark may load it.  It shares no code, header, table or helper
+ * with the CUDA library and includes nothing from it.
+ *
+ * Sources (web pages about the paper), cited below by tag:
+ *   [PL] paperlayer.ai, "DSpark: Confidence-Scheduled Speculative Decoding with
+ *        Semi-Autoregressive Generation" (section-by-section summary):
+ *        §2 Background, §3.1 Semi-autoregressive generation, §3.2
+ *        Confidence-scheduled verification, Appendix A (counterexample:
+ *        selection bias without early stopping).
+ *   [KB] menfem.com knowledge-base entry on the same paper: "Key
+ *        Contributions" and "Methodology".
+ *   [WK] llm-wiki.hwlabs.dev study 116 on DSpark: the draft-generation
+ *        figure of the semi-autoregressive Markov head section, and the
+ *        confidence-scheduling section.
+ *
+ * Arithmetic: every input (fp32, or bf16 values carried exactly in fp32) is
+ * widened to double; all sums run sequentially in index order; exp() is the C
+ * library's.  No blocking, fusion or reordering beyond the definitions.
+ *
+ * Readings where the pages are silent (each is listed in the design doc):
+ *   - the Markov bias at position i is U[x_{i-1}] W with x_0 the last committed
+ *     token, also at i = 1;
+ *   - temperature T scales draft and target logits alike; T = 0 means greedy
+ *     (argmax, lowest index on ties) with the exact-match accept rule;
+ *   - inverse-CDF sampling takes the smallest v with u < C_v;
+ *   - accept iff u < p_t(x)/p_d(x), i.e. with probability min(1, ratio);
+ *   - the scheduler objective is Theta(n) = (B + sum of admitted S) / t(n);
+ *     it stops at the first strict decrease (cross-multiplied compare);
+ *   - candidates are laid out position-major and sorted stably by S
+ *     descending, so ties go to the lower position, then the lower request;
+ *   - an all-zero residual falls back to sampling from p_t.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_NOMEM 2
+
+/* ------------------------------------------------------------------------ */
+/* Markov transition bias: [PL] §3.1 (a low-rank transition matrix conditions
+ * each position on the previously sampled token); [KB] Methodology (rank-256
+ * factorization); [WK] draft-generation figure (final logits L[i] + Delta[i]).
+ * delta[v] = sum_k U[a][k] * W[k][v], with U stored [V][r] and W stored [r][V]. */
+static void markov_bias_row(const float *U, const float *W, int V, int r, int a,
+                            double *delta)
+{
+    for (int v = 0; v < V; ++v) delta[v] = 0.0;
+    for (int k = 0; k < r; ++k) {
+        double uk = (double)U[(size_t)a * r + k];
+        const float *wk = W + (size_t)k * V;
+        for (int v = 0; v < V; ++v) delta[v] += uk * (double)wk[v];
+    }
+}
+
+/* Index of the largest entry (lowest index on ties) and the gap to the
+ * largest entry at any other index (the decision margin of an argmax). */
+static int argmax_with_gap(const double *z, int V, double *gap)
+{
+    int best = 0;
+    for (int v = 1; v < V; ++v)
+        if (z[v] > z[best]) best = v;
+    double second = -INFINITY;
+    for (int v = 0; v < V; ++v)
+        if (v != best && z[v] > second) second = z[v];
+    *gap = (V > 1) ? z[best] - second : INFINITY;
+    return best;
+}
+
+/* Inverse-CDF draw from non-negative weights e[0..V-1] with total tot:
+ * the smallest v with u < C_v, C_v = (e_0 + ... + e_v) / tot.  margin is the
+ * distance from u to the nearer end of the chosen interval.  If rounding
+ * leaves u >= C_{V-1}, the last index with positive weight is taken. */
+static int inverse_cdf(const double *e, int V, double tot, double u, double *margin)
+{
+    double run = 0.0, prev = 0.0;
+    for (int v = 0; v < V; ++v) {
+        run += e[v];
+        double c = run / tot;
+        if (u < c) {
+            double m0 = u - prev, m1 = c - u;
+            *margin = m0 < m1 ? m0 : m1;
+            return v;
+        }
+        prev = c;
+    }
+    int last = V - 1;
+    while (last > 0 && !(e[last] > 0.0)) --last;
+    *margin = 0.0;
+    return last;
+}
+
+/* Temperature softmax of one logit row: z = row / T, m = max z,
+ * e_v = exp(z_v - m), returns Z = sum e_v.  T > 0. */
+static double softmax_row(const double *row, int V, double T, double *e, double *m_out)
+{
+    double m = -INFINITY;
+    for (int v = 0; v < V; ++v) {
+        double z = row[v] / T;
+        if (z > m) m = z;
+    }
+    double Z = 0.0;
+    for (int v = 0; v < V; ++v) {
+        e[v] = exp(row[v] / T - m);
+        Z += e[v];
+    }
+    *m_out = m;
+    return Z;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stage 1, semi-autoregressive drafting: [PL] §3.1 (the parallel stage gives
+ * all draft logits in one pass; the sequential stage samples left to right,
+ * conditioning each position on the previously sampled token); [WK]
+ * draft-generation figure (L[i] + Delta[i], then sample the draft token).
+ *
+ * L [B][G][V], U [V][r], W [r][V]; x0 [B] last committed token per request;
+ * temp [B]; u_draft [B][G] uniforms in [0,1).  force_x (nullable, [B][G]):
+ * entries >= 0 replace the sampled token (used to follow another
+ * implementation's decision after a reported near-tie).
+ * Outputs per (b,i): x, pd = p_d(x), rowmax = max_v z_v, rowsum = sum exp(z-m),
+ * margin = decision margin.  For T = 0: x = argmax (L + Delta), pd = 1,
+ * rowmax = max (L + Delta), rowsum = 1, margin = top-two gap. */
+int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float *U,
+                        const float *W, const int *x0, const float *temp,
+                        const double *u_draft, const int *force_x, int *x_out,
+                        double *pd_out, double *rowmax_out, double *rowsum_out,
+                        double *margin_out)
+{
+    if (B < 0 || G < 1 || V < 2 || r < 1) return ORACLE_ERR_ARG;
+    double *delta = malloc(sizeof(double) * (size_t)V);
+    double *y = malloc(sizeof(double) * (size_t)V);
+    double *e = malloc(sizeof(double) * (size_t)V);
+    if (!delta || !y || !e) { free(delta); free(y); free(e); return ORACLE_ERR_NOMEM; }
+    for (int b = 0; b < B; ++b) {
+        int prev = x0[b];
+        if (prev < 0 || prev >= V) { free(delta); free(y); free(e); return ORACLE_ERR_ARG; }
+        double T = (double)temp[b];
+        for (int i = 0; i < G; ++i) {
+            size_t o = (size_t)b * G + i;
+            markov_bias_row(U, W, V, r, prev, delta);
+            const float *Lrow = L + o * (size_t)V;
+            for (int v = 0; v < V; ++v) y[v] = (double)Lrow[v] + delta[v];
+            int x;
+            if (T == 0.0) {
+                double gap;
+                x = argmax_with_gap(y, V, &gap);
+                margin_out[o] = gap;
+                rowmax_out[o] = y[x];
+                rowsum_out[o] = 1.0;
+                if (force_x && force_x[o] >= 0) x = force_x[o];
+                pd_out[o] = 1.0;
+            } else {
+                double m, Z = softmax_row(y, V, T, e, &m), mg;
+                x = inverse_cdf(e, V, Z, u_draft[o], &mg);
+                margin_out[o] = mg;
+                if (force_x && force_x[o] >= 0) x = force_x[o];
+                rowmax_out[o] = m;
+                rowsum_out[o] = Z;
+                pd_out[o] = e[x] / Z;
+            }
+            x_out[o] = x;
+            prev = x;
+        }
+    }
+    free(delta); free(y); free(e);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stage 2, confidence and prefix survival: [KB] Key Contributions (a
+ * lightweight linear confidence head gives a per-position survival
+ * probability); [PL] §3.2 (the head estimates the conditional survival of
+ * each draft token; sequential temperature scaling calibrates the cumulative
+ * products left to right); [WK] confidence-scheduling section (the survival
+ * of position i is the probability that positions 1..i are all accepted).
+ * c = sigmoid((w . h + bias) / tau_i), S_i = S_{i-1} c_i, S_0 = 1.
+ * h [B][G][d], w [d], tau [G] or NULL (all ones). */
+int dspark_oracle_confidence(int B, int G, int d, const float *h, const float *w,
+                             double bias, const double *tau, double *c_out,
+                             double *S_out)
+{
+    if (B < 0 || G < 1 || d < 1) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        double S = 1.0;
+        for (int i = 0; i < G; ++i) {
+            size_t o = (size_t)b * G + i;
+            const float *hr = h + o * (size_t)d;
+            double a = 0.0;
+            for (int j = 0; j < d; ++j) a += (double)w[j] * (double)hr[j];
+            a += bias;
+            if (tau) a /= tau[i];
+            double c = 1.0 / (1.0 + exp(-a));
+            S *= c;
+            c_out[o] = c;
+            S_out[o] = S;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Throughput profile t(n): piecewise linear through the knots (n_j, t_j),
+ * n_0 = 0, extended past the last knot with the last segment's slope
+ * (constant if there is a single knot).  [PL] §1 and §3.2 (engine-specific
+ * throughput profiles drive the verification length). */
+static double profile_t(int P, const int *kn, const double *kt, double n)
+{
+    if (P == 1) return kt[0];
+    int j = 0;
+    while (j + 1 < P - 1 && n >= (double)kn[j + 1]) ++j;
+    double slope = (kt[j + 1] - kt[j]) / (double)(kn[j + 1] - kn[j]);
+    return kt[j] + (n - (double)kn[j]) * slope;
+}
+
+typedef struct { double s; int idx; } cand_t;
+
+/* S descending; equal S keeps the position-major index order (stable). */
+static int cand_cmp(const void *pa, const void *pb)
+{
+    const cand_t *a = pa, *b = pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    return (a->idx > b->idx) - (a->idx < b->idx);
+}
+
+#define SCHED_ALL 0
+#define SCHED_GREEDY_EARLY_STOP 1
+#define SCHED_GLOBAL_ARGMAX 2 /* offline search of [PL] Appendix A: test-only negative control */
+
+/* Stage 3, Algorithm 1 (hardware-aware prefix scheduler): [KB] Key
+ * Contributions (greedy global sort of candidate tokens by cumulative
+ * survival, incremental batch admission with early stopping that keeps
+ * admissions causal); [PL] Appendix A (stop as soon as Theta_{n+1} < Theta_n;
+ * admitting token k may only use information available before x_k is drawn;
+ * with Theta_0 = 1.0 for one request and nothing admitted).
+ *
+ * S [B][G] survivals.  Candidates are indexed position-major, idx = i*B + b,
+ * and sorted by S descending, ties by idx.  V_0 = B (every request emits at
+ * least one token), Theta_0 = B / t(0); candidate n+1 is admitted unless
+ * (V_n + S_(n+1)) t(n) < V_n t(n+1).  Admission also stops at `budget`
+ * (budget < 0: none) and when every candidate is admitted.
+ * mode ALL: every request gets ell = G.  mode GLOBAL_ARGMAX: the admitted
+ * count maximises Theta over all n (no early stop).  force_n >= 0 replaces
+ * the admitted count (used to follow another implementation after a
+ * near-tie).  Outputs: ell [B], n_adm, theta (objective at the admitted
+ * count), order [B*G] (sorted candidate indices), margin_theta (smallest
+ * relative |Theta_{n+1} - Theta_n| / Theta_n over the comparisons made),
+ * margin_gap (S gap across the cut, +inf if nothing is cut). */
+int dspark_oracle_schedule(int B, int G, const double *S, int P, const int *knots_n,
+                           const double *knots_t, int budget, int mode, int force_n,
+                           int *ell_out, int *n_adm_out, double *theta_out,
+                           int *order_out, double *margin_theta_out,
+                           double *margin_gap_out)
+{
+    if (B < 1 || G < 1 || P < 1 || knots_n[0] != 0) return ORACLE_ERR_ARG;
+    int N = B * G;
+    cand_t *c = malloc(sizeof(cand_t) * (size_t)N);
+    if (!c) return ORACLE_ERR_NOMEM;
+    for (int i = 0; i < G; ++i)
+        for (int b = 0; b < B; ++b) {
+            c[i * B + b].s = S[(size_t)b * G + i];
+            c[i * B + b].idx = i * B + b;
+        }
+    qsort(c, (size_t)N, sizeof(cand_t), cand_cmp);
+    if (order_out)
+        for (int n = 0; n < N; ++n) order_out[n] = c[n].idx;
+
+    int limit = N;
+    if (budget >= 0 && budget < limit) limit = budget;
+    double Vn = (double)B;
+    double theta = Vn / profile_t(P, knots_n, knots_t, 0.0);
+    double mtheta = INFINITY;
+    int n = 0;
+    if (mode == SCHED_ALL) {
+        n = N;
+        for (int k = 0; k < N; ++k) Vn += c[k].s;
+        theta = Vn / profile_t(P, knots_n, knots_t, (double)N);
+    } else if (mode == SCHED_GREEDY_EARLY_STOP) {
+        while (n < limit) {
+            double t0 = profile_t(P, knots_n, knots_t, (double)n);
+            double t1 = profile_t(P, knots_n, knots_t, (double)(n + 1));
+            double Vn1 = Vn + c[n].s;
+            double th1 = Vn1 / t1;
+            double rel = fabs(th1 - theta) / theta;
+            if (rel < mtheta) mtheta = rel;
+            if (Vn1 * t0 < Vn * t1) break; /* Theta_{n+1} < Theta_n: stop */
+            Vn = Vn1;
+            theta = th1;
+            ++n;
+        }
+    } else if (mode == SCHED_GLOBAL_ARGMAX) {
+        double best = theta, run = Vn;
+        int bestn = 0;
+        for (int k = 0; k < limit; ++k) {
+            run += c[k].s;
+            double th = run / profile_t(P, knots_n, knots_t, (double)(k + 1));
+            if (th > best) { best = th; bestn = k + 1; }
+        }
+        n = bestn;
+        theta = best;
+    } else {
+        free(c);
+        return ORACLE_ERR_ARG;
+    }
+    if (force_n >= 0 && force_n <= N) {
+        n = force_n;
+        Vn = (double)B;
+        for (int k = 0; k < n; ++k) Vn += c[k].s;
+        theta = Vn / profile_t(P, knots_n, knots_t, (double)n);
+    }
+    for (int b = 0; b < B; ++b) ell_out[b] = 0;
+    for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;
+    *n_adm_out = n;
+    *theta_out = theta;
+    *margin_theta_out = mtheta;
+    *margin_gap_out = (n > 0 && n < N) ? fabs(c[n - 1].s - c[n].s) : INFINITY;
+    free(c);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Stage 4, exact rejection-sampling verification: [KB] Methodology (x_k is
+ * accepted with probability min(1, p_t(x_k)/p_d(x_k)); the first rejection
+ * discards every later token; the output stays distributed as the target);
+ * [PL] §2 (the longest consistent prefix is kept, verification runs left to
+ * right); [PL] Appendix A (with nothing admitted the target draws a fresh
+ * token from p_t).  On a rejection at k* the replacement is drawn from the
+ * normalised residual max(0, p_t - p_d) at k*; if every admitted token is
+ * accepted a bonus token is drawn from p_t at row ell+1.
+ *
+ * Tlog [B][G+1][V] target logits (row k verifies x_k; row G+1 is the bonus
+ * row), L, U, W, x0 as for drafting, x [B][G] draft tokens, temp [B],
+ * u_accept [B][G], u_final [B], ell [B] admitted counts.  The draft
+ * probabilities are recomputed here from L, U, W and x (fp64), not taken
+ * from the drafting stage.  force_accept (nullable, [B][G]): entries 0/1
+ * replace the accept decision at that position.
+ * Outputs: acc [B] accepted count A, tokens [B][G+1] = x_1..x_A, y, then -1,
+ * nout [B] = A+1, pt_x / pd_x [B][G] = p_t(x_k), p_d(x_k) for k <= ell (NaN
+ * elsewhere; for T = 0 both are 1 when the argmax matches, else 0 / 1),
+ * margin_acc [B][G] (|u - ratio|, or the top-two gap for T = 0; +inf beyond
+ * ell), margin_fin [B], final_kind [B]: 0 residual, 1 bonus/fresh token,
+ * 2 greedy, 3 residual that was all zero (drawn from p_t). */
+int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const float *L,
+                         const float *U, const float *W, const int *x0, const int *x,
+                         const float *temp, const double *u_accept,
+                         const double *u_final, const int *ell,
+                         const int *force_accept, int *acc_out, int *tokens_out,
+                         int *nout_out, double *pt_x_out, double *pd_x_out,
+                         double *margin_acc_out, double *margin_fin_out,
+                         int *final_kind_out)
+{
+    if (B < 0 || G < 1 || V < 2 || r < 1) return ORACLE_ERR_ARG;
+    double *delta = malloc(sizeof(double) * (size_t)V);
+    double *yd = malloc(sizeof(double) * (size_t)V);
+    double *yt = malloc(sizeof(double) * (size_t)V);
+    double *ed = malloc(sizeof(double) * (size_t)V);
+    double *et = malloc(sizeof(double) * (size_t)V);
+    double *q = malloc(sizeof(double) * (size_t)V);
+    if (!delta || !yd || !yt || !ed || !et || !q) {
+        free(delta); free(yd); free(yt); free(ed); free(et); free(q);
+        return ORACLE_ERR_NOMEM;
+    }
+    int rc = ORACLE_OK;
+    for (int b = 0; b < B && rc == ORACLE_OK; ++b) {
+        double T = (double)temp[b];
+        int lb = ell[b];
+        if (lb < 0 || lb > G) { rc = ORACLE_ERR_ARG; break; }
+        for (int k = 0; k < G; ++k) {
+            size_t o = (size_t)b * G + k;
+            pt_x_out[o] = NAN;
+            pd_x_out[o] = NAN;
+            margin_acc_out[o] = INFINITY;
+        }
+        /* Per admitted position: target and draft probability of x_k. */
+        int A = 0, rejected = 0;
+        for (int k = 1; k <= lb; ++k) {
+            size_t o = (size_t)b * G + (k - 1);
+            int xk = x[o];
+            int prev = (k == 1) ? x0[b] : x[o - 1];
+            const float *Trow = Tlog + ((size_t)b * (G + 1) + (k - 1)) * (size_t)V;
+            for (int v = 0; v < V; ++v) yt[v] = (double)Trow[v];
+            int accept;
+            if (T == 0.0) {
+                double gap;
+                int am = argmax_with_gap(yt, V, &gap);
+                accept = (am == xk);
+                /* The decision flips only if x_k and the argmax swap: margin is
+                 * the distance between z[x_k] and the best other entry. */
+                double best_other = -INFINITY;
+                for (int v = 0; v < V; ++v)
+                    if (v != xk && yt[v] > best_other) best_other = yt[v];
+                margin_acc_out[o] = fabs(yt[xk] - best_other);
+                pt_x_out[o] = accept ? 1.0 : 0.0;
+                pd_x_out[o] = 1.0;
+            } else {
+                double mt, Zt = softmax_row(yt, V, T, et, &mt);
+                markov_bias_row(U, W, V, r, prev, delta);
+                const float *Lrow = L + o * (size_t)V;
+                for (int v = 0; v < V; ++v) yd[v] = (double)Lrow[v] + delta[v];
+                double md, Zd = softmax_row(yd, V, T, ed, &md);
+                double pt = et[xk] / Zt, pd = ed[xk] / Zd;
+                double ratio = pt / pd;
+                accept = u_accept[o] < ratio;
+                margin_acc_out[o] = fabs(u_accept[o] - ratio);
+                pt_x_out[o] = pt;
+                pd_x_out[o] = pd;
+            }
+            if (force_accept && force_accept[o] >= 0) accept = force_accept[o] ? 1 : 0;
+            if (!rejected) {
+                if (accept) ++A;
+                else rejected = 1;
+            }
+        }
+        /* Final token from row k* = A + 1 (1-based). */
+        int ks = A + 1;
+        const float *Trow = Tlog + ((size_t)b * (G + 1) + (ks - 1)) * (size_t)V;
+        for (int v = 0; v < V; ++v) yt[v] = (double)Trow[v];
+        int yv, kind;
+        double mfin;
+        if (T == 0.0) {
+            yv = argmax_with_gap(yt, V, &mfin);
+            kind = 2;
+        } else {
+            double mt, Zt = softmax_row(yt, V, T, et, &mt);
+            if (A < lb) {
+                size_t o = (size_t)b * G + (ks - 1);
+                int prev = (ks == 1) ? x0[b] : x[o - 1];
+                markov_bias_row(U, W, V, r, prev, delta);
+                const float *Lrow = L + o * (size_t)V;
+                for (int v = 0; v < V; ++v) yd[v] = (double)Lrow[v] + delta[v];
+                double md, Zd = softmax_row(yd, V, T, ed, &md);
+                double Q = 0.0;
+                for (int v = 0; v < V; ++v) {
+                    double d = et[v] / Zt - ed[v] / Zd;
+                    q[v] = d > 0.0 ? d : 0.0;
+                    Q += q[v];
+                }
+                if (Q > 0.0) {
+                    yv = inverse_cdf(q, V, Q, u_final[b], &mfin);
+                    kind = 0;
+                } else {
+                    yv = inverse_cdf(et, V, Zt, u_final[b], &mfin);
+                    kind = 3;
+                }
+            } else {
+                yv = inverse_cdf(et, V, Zt, u_final[b], &mfin);
+                kind = 1;
+            }
+        }
+        int *tok = tokens_out + (size_t)b * (G + 1);
+        for (int j = 0; j < G + 1; ++j) tok[j] = -1;
+        for (int j = 0; j < A; ++j) tok[j] = x[(size_t)b * G + j];
+        tok[A] = yv;
+        acc_out[b] = A;
+        nout_out[b] = A + 1;
+        margin_fin_out[b] = mfin;
+        final_kind_out[b] = kind;
+    }
+    free(delta); free(yd); free(yt); free(ed); free(et); free(q);
+    return rc;
+}

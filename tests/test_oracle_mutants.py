@@ -1,0 +1,72 @@
+"""The pins must catch plausible mistakes.  Each case compiles a copy of the
+oracle with one planted error (on the CPU, in a temporary directory) and
+checks that at least one pin fails against it; the real oracle is restored
+afterwards."""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import enum_harness as eh
+from oracle import oracle
+
+# (name, exact source fragment, planted replacement)
+MUTANTS = [
+    ("residual_sign", "double d = et[v] / Zt - ed[v] / Zd;", "double d = ed[v] / Zd - et[v] / Zt;"),
+    ("ratio_inverted", "double ratio = pt / pd;", "double ratio = pd / pt;"),
+    ("verify_conditions_on_current_token",
+     "int prev = (k == 1) ? x0[b] : x[o - 1];\n            const float *Trow",
+     "int prev = x[o];\n            const float *Trow"),
+    ("draft_ignores_previous_token", "            x_out[o] = x;\n            prev = x;",
+     "            x_out[o] = x;"),
+    ("bonus_from_last_admitted_row", "int ks = A + 1;", "int ks = (A == lb && A > 0) ? A : A + 1;"),
+    ("residual_without_clamp", "q[v] = d > 0.0 ? d : 0.0;", "q[v] = d > 0.0 ? d : -d;"),
+    ("target_row_shifted", "const float *Trow = Tlog + ((size_t)b * (G + 1) + (k - 1)) * (size_t)V;",
+     "const float *Trow = Tlog + ((size_t)b * (G + 1) + k) * (size_t)V;"),
+]
+
+
+def _build_mutant(tmp_path, name, old, new):
+    src = open(oracle.source_path()).read()
+    assert src.count(old) == 1, name
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / f"lib{name}.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-o",
+                    str(so), str(path), "-lm"], check=True)
+    return str(so)
+
+
+def _preservation_probe():
+    """Worst preservation error over a few exact-enumeration scenarios."""
+    worst = 0.0
+    for seed, (V, G, r, T) in enumerate([(3, 3, 2, 1.0), (4, 2, 2, float(np.float32(0.7)))]):
+        rng = np.random.default_rng(100 + seed)
+        Lrows = rng.normal(0, 1.5, (G, V)).astype(np.float32)
+        U = rng.normal(0, 1.0, (V, r)).astype(np.float32)
+        W = rng.normal(0, 1.0, (r, V)).astype(np.float32)
+        target = eh.random_target(rng, V, G)
+        for ell in range(G + 1):
+            sc = eh.Scenario(Lrows, U, W, int(rng.integers(0, V)), T, target, ell_fixed=ell)
+            try:
+                law = sc.output_law()
+            except Exception:
+                return np.inf
+            worst = max(worst, eh.preservation_error(law, target, T, V))
+    return worst
+
+
+def test_real_oracle_passes_probe():
+    oracle.use_library(oracle.build())
+    assert _preservation_probe() < 1e-12
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, name, old, new)
+    try:
+        oracle.use_library(so)
+        assert _preservation_probe() > 1e-6
+    finally:
+        oracle.use_library(oracle.build())

@@ -1,0 +1,192 @@
+/*
+ * dspark.h -- C ABI of the DSpark per-round token path on B200 (sm_100a).
+ *
+ * One speculative-decoding round for a batch of B requests with draft block
+ * size G over a V-token vocabulary, in four calls:
+ *   dspark_draft_markov  semi-autoregressive drafting with the Markov head
+ *   dspark_confidence    linear confidence head and prefix survival
+ *   dspark_schedule      Algorithm-1 hardware-aware prefix scheduler
+ *   dspark_verify        exact rejection-sampling verification
+ *
+ * Sources (web pages about arXiv:2607.05147, "DSpark: Confidence-Scheduled
+ * Speculative Decoding with Semi-Autoregressive Generation"), cited by tag:
+ *   [PL] paperlayer.ai section-by-section summary (§2 Background, §3.1
+ *        Semi-autoregressive generation, §3.2 Confidence-scheduled
+ *        verification, Appendix A counterexample);
+ *   [KB] menfem.com knowledge-base entry ("Key Contributions",
+ *        "Methodology");
+ *   [WK] llm-wiki.hwlabs.dev study 116 (draft-generation figure of the
+ *        Markov-head section; confidence-scheduling section).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every array pointer is a DEVICE pointer owned by the caller; the library
+ *   keeps no pointer past the call's return, never allocates device or host
+ *   memory, and never synchronises (except dspark_get_device_status).  Work
+ *   is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *   stream), so every call may be captured in a CUDA graph.
+ * - Arrays are dense, row-major, with the shapes given; "dtype" arrays hold
+ *   DSPARK_F32 (fp32) or DSPARK_BF16 (bf16 bit patterns) elements.
+ * - Host-detectable errors (bad sizes, null pointers, short workspace, CUDA
+ *   launch failures) return a non-zero dspark_status before or instead of
+ *   enqueuing work.  Data errors that only the device can see (a token id
+ *   outside [0, V), an admitted length outside [0, G], a negative or NaN
+ *   temperature) are clamped to the valid range and recorded as bits of a
+ *   status word at the start of the caller's workspace; read them with
+ *   dspark_get_device_status.  No call traps, asserts or spins unbounded on
+ *   the device.
+ * - A workspace is caller-allocated device memory of at least the size the
+ *   matching *_workspace_size query returns, aligned to 256 bytes.  One
+ *   buffer of the largest size may serve every call of a round.  Workspace
+ *   contents need no initialisation except the status word (see
+ *   dspark_clear_device_status); calls that share a workspace must not run
+ *   concurrently.
+ * - Limits checked on the host: 1 <= B <= 4096, 1 <= G <= 16,
+ *   2 <= V <= 2^20, 1 <= r <= 512 (a multiple of 16 for bf16), 1 <= d <= 65536,
+ *   B*G <= 16384 for the scheduler, 1 <= P <= 64 profile knots.
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSPARK_OK = 0,
+    DSPARK_ERR_INVALID_ARG = 1,      /* a size, pointer, mode or dtype is out of range */
+    DSPARK_ERR_UNSUPPORTED_DTYPE = 2,
+    DSPARK_ERR_WORKSPACE = 3,        /* workspace missing, short or misaligned */
+    DSPARK_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed */
+    DSPARK_ERR_TIMEOUT = 5           /* a bounded device wait gave up */
+} dspark_status;
+
+typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
+
+typedef enum {
+    DSPARK_SCHED_ALL = 0,               /* verify every drafted position */
+    DSPARK_SCHED_GREEDY_EARLY_STOP = 1  /* Algorithm 1 */
+} dspark_sched_mode;
+
+/* Bits of the device status word. */
+#define DSPARK_DEV_TOKEN_RANGE 0x1u  /* a token id outside [0, V) was clamped */
+#define DSPARK_DEV_ELL_RANGE 0x2u    /* an admitted length outside [0, G] was clamped */
+#define DSPARK_DEV_BAD_TEMP 0x4u     /* a temperature < 0 or NaN was treated as 0 */
+#define DSPARK_DEV_TIMEOUT 0x8u      /* a bounded device wait ran out */
+
+/* Library version and the build's target (a string such as "sm_100a"). */
+const char *dspark_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 1: semi-autoregressive drafting with the Markov head.
+ * [PL] §3.1: the parallel backbone gives all G draft logit rows in one pass;
+ * a lightweight sequential module then samples left to right, each position
+ * conditioned on the previously sampled token through a low-rank transition
+ * matrix.  [KB] Methodology: rank-256 factorisation.  [WK] draft-generation
+ * figure: final logits L[i] + Delta[i], then the draft token is sampled.
+ *
+ * For i = 1..G in order (x_0 = x0[b], the last committed token):
+ *   y = L[b,i,:] + Delta_i[b,:],  Delta_i[b,v] = sum_k U[x_{i-1},k] * Wt[v,k]
+ *   z = y / T_b,  m = max z,  Z = sum_v exp(z_v - m)
+ *   x_i = smallest v with u_draft[b,i] < sum_{j<=v} exp(z_j - m) / Z
+ *   (T_b = 0: x_i = argmax y, lowest index on ties).
+ * Inputs:  L [B,G,V] dtype, U [V,r] dtype, Wt [V,r] dtype (the transition
+ *          factor W stored transposed: row v is column v of W), x0 [B] int32,
+ *          temp [B] f32 (>= 0), u_draft [B,G] f32 in [0,1).
+ * Outputs: x_out [B,G] int32; pd_x_out [B,G] f32 = p_d(x_i) (1 for T = 0);
+ *          rowmax_out [B,G] f32 = max_v y_v (before the temperature);
+ *          rowsum_out [B,G] f32 = Z (1 for T = 0).
+ * rowmax/rowsum are what dspark_verify needs to rebuild p_d at a rejection. */
+size_t dspark_draft_workspace_size(int B, int G, int V, int r, int dtype);
+dspark_status dspark_draft_markov(const void *L, const void *U, const void *Wt,
+                                  const int32_t *x0, const float *temp,
+                                  const float *u_draft, int B, int G, int V, int r,
+                                  int dtype, void *ws, size_t ws_bytes, int32_t *x_out,
+                                  float *pd_x_out, float *rowmax_out, float *rowsum_out,
+                                  void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 2: confidence head and prefix survival.
+ * [KB] Key Contributions: a lightweight linear confidence head emits a
+ * per-position survival probability.  [PL] §3.2: it estimates each draft
+ * token's conditional survival; cumulative products give prefix survival,
+ * calibrated left to right by sequential temperature scaling.
+ *   c[b,i] = sigmoid((w . h[b,i,:] + bias) / tau[i]),  S[b,i] = prod_{j<=i} c[b,j].
+ * Inputs:  h [B,G,d] dtype, w [d] dtype, bias, tau [G] f32 or NULL (all 1).
+ * Outputs: c_out [B,G] f32, S_out [B,G] f32 (non-increasing along i).
+ * Needs no workspace. */
+dspark_status dspark_confidence(const void *h, const void *w, float bias, const float *tau,
+                                int B, int G, int d, int dtype, float *c_out, float *S_out,
+                                void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 3: Algorithm 1, the hardware-aware prefix scheduler.
+ * [KB] Key Contributions: greedy global sort of candidate tokens by
+ * cumulative survival, incremental batch admission with early stopping that
+ * keeps admissions causal.  [PL] Appendix A: stop as soon as the objective
+ * drops (Theta_{n+1} < Theta_n); admitting token k may use only information
+ * available before x_k is sampled.
+ *   Candidates (b, i) are laid out position-major (idx = i*B + b) and sorted
+ *   by S descending, ties by idx, so every request's admitted set is a prefix.
+ *   V_0 = B, Theta_n = V_n / t(n); candidate n+1 is admitted unless
+ *   (V_n + S_(n+1)) * t(n) < V_n * t(n+1) (evaluated in fp64); admission
+ *   also ends at `budget` (< 0: none) or when all B*G are admitted.
+ *   t(n) is piecewise linear through the P knots (knots_n[j], knots_t[j]),
+ *   knots_n[0] = 0 and strictly increasing, continued past the last knot
+ *   with the last segment's slope (constant when P = 1); knots_t > 0.
+ * Inputs:  S [B,G] f32, knots_n [P] int32, knots_t [P] f64 (device arrays),
+ *          budget, mode (dspark_sched_mode).
+ * Outputs: ell_out [B] int32 admitted prefix length per request;
+ *          n_adm_out [1] int32; theta_out [1] f64 = Theta at n_adm;
+ *          order_out [B*G] int32 sorted candidate indices, or NULL. */
+size_t dspark_schedule_workspace_size(int B, int G);
+dspark_status dspark_schedule(const float *S, int B, int G, const int32_t *knots_n,
+                              const double *knots_t, int P, int budget, int mode, void *ws,
+                              size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out,
+                              double *theta_out, int32_t *order_out, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 4: exact rejection-sampling verification.
+ * [KB] Methodology: x_k is accepted with probability min(1, p_t(x_k) /
+ * p_d(x_k)); the first rejection discards every later token.  [PL] §2:
+ * verification runs left to right and keeps the longest consistent prefix.
+ * [PL] Appendix A: with nothing admitted the target draws a fresh token.
+ *   p_t = softmax(Tlog[b,k,:] / T_b).  For k = 1..ell_b: accept x_k iff
+ *   u_accept[b,k] < p_t(x_k) / pd_x[b,k]; A_b = leading accepts.
+ *   If A_b < ell_b: y ~ normalised max(0, p_t - p_d) at k* = A_b + 1, with
+ *   p_d rebuilt from L, U, Wt, rowmax, rowsum (an all-zero residual falls
+ *   back to p_t).  Else y ~ p_t at row ell_b + 1 (the bonus token).  Draws
+ *   are inverse-CDF with u_final[b].  T_b = 0: accept iff argmax Tlog[b,k]
+ *   = x_k, and y = argmax Tlog[b, A_b + 1].
+ * Inputs:  Tlog [B,G+1,V] dtype (row k verifies x_k; row G+1 is the bonus
+ *          row), L, U, Wt, x0 as for drafting, x/pd_x/rowmax/rowsum from
+ *          dspark_draft_markov, temp [B], u_accept [B,G], u_final [B] f32,
+ *          ell [B] int32 from dspark_schedule.
+ * Outputs: acc_out [B] int32 = A_b; tokens_out [B,G+1] int32 = x_1..x_A, y,
+ *          then -1; nout_out [B] int32 = A_b + 1; pt_x_out [B,G] f32 =
+ *          p_t(x_k) for k <= ell_b (1/0 for T = 0, match/no match; -1
+ *          elsewhere), or NULL. */
+size_t dspark_verify_workspace_size(int B, int G, int V, int r, int dtype);
+dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, const void *Wt,
+                            const int32_t *x0, const int32_t *x, const float *pd_x,
+                            const float *rowmax, const float *rowsum, const float *temp,
+                            const float *u_accept, const float *u_final, const int32_t *ell,
+                            int B, int G, int V, int r, int dtype, void *ws, size_t ws_bytes,
+                            int32_t *acc_out, int32_t *tokens_out, int32_t *nout_out,
+                            float *pt_x_out, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Device status word of a workspace: dspark_get_device_status synchronises
+ * `stream`, then copies the word to *status_out (0 = no data error since the
+ * last clear).  dspark_clear_device_status enqueues a reset of the word. */
+dspark_status dspark_get_device_status(const void *ws, void *stream, uint32_t *status_out);
+dspark_status dspark_clear_device_status(void *ws, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H */

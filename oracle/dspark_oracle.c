@@ -125,9 +125,10 @@ static double softmax_row(const double *row, int V, double T, double *e, double 
  * temp [B]; u_draft [B][G] uniforms in [0,1).  force_x (nullable, [B][G]):
  * entries >= 0 replace the sampled token (used to follow another
  * implementation's decision after a reported near-tie).
- * Outputs per (b,i): x, pd = p_d(x), rowmax = max_v z_v, rowsum = sum exp(z-m),
- * margin = decision margin.  For T = 0: x = argmax (L + Delta), pd = 1,
- * rowmax = max (L + Delta), rowsum = 1, margin = top-two gap. */
+ * Outputs per (b,i), with y = L + Delta and z = y / T: x, pd = p_d(x),
+ * rowmax = max_v y_v (logit units, before the temperature), rowsum =
+ * sum_v exp(z_v - max z), margin = decision margin.  For T = 0: x = argmax y,
+ * pd = 1, rowmax = max y, rowsum = 1, margin = top-two gap. */
 int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float *U,
                         const float *W, const int *x0, const float *temp,
                         const double *u_draft, const int *force_x, int *x_out,
@@ -162,7 +163,10 @@ int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float 
                 x = inverse_cdf(e, V, Z, u_draft[o], &mg);
                 margin_out[o] = mg;
                 if (force_x && force_x[o] >= 0) x = force_x[o];
-                rowmax_out[o] = m;
+                double ymax = y[0];
+                for (int v = 1; v < V; ++v)
+                    if (y[v] > ymax) ymax = y[v];
+                rowmax_out[o] = ymax;
                 rowsum_out[o] = Z;
                 pd_out[o] = e[x] / Z;
             }

@@ -86,8 +86,8 @@ def _check(rc, name):
 class DraftResult:
     x: np.ndarray        # [B, G] int32
     pd: np.ndarray       # [B, G] p_d(x)
-    rowmax: np.ndarray   # [B, G] max_v z_v
-    rowsum: np.ndarray   # [B, G] sum_v exp(z_v - max)
+    rowmax: np.ndarray   # [B, G] max_v (L + Delta)_v, before the temperature
+    rowsum: np.ndarray   # [B, G] sum_v exp(z_v - max z), z = (L + Delta) / T
     margin: np.ndarray   # [B, G] decision margin
 
 

@@ -1,0 +1,159 @@
+"""ctypes binding of libdspark (the C ABI declared in include/dspark.h).
+
+Argument marshalling only: torch tensors supply device pointers and sizes,
+torch streams supply the cudaStream_t.  Every step of the round runs in the
+library's CUDA kernels; there is no fallback.  Importing this module on a
+machine without the built library, or calling it without a CUDA device,
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdspark.so")
+
+DSPARK_F32 = 0
+DSPARK_BF16 = 1
+SCHED_ALL = 0
+SCHED_GREEDY_EARLY_STOP = 1
+
+STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DTYPE", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
+DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov", "dspark_confidence",
+           "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
+           "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status")
+
+
+class DsparkError(RuntimeError):
+    def __init__(self, fn, status):
+        super().__init__(f"{fn} returned {status} ({STATUS.get(status, '?')})")
+        self.status = status
+
+
+_lib = None
+_vp, _i, _f, _sz, _d = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_double
+
+
+def load() -> ctypes.CDLL:
+    """Load libdspark.so from the package directory (build it first with
+    ``python -m speculative_decoding_draft_rank_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libdspark.so is not built ({LIB_PATH}); run the package build step")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.dspark_version.restype = ctypes.c_char_p
+    lib.dspark_draft_workspace_size.restype = _sz
+    lib.dspark_draft_workspace_size.argtypes = [_i] * 5
+    lib.dspark_draft_markov.restype = _i
+    lib.dspark_draft_markov.argtypes = [_vp] * 6 + [_i] * 5 + [_vp, _sz] + [_vp] * 5
+    lib.dspark_confidence.restype = _i
+    lib.dspark_confidence.argtypes = [_vp, _vp, _f, _vp, _i, _i, _i, _i, _vp, _vp, _vp]
+    lib.dspark_schedule_workspace_size.restype = _sz
+    lib.dspark_schedule_workspace_size.argtypes = [_i, _i]
+    lib.dspark_schedule.restype = _i
+    lib.dspark_schedule.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _sz, _vp, _vp, _vp, _vp, _vp]
+    lib.dspark_verify_workspace_size.restype = _sz
+    lib.dspark_verify_workspace_size.argtypes = [_i] * 5
+    lib.dspark_verify.restype = _i
+    lib.dspark_verify.argtypes = [_vp] * 13 + [_i] * 5 + [_vp, _sz] + [_vp] * 5
+    lib.dspark_get_device_status.restype = _i
+    lib.dspark_get_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.dspark_clear_device_status.restype = _i
+    lib.dspark_clear_device_status.argtypes = [_vp, _vp]
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libdspark takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libdspark takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t):
+    if t.dtype == torch.bfloat16:
+        return DSPARK_BF16
+    if t.dtype == torch.float32:
+        return DSPARK_F32
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _call(fn, *args):
+    st = getattr(load(), fn)(*args)
+    if st != 0:
+        raise DsparkError(fn, st)
+
+
+def version() -> str:
+    return load().dspark_version().decode()
+
+
+def dspark_draft_workspace_size(B, G, V, r, dtype) -> int:
+    return int(load().dspark_draft_workspace_size(B, G, V, r, dtype))
+
+
+def dspark_schedule_workspace_size(B, G) -> int:
+    return int(load().dspark_schedule_workspace_size(B, G))
+
+
+def dspark_verify_workspace_size(B, G, V, r, dtype) -> int:
+    return int(load().dspark_verify_workspace_size(B, G, V, r, dtype))
+
+
+def dspark_draft_markov(L, U, Wt, x0, temp, u_draft, ws, x_out, pd_x_out, rowmax_out, rowsum_out,
+                        stream=None):
+    B, G, V = L.shape
+    r = U.shape[1]
+    _call("dspark_draft_markov", _ptr(L), _ptr(U), _ptr(Wt), _ptr(x0), _ptr(temp), _ptr(u_draft), B, G, V,
+          r, _dtype(L), _ptr(ws), ws.numel() * ws.element_size(), _ptr(x_out), _ptr(pd_x_out),
+          _ptr(rowmax_out), _ptr(rowsum_out), _stream(stream))
+
+
+def dspark_confidence(h, w, bias, tau, c_out, S_out, stream=None):
+    B, G, d = h.shape
+    _call("dspark_confidence", _ptr(h), _ptr(w), ctypes.c_float(bias), _ptr(tau), B, G, d, _dtype(h),
+          _ptr(c_out), _ptr(S_out), _stream(stream))
+
+
+def dspark_schedule(S, knots_n, knots_t, budget, mode, ws, ell_out, n_adm_out, theta_out, order_out=None,
+                    stream=None):
+    B, G = S.shape
+    _call("dspark_schedule", _ptr(S), B, G, _ptr(knots_n), _ptr(knots_t), knots_n.numel(), int(budget),
+          int(mode), _ptr(ws), ws.numel() * ws.element_size(), _ptr(ell_out), _ptr(n_adm_out),
+          _ptr(theta_out), _ptr(order_out), _stream(stream))
+
+
+def dspark_verify(Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell, ws, acc_out,
+                  tokens_out, nout_out, pt_x_out=None, stream=None):
+    B, G1, V = Tlog.shape
+    r = U.shape[1]
+    _call("dspark_verify", _ptr(Tlog), _ptr(L), _ptr(U), _ptr(Wt), _ptr(x0), _ptr(x), _ptr(pd_x),
+          _ptr(rowmax), _ptr(rowsum), _ptr(temp), _ptr(u_accept), _ptr(u_final), _ptr(ell), B, G1 - 1, V, r,
+          _dtype(Tlog), _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out), _ptr(tokens_out),
+          _ptr(nout_out), _ptr(pt_x_out), _stream(stream))
+
+
+def dspark_get_device_status(ws, stream=None) -> int:
+    out = ctypes.c_uint32(0)
+    _call("dspark_get_device_status", _ptr(ws), _stream(stream), ctypes.byref(out))
+    return int(out.value)
+
+
+def dspark_clear_device_status(ws, stream=None):
+    _call("dspark_clear_device_status", _ptr(ws), _stream(stream))

@@ -1,0 +1,134 @@
+// abi.cu -- the extern "C" entry points of libdspark: host-side argument
+// checks, workspace checks, then the stage launchers.  Nothing here
+// allocates memory or synchronises, except dspark_get_device_status.
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+using namespace dspark;
+
+namespace {
+
+bool dtype_ok(int dt) { return dt == DSPARK_F32 || dt == DSPARK_BF16; }
+bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+
+dspark_status check_common(int B, int G, int V, int r, int dtype) {
+    if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || V < 2 || V > (1 << 20) || r < 1 || r > 512)
+        return DSPARK_ERR_INVALID_ARG;
+    if (dtype == DSPARK_BF16 && (r % 16) != 0) return DSPARK_ERR_INVALID_ARG;
+    return DSPARK_OK;
+}
+
+dspark_status check_ws(const void *ws, size_t have, size_t need) {
+    if (ws == nullptr || !aligned256(ws) || have < need) return DSPARK_ERR_WORKSPACE;
+    return DSPARK_OK;
+}
+
+// Host-side fault injection for failure-path tests: DSPARK_INJECT_ERROR=<entry
+// point name>=<status> makes that entry point return <status> without
+// enqueuing work.
+dspark_status injected(const char *name) {
+    const char *env = getenv("DSPARK_INJECT_ERROR");
+    if (env == nullptr) return DSPARK_OK;
+    const size_t n = strlen(name);
+    if (strncmp(env, name, n) == 0 && env[n] == '=') return (dspark_status)atoi(env + n + 1);
+    return DSPARK_OK;
+}
+
+dspark_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *dspark_version(void) { return "dspark-b200 0.1 (sm_100a)"; }
+
+size_t dspark_draft_workspace_size(int B, int G, int V, int r, int dtype) {
+    if (check_common(B, G, V, r, dtype) != DSPARK_OK) return 0;
+    return draft_ws_bytes(B, G, V, r, dtype);
+}
+
+dspark_status dspark_draft_markov(const void *L, const void *U, const void *Wt, const int32_t *x0,
+                                  const float *temp, const float *u_draft, int B, int G, int V, int r,
+                                  int dtype, void *ws, size_t ws_bytes, int32_t *x_out,
+                                  float *pd_x_out, float *rowmax_out, float *rowsum_out,
+                                  void *stream) {
+    if (dspark_status s = injected("dspark_draft_markov")) return s;
+    if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
+    if (!L || !U || !Wt || !x0 || !temp || !u_draft || !x_out || !pd_x_out || !rowmax_out || !rowsum_out)
+        return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, draft_ws_bytes(B, G, V, r, dtype))) return s;
+    DraftArgs a{L, U, Wt, x0, temp, u_draft, B, G, V, r, dtype, x_out, pd_x_out, rowmax_out, rowsum_out};
+    return cuda_status(launch_draft(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_confidence(const void *h, const void *w, float bias, const float *tau, int B,
+                                int G, int d, int dtype, float *c_out, float *S_out, void *stream) {
+    if (dspark_status s = injected("dspark_confidence")) return s;
+    if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || d < 1 || d > 65536) return DSPARK_ERR_INVALID_ARG;
+    if (!h || !w || !c_out || !S_out) return DSPARK_ERR_INVALID_ARG;
+    return cuda_status(launch_confidence(h, w, bias, tau, B, G, d, dtype, c_out, S_out,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t dspark_schedule_workspace_size(int B, int G) {
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || B * G > 16384) return 0;
+    return schedule_ws_bytes(B, G);
+}
+
+dspark_status dspark_schedule(const float *S, int B, int G, const int32_t *knots_n,
+                              const double *knots_t, int P, int budget, int mode, void *ws,
+                              size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
+                              int32_t *order_out, void *stream) {
+    if (dspark_status s = injected("dspark_schedule")) return s;
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || B * G > 16384 || P < 1 || P > 64)
+        return DSPARK_ERR_INVALID_ARG;
+    if (mode != DSPARK_SCHED_ALL && mode != DSPARK_SCHED_GREEDY_EARLY_STOP) return DSPARK_ERR_INVALID_ARG;
+    if (!S || !knots_n || !knots_t || !ell_out || !n_adm_out || !theta_out) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, schedule_ws_bytes(B, G))) return s;
+    return cuda_status(launch_schedule(S, B, G, knots_n, knots_t, P, budget, mode, ws, ell_out, n_adm_out,
+                                       theta_out, order_out, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dspark_verify_workspace_size(int B, int G, int V, int r, int dtype) {
+    if (check_common(B, G, V, r, dtype) != DSPARK_OK) return 0;
+    return verify_ws_bytes(B, G, V, r, dtype);
+}
+
+dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, const void *Wt,
+                            const int32_t *x0, const int32_t *x, const float *pd_x,
+                            const float *rowmax, const float *rowsum, const float *temp,
+                            const float *u_accept, const float *u_final, const int32_t *ell, int B,
+                            int G, int V, int r, int dtype, void *ws, size_t ws_bytes,
+                            int32_t *acc_out, int32_t *tokens_out, int32_t *nout_out,
+                            float *pt_x_out, void *stream) {
+    if (dspark_status s = injected("dspark_verify")) return s;
+    if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
+    if (!Tlog || !L || !U || !Wt || !x0 || !x || !pd_x || !rowmax || !rowsum || !temp || !u_accept ||
+        !u_final || !ell || !acc_out || !tokens_out || !nout_out)
+        return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, verify_ws_bytes(B, G, V, r, dtype))) return s;
+    VerifyArgs a{Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell,
+                 B, G, V, r, dtype, acc_out, tokens_out, nout_out, pt_x_out};
+    return cuda_status(launch_verify(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_get_device_status(const void *ws, void *stream, uint32_t *status_out) {
+    if (!ws || !status_out) return DSPARK_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSPARK_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return DSPARK_ERR_CUDA;
+    *status_out = v;
+    return DSPARK_OK;
+}
+
+dspark_status dspark_clear_device_status(void *ws, void *stream) {
+    if (!ws) return DSPARK_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

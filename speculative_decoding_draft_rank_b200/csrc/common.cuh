@@ -1,0 +1,185 @@
+// common.cuh -- shared device helpers of the DSpark round kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+constexpr int kWarp = 32;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Workspace header: the first 256 bytes of every workspace hold the device
+// status word (bit set by kernels that clamp bad data) and spare counters.
+struct WsHeader {
+    uint32_t status;
+    uint32_t pad[63];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+__device__ __forceinline__ void flag_status(WsHeader *h, uint32_t bit) {
+    atomicOr(&h->status, bit);
+}
+
+// Element loads: fp32 or bf16 widened exactly to fp32.
+__device__ __forceinline__ float ld_elem(const float *p, size_t i) { return __ldg(p + i); }
+__device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Streaming (read-once) 16-byte load that does not allocate in L1.
+__device__ __forceinline__ uint4 ld_stream16(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+// exp(x) through the hardware base-2 exponential.
+__device__ __forceinline__ float exp_e(float x) { return fast_exp2(x * kLog2e); }
+
+// ---------------------------------------------------------------------------
+// Warp reductions and scans.
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+__device__ __forceinline__ int warp_min_i(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+// (value, index) max with the lower index winning ties.
+__device__ __forceinline__ void warp_argmax(float &v, int &i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, v, o);
+        int oi = __shfl_xor_sync(0xffffffffu, i, o);
+        if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+    }
+}
+// Inclusive prefix sum across the warp (lane order).
+__device__ __forceinline__ float warp_incl_scan(float v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+__device__ __forceinline__ double warp_incl_scan_d(double v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        double n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+__device__ __forceinline__ int warp_incl_scan_i(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    return v;
+}
+
+// Block-wide inclusive scan of one float per thread (blockDim a multiple of
+// 32, at most 1024).  `smem` holds >= 33 floats.  Returns the inclusive
+// prefix; *total receives the block sum.
+__device__ __forceinline__ float block_incl_scan(float v, float *smem, float *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    float s = warp_incl_scan(v);
+    if (lane == 31) smem[wid] = s;
+    __syncthreads();
+    if (wid == 0) {
+        float t = lane < nw ? smem[lane] : 0.f;
+        t = warp_incl_scan(t);
+        if (lane < nw) smem[lane] = t;
+        if (lane == nw - 1) smem[32] = t;
+    }
+    __syncthreads();
+    float r = s + (wid > 0 ? smem[wid - 1] : 0.f);
+    *total = smem[32];
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float *smem) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_max(v);
+    if (lane == 0) smem[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        float t = lane < nw ? smem[lane] : -INFINITY;
+        t = warp_max(t);
+        if (lane == 0) smem[32] = t;
+    }
+    __syncthreads();
+    float r = smem[32];
+    __syncthreads();
+    return r;
+}
+
+__device__ __forceinline__ int block_min_i(int v, int *smem) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_min_i(v);
+    if (lane == 0) smem[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        int t = lane < nw ? smem[lane] : 0x7fffffff;
+        t = warp_min_i(t);
+        if (lane == 0) smem[32] = t;
+    }
+    __syncthreads();
+    int r = smem[32];
+    __syncthreads();
+    return r;
+}
+
+// Clamp a token id to [0, V), flagging the status word when it was outside.
+__device__ __forceinline__ int clamp_token(int t, int V, WsHeader *h) {
+    if (t < 0 || t >= V) {
+        flag_status(h, DSPARK_DEV_TOKEN_RANGE);
+        t = t < 0 ? 0 : V - 1;
+    }
+    return t;
+}
+// Temperatures: negative or NaN -> 0 (greedy), flagged.
+__device__ __forceinline__ float sane_temp(float T, WsHeader *h) {
+    if (!(T >= 0.f)) {
+        flag_status(h, DSPARK_DEV_BAD_TEMP);
+        T = 0.f;
+    }
+    return T;
+}
+
+}  // namespace dspark

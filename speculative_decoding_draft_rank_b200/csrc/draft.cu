@@ -1,0 +1,355 @@
+// draft.cu -- stage 1, semi-autoregressive drafting with the Markov head.
+//
+// Method (paperlayer.ai summary of DSpark, §3.1 Semi-autoregressive
+// generation; llm-wiki.hwlabs.dev study 116, draft-generation figure): for
+// positions i = 1..G in turn, the backbone logits L[i] get the bias
+// Delta_i = U[x_{i-1}] W, then a temperature softmax and an inverse-CDF draw.
+//
+// Per position two launches:
+//   tile kernel   Delta tile (GEMM over the rank r) fused with the softmax
+//                 epilogue: per (row, column tile) the max of y = L + Delta,
+//                 the sum of exp((y - max) / T) and the argmax.  Delta never
+//                 reaches HBM.  (bf16 rounds use the tcgen05 kernel of
+//                 draft_tc.cu; this file holds the CUDA-core kernel used for
+//                 fp32 rounds.)
+//   finalize      one CTA per row: combines the tile partials into (max, Z),
+//                 finds the tile where u Z falls by a prefix scan over the
+//                 tile sums, recomputes that one tile's values and scans it to
+//                 the sampled token; writes x_i, p_d(x_i), max, Z and, for the
+//                 tensor-core kernel, the next position's gathered U row.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dspark {
+
+// ---------------------------------------------------------------------------
+// CUDA-core tile kernel: 32 rows x 256 columns per CTA of 256 threads.  Each
+// thread owns one column and accumulates Delta for the 32 rows over the rank.
+constexpr int kSimtRows = 32;
+constexpr int kSimtCols = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(256) draft_tile_simt(
+    const T *__restrict__ L, const T *__restrict__ U, const T *__restrict__ Wt,
+    const int32_t *__restrict__ x0, const int32_t *__restrict__ xprev_base,
+    const float *__restrict__ temp, int B, int G, int V, int r, int pos, int nTiles,
+    float *__restrict__ part_m, float *__restrict__ part_s, int32_t *__restrict__ part_a,
+    WsHeader *hdr)
+{
+    __shared__ float Es[kSimtRows][33];
+    __shared__ int prev_s[kSimtRows];
+    __shared__ float red_v[8][kSimtRows];
+    __shared__ int red_i[8][kSimtRows];
+    __shared__ float row_m[kSimtRows];
+    __shared__ float row_invT[kSimtRows];
+
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int tile = blockIdx.x;
+    const int row0 = blockIdx.y * kSimtRows;
+    const int col = tile * kSimtCols + tid;
+    const bool colok = col < V;
+
+    if (tid < kSimtRows) {
+        int b = row0 + tid, p = 0;
+        float invT = 0.f;
+        if (b < B) {
+            p = (pos == 0) ? clamp_token(x0[b], V, hdr) : xprev_base[(size_t)b * G + pos - 1];
+            float Tb = sane_temp(temp[b], hdr);
+            invT = Tb > 0.f ? 1.f / Tb : 0.f;
+        }
+        prev_s[tid] = p;
+        row_invT[tid] = invT;
+    }
+
+    float acc[kSimtRows];
+#pragma unroll
+    for (int j = 0; j < kSimtRows; ++j) acc[j] = 0.f;
+
+    for (int k0 = 0; k0 < r; k0 += 32) {
+        __syncthreads();
+        for (int e = tid; e < kSimtRows * 32; e += blockDim.x) {
+            int rr = e >> 5, kk = e & 31;
+            float v = 0.f;
+            if (row0 + rr < B && k0 + kk < r) v = ld_elem(U, (size_t)prev_s[rr] * r + k0 + kk);
+            Es[rr][kk] = v;
+        }
+        __syncthreads();
+        float wv[32];
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk)
+            wv[kk] = (colok && k0 + kk < r) ? ld_elem(Wt, (size_t)col * r + k0 + kk) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kSimtRows; ++j) {
+            float a = acc[j];
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) a = fmaf(Es[j][kk], wv[kk], a);
+            acc[j] = a;
+        }
+    }
+
+    // Epilogue, phase 1: per-row max of y = L + Delta and its lowest argmax.
+    float lv[kSimtRows];
+#pragma unroll
+    for (int j = 0; j < kSimtRows; ++j) {
+        int b = row0 + j;
+        float l = 0.f, y = -INFINITY;
+        if (b < B && colok) {
+            l = ld_elem(L, ((size_t)b * G + pos) * V + col);
+            y = l + acc[j];
+        }
+        lv[j] = l;
+        float v = y;
+        int ix = colok ? col : 0x7fffffff;
+        warp_argmax(v, ix);
+        if (lane == 0) { red_v[wid][j] = v; red_i[wid][j] = ix; }
+    }
+    __syncthreads();
+    if (tid < kSimtRows) {
+        float v = red_v[0][tid];
+        int ix = red_i[0][tid];
+        for (int w = 1; w < 8; ++w) {
+            float ov = red_v[w][tid];
+            int oi = red_i[w][tid];
+            if (ov > v || (ov == v && oi < ix)) { v = ov; ix = oi; }
+        }
+        row_m[tid] = v;
+        int b = row0 + tid;
+        if (b < B) {
+            part_m[(size_t)b * nTiles + tile] = v;
+            part_a[(size_t)b * nTiles + tile] = ix;
+        }
+    }
+    __syncthreads();
+    // Phase 2: sum of exp(((L - m) + Delta) / T) over the tile.
+#pragma unroll
+    for (int j = 0; j < kSimtRows; ++j) {
+        float e = 0.f;
+        if (row0 + j < B && colok && row_invT[j] > 0.f)
+            e = exp_e(((lv[j] - row_m[j]) + acc[j]) * row_invT[j]);
+        e = warp_sum(e);
+        if (lane == 0) red_v[wid][j] = e;
+    }
+    __syncthreads();
+    if (tid < kSimtRows && row0 + tid < B) {
+        float s = 0.f;
+        for (int w = 0; w < 8; ++w) s += red_v[w][tid];
+        part_s[(size_t)(row0 + tid) * nTiles + tile] = s;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Gather E[b] = U[x0[b]] (bf16 rows) for the tensor-core kernel's first position.
+__global__ void gather_rows_bf16(const __nv_bfloat16 *__restrict__ U, const int32_t *__restrict__ tok,
+                                 int B, int V, int r, __nv_bfloat16 *__restrict__ E, WsHeader *hdr)
+{
+    int b = blockIdx.x;
+    int t = clamp_token(tok[b], V, hdr);
+    const uint4 *src = reinterpret_cast<const uint4 *>(U + (size_t)t * r);
+    uint4 *dst = reinterpret_cast<uint4 *>(E + (size_t)b * r);
+    for (int j = threadIdx.x; j < r / 8; j += blockDim.x) dst[j] = src[j];
+}
+
+// ---------------------------------------------------------------------------
+// Finalize: one CTA (kFinThreads threads) per request row.
+constexpr int kFinThreads = 512;
+
+template <typename T>
+__global__ void __launch_bounds__(kFinThreads) draft_finalize(
+    const T *__restrict__ L, const T *__restrict__ U, const T *__restrict__ Wt,
+    const int32_t *__restrict__ x0, const float *__restrict__ temp,
+    const float *__restrict__ u_draft, int B, int G, int V, int r, int pos, int nTiles, int TN,
+    const float *__restrict__ part_m, const float *__restrict__ part_s,
+    const int32_t *__restrict__ part_a, int32_t *__restrict__ x_out, float *__restrict__ pd_out,
+    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out,
+    __nv_bfloat16 *__restrict__ Enext, WsHeader *hdr)
+{
+    extern __shared__ float fin_smem[];
+    float *pref = fin_smem;                 // [nTiles] inclusive tile prefixes
+    float *urow = fin_smem + nTiles;        // [r] U[x_{i-1}] row
+    __shared__ float red[33];
+    __shared__ int redi[33];
+    __shared__ float carry_s;
+
+    const int b = blockIdx.x, tid = threadIdx.x;
+    const size_t ro = (size_t)b * G + pos;
+    const float *pm = part_m + (size_t)b * nTiles;
+    const float *ps = part_s + (size_t)b * nTiles;
+    const float Tb = sane_temp(temp[b], hdr);
+
+    float m = -INFINITY;
+    for (int t = tid; t < nTiles; t += blockDim.x) m = fmaxf(m, pm[t]);
+    const float M = block_max(m, red);
+
+    int x;
+    float pd, Z;
+    if (Tb == 0.f) {
+        int first = 0x7fffffff;
+        for (int t = tid; t < nTiles; t += blockDim.x)
+            if (pm[t] == M) first = min(first, t);
+        first = block_min_i(first, redi);
+        if (first >= nTiles) first = 0;  // no tile matched (non-finite inputs)
+        x = part_a[(size_t)b * nTiles + first];
+        if (x < 0 || x >= V) x = 0;
+        pd = 1.f;
+        Z = 1.f;
+    } else {
+        const float invT = 1.f / Tb;
+        // Inclusive prefix over the scaled tile sums, in tile order.
+        if (tid == 0) carry_s = 0.f;
+        __syncthreads();
+        for (int t0 = 0; t0 < nTiles; t0 += blockDim.x) {
+            int t = t0 + tid;
+            float w = t < nTiles ? ps[t] * exp_e((pm[t] - M) * invT) : 0.f;
+            float tot;
+            float inc = block_incl_scan(w, red, &tot);
+            float c = carry_s;
+            if (t < nTiles) pref[t] = c + inc;
+            __syncthreads();
+            if (tid == 0) carry_s = c + tot;
+            __syncthreads();
+        }
+        Z = carry_s;
+        const float target = u_draft[ro] * Z;
+        int ts = 0x7fffffff;
+        for (int t = tid; t < nTiles; t += blockDim.x)
+            if (pref[t] > target) ts = min(ts, t);
+        ts = block_min_i(ts, redi);
+        if (ts == 0x7fffffff) {  // rounding left u Z at the top: last tile with mass
+            int lt = -1;
+            for (int t = tid; t < nTiles; t += blockDim.x)
+                if (ps[t] > 0.f) lt = max(lt, t);
+            ts = -block_min_i(-lt, redi);
+            if (ts < 0) ts = nTiles - 1;
+        }
+        const float rem = target - (ts > 0 ? pref[ts - 1] : 0.f);
+        // Recompute the chosen tile: Delta on CUDA cores for its TN columns.
+        const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
+        for (int k = tid; k < r; k += blockDim.x) urow[k] = ld_elem(U, (size_t)prev * r + k);
+        __syncthreads();
+        const int c0 = ts * TN;
+        float e = 0.f;
+        const int col = c0 + tid;
+        if (tid < TN && col < V) {
+            float dl = 0.f;
+            for (int k = 0; k < r; ++k) dl = fmaf(urow[k], ld_elem(Wt, (size_t)col * r + k), dl);
+            float l = ld_elem(L, ro * V + col);
+            e = exp_e(((l - M) + dl) * invT);
+        }
+        float tot;
+        float inc = block_incl_scan(e, red, &tot);
+        int xs = (tid < TN && col < V && inc > rem) ? col : 0x7fffffff;
+        xs = block_min_i(xs, redi);
+        if (xs == 0x7fffffff) {  // the tile's recomputed mass fell short: last positive
+            int lc = (e > 0.f) ? col : -1;
+            xs = -block_min_i(-lc, redi);
+            if (xs < 0) xs = min(c0 + TN, V) - 1;
+        }
+        x = xs;
+        // p_d(x) from the recomputed value of the chosen column.
+        __shared__ float ex_s;
+        if (col == x) ex_s = e;
+        __syncthreads();
+        pd = ex_s / Z;
+    }
+    if (tid == 0) {
+        x_out[ro] = x;
+        pd_out[ro] = pd;
+        rowmax_out[ro] = M;
+        rowsum_out[ro] = Z;
+    }
+    if (Enext != nullptr) {  // next position's A-operand row for the tensor-core kernel
+        const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(U) +
+                                                           (size_t)x * r);
+        uint4 *dst = reinterpret_cast<uint4 *>(Enext + (size_t)b * r);
+        for (int j = tid; j < r / 8; j += blockDim.x) dst[j] = src[j];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+size_t draft_tiles(int V, int dtype) { return (size_t)((V + draft_tile_cols(dtype) - 1) / draft_tile_cols(dtype)); }
+
+int draft_tile_cols(int dtype) { return dtype == DSPARK_BF16 ? kTcTileN : kSimtCols; }
+
+size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
+    size_t nt = draft_tiles(V, dtype);
+    size_t bytes = sizeof(WsHeader);
+    bytes += align256(sizeof(float) * (size_t)B * nt);    // part_m
+    bytes += align256(sizeof(float) * (size_t)B * nt);    // part_s
+    bytes += align256(sizeof(int32_t) * (size_t)B * nt);  // part_a
+    if (dtype == DSPARK_BF16) bytes += align256(sizeof(__nv_bfloat16) * (size_t)round_up(B, 128) * r);  // E
+    return bytes;
+}
+
+DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
+    DraftWs w;
+    size_t nt = draft_tiles(V, dtype);
+    char *p = static_cast<char *>(ws);
+    w.hdr = reinterpret_cast<WsHeader *>(p);
+    p += sizeof(WsHeader);
+    w.part_m = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
+    w.part_s = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
+    w.part_a = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (size_t)B * nt);
+    w.E = nullptr;
+    if (dtype == DSPARK_BF16) w.E = reinterpret_cast<__nv_bfloat16 *>(p);
+    w.nTiles = (int)nt;
+    return w;
+}
+
+template <typename T>
+static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st,
+                                   __nv_bfloat16 *Enext) {
+    size_t smem = sizeof(float) * ((size_t)w.nTiles + a.r);
+    auto kern = draft_finalize<T>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<a.B, kFinThreads, smem, st>>>(
+        static_cast<const T *>(a.L), static_cast<const T *>(a.U), static_cast<const T *>(a.Wt), a.x0,
+        a.temp, a.u_draft, a.B, a.G, a.V, a.r, pos, w.nTiles, draft_tile_cols(a.dtype), w.part_m,
+        w.part_s, w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out, Enext, w.hdr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
+    DraftWs w = carve_draft_ws(ws, a.B, a.V, a.r, a.dtype);
+    cudaError_t e;
+    if (a.dtype == DSPARK_F32) {
+        dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
+        for (int pos = 0; pos < a.G; ++pos) {
+            draft_tile_simt<float><<<grid, 256, 0, st>>>(
+                static_cast<const float *>(a.L), static_cast<const float *>(a.U),
+                static_cast<const float *>(a.Wt), a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos,
+                w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if ((e = launch_finalize<float>(a, w, pos, st, nullptr)) != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
+    // bf16: tensor-core tile kernel, A operand gathered into w.E.
+    gather_rows_bf16<<<a.B, 64, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.U), a.x0, a.B, a.V, a.r,
+                                         w.E, w.hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    for (int pos = 0; pos < a.G; ++pos) {
+        if ((e = launch_draft_tile_tc(a, w, pos, st)) != cudaSuccess) return e;
+        __nv_bfloat16 *En = (pos + 1 < a.G) ? w.E : nullptr;
+        if ((e = launch_finalize<__nv_bfloat16>(a, w, pos, st, En)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace dspark
+
+namespace dspark {
+// Interim bf16 tile launcher on CUDA cores (same tile width as the tensor-core kernel).
+cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
+    static_assert(kTcTileN == kSimtCols, "interim path shares the tile width");
+    dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
+    draft_tile_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(a.L), static_cast<const __nv_bfloat16 *>(a.U),
+        static_cast<const __nv_bfloat16 *>(a.Wt), a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos,
+        w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
+    return cudaGetLastError();
+}
+}  // namespace dspark

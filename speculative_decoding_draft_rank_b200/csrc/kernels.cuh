@@ -1,0 +1,63 @@
+// kernels.cuh -- launch interfaces shared by the stage files of the library.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Column-tile width of the bf16 (tensor-core) drafting and residual kernels.
+constexpr int kTcTileN = 256;
+
+// ----------------------------------------------------------------- drafting
+struct DraftArgs {
+    const void *L, *U, *Wt;
+    const int32_t *x0;
+    const float *temp, *u_draft;
+    int B, G, V, r, dtype;
+    int32_t *x_out;
+    float *pd_out, *rowmax_out, *rowsum_out;
+};
+
+struct DraftWs {
+    WsHeader *hdr;
+    float *part_m, *part_s;
+    int32_t *part_a;
+    __nv_bfloat16 *E;   // [round_up(B,128), r] gathered U rows (bf16 only)
+    int nTiles;
+};
+
+int draft_tile_cols(int dtype);
+size_t draft_tiles(int V, int dtype);
+size_t draft_ws_bytes(int B, int G, int V, int r, int dtype);
+DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype);
+cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st);
+cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st);
+
+// --------------------------------------------------------------- confidence
+cudaError_t launch_confidence(const void *h, const void *w, float bias, const float *tau, int B,
+                              int G, int d, int dtype, float *c_out, float *S_out, cudaStream_t st);
+
+// ---------------------------------------------------------------- scheduler
+size_t schedule_ws_bytes(int B, int G);
+cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
+                            const double *knots_t, int P, int budget, int mode, void *ws,
+                            int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
+                            int32_t *order_out, cudaStream_t st);
+
+// ------------------------------------------------------------- verification
+struct VerifyArgs {
+    const void *Tlog, *L, *U, *Wt;
+    const int32_t *x0, *x;
+    const float *pd_x, *rowmax, *rowsum, *temp, *u_accept, *u_final;
+    const int32_t *ell;
+    int B, G, V, r, dtype;
+    int32_t *acc_out, *tokens_out, *nout_out;
+    float *pt_x_out;
+};
+size_t verify_ws_bytes(int B, int G, int V, int r, int dtype);
+cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st);
+
+}  // namespace dspark

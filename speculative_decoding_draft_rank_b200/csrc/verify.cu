@@ -1,0 +1,558 @@
+// verify.cu -- stage 4, exact rejection-sampling verification.
+//
+// Method (menfem.com KB entry on DSpark, "Methodology": x_k is accepted with
+// probability min(1, p_t(x_k) / p_d(x_k)) and the first rejection discards
+// every later token; paperlayer.ai summary, §2: the longest consistent prefix
+// is kept; Appendix A: with nothing admitted the target draws a fresh
+// token).  A rejection at k* is replaced by a draw from the normalised
+// residual max(0, p_t - p_d) at k*; a fully accepted prefix earns a bonus
+// draw from p_t at row ell + 1.
+//
+// Launch sequence (fixed, graph-capturable; work counts live on the device):
+//   plan        1 CTA: row list of the admitted target rows, rows (b, k) for
+//               k = 0..ell_b (0-based), and their offsets per request.
+//   rows        persistent grid over (row, 8192-column chunk) work items:
+//               one streaming pass over each target row with 16-byte loads,
+//               giving per chunk the max, lowest argmax and sum of
+//               exp((t - max) / T).
+//   decide      1 CTA per request: row max / Z from the chunk partials,
+//               p_t(x_k), the accept tests, the first-rejection count A, the
+//               bonus draw (prefix over chunk sums, then one chunk rescanned)
+//               or the greedy token; rejected rows are queued for the residual.
+//   residual    Delta recomputed for the queued rows (CUDA-core GEMM tile,
+//               as in drafting) fused with q = max(0, p_t - p_d) tile sums.
+//   res_final   1 CTA per queued row: prefix over tile sums, one tile
+//               recomputed and scanned to the replacement token.
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace dspark {
+
+constexpr int kChunk = 8192;          // columns per row work item
+constexpr int kRowThreads = 256;      // threads of the row and decide kernels
+constexpr int kResRows = 32;          // queued rows per residual tile CTA
+constexpr int kResCols = 256;         // columns per residual tile
+
+struct VerifyWs {
+    WsHeader *hdr;             // pad[0] = row count, pad[1] = residual count
+    int32_t *rows;             // [B*(G+1)] packed b * 32 + k
+    int32_t *row_off;          // [B+1]
+    float *cm, *cs;            // [B*(G+1)*nChunks] chunk max / sum
+    int32_t *ca;               // [B*(G+1)*nChunks] chunk argmax
+    int32_t *res_b;            // [B] queued request
+    int32_t *res_k;            // [B] rejected position (0-based)
+    float *res_mt, *res_zt;    // [B] target row max / Z of the rejected row
+    float *rp;                 // [B*nResTiles] residual tile sums
+    int nChunks, nResTiles;
+};
+
+static VerifyWs carve_verify_ws(void *ws, int B, int G, int V) {
+    VerifyWs w;
+    w.nChunks = (V + kChunk - 1) / kChunk;
+    w.nResTiles = (V + kResCols - 1) / kResCols;
+    const size_t R = (size_t)B * (G + 1);
+    char *p = static_cast<char *>(ws);
+    w.hdr = reinterpret_cast<WsHeader *>(p); p += sizeof(WsHeader);
+    w.rows = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * R);
+    w.row_off = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (B + 1));
+    w.cm = reinterpret_cast<float *>(p); p += align256(sizeof(float) * R * w.nChunks);
+    w.cs = reinterpret_cast<float *>(p); p += align256(sizeof(float) * R * w.nChunks);
+    w.ca = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * R * w.nChunks);
+    w.res_b = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * B);
+    w.res_k = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * B);
+    w.res_mt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
+    w.res_zt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
+    w.rp = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * w.nResTiles);
+    return w;
+}
+
+size_t verify_ws_bytes(int B, int G, int V, int, int) {
+    const int nChunks = (V + kChunk - 1) / kChunk, nResTiles = (V + kResCols - 1) / kResCols;
+    const size_t R = (size_t)B * (G + 1);
+    return sizeof(WsHeader) + align256(4 * R) + align256(4 * (B + 1)) + 3 * align256(4 * R * nChunks) +
+           4 * align256(4 * (size_t)B) + align256(4 * (size_t)B * nResTiles);
+}
+
+// Eight consecutive elements starting at index i of a row (bounds-checked;
+// one or two 16-byte loads when aligned and complete).
+__device__ __forceinline__ void load8(const __nv_bfloat16 *row, int i, int n, float (&v)[8]) {
+    const __nv_bfloat16 *p = row + i;
+    if (i + 8 <= n && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+        uint4 q = ld_stream16(p);
+        v[0] = bf16lo(q.x); v[1] = bf16hi(q.x); v[2] = bf16lo(q.y); v[3] = bf16hi(q.y);
+        v[4] = bf16lo(q.z); v[5] = bf16hi(q.z); v[6] = bf16lo(q.w); v[7] = bf16hi(q.w);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = (i + q < n) ? __bfloat162float(p[q]) : -INFINITY;
+    }
+}
+__device__ __forceinline__ void load8(const float *row, int i, int n, float (&v)[8]) {
+    const float *p = row + i;
+    if (i + 8 <= n && (reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+        uint4 a = ld_stream16(p), b = ld_stream16(p + 4);
+        v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y); v[2] = __uint_as_float(a.z);
+        v[3] = __uint_as_float(a.w); v[4] = __uint_as_float(b.x); v[5] = __uint_as_float(b.y);
+        v[6] = __uint_as_float(b.z); v[7] = __uint_as_float(b.w);
+    } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = (i + q < n) ? p[q] : -INFINITY;
+    }
+}
+
+// ----------------------------------------------------------------- plan
+__global__ void verify_plan(const int32_t *__restrict__ ell, int B, int G, VerifyWs w) {
+    __shared__ int tot[33];
+    __shared__ int carry;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    if (tid == 0) { carry = 0; w.hdr->pad[1] = 0; }
+    __syncthreads();
+    for (int b0 = 0; b0 < B; b0 += blockDim.x) {
+        const int b = b0 + tid;
+        int n = 0;
+        if (b < B) {
+            int l = ell[b];
+            if (l < 0 || l > G) { flag_status(w.hdr, DSPARK_DEV_ELL_RANGE); l = l < 0 ? 0 : G; }
+            n = l + 1;
+        }
+        int inc = warp_incl_scan_i(n);
+        if (lane == 31) tot[wid] = inc;
+        __syncthreads();
+        if (wid == 0) {
+            int t = lane < (int)(blockDim.x >> 5) ? tot[lane] : 0;
+            t = warp_incl_scan_i(t);
+            tot[lane] = t;
+        }
+        __syncthreads();
+        const int off = carry + inc - n + (wid > 0 ? tot[wid - 1] : 0);
+        if (b < B) {
+            w.row_off[b] = off;
+            for (int k = 0; k < n; ++k) w.rows[off + k] = b * 32 + k;
+        }
+        __syncthreads();
+        if (tid == 0) carry += tot[(blockDim.x >> 5) - 1];
+        __syncthreads();
+    }
+    if (tid == 0) { w.row_off[B] = carry; w.hdr->pad[0] = carry; }
+}
+
+// ----------------------------------------------------------------- rows
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__ Tlog,
+                                                           const float *__restrict__ temp, int G,
+                                                           int V, VerifyWs w) {
+    __shared__ float rv[8];
+    __shared__ int ri[8];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
+    const int nwork = nrows * w.nChunks;
+    for (int item = blockIdx.x; item < nwork; item += gridDim.x) {
+        const int j = item / w.nChunks, c = item - j * w.nChunks;
+        const int rk = w.rows[j], b = rk >> 5, k = rk & 31;
+        float Tb = temp[b];
+        Tb = Tb >= 0.f ? Tb : 0.f;
+        const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
+        const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
+        const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
+        float v[4][8];
+        float m = -INFINITY;
+        int am = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int i = c0 + (q * kRowThreads + tid) * 8;
+            if (i < c1) {
+                load8(row, i, c1, v[q]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (v[q][e] > m) { m = v[q][e]; am = i + e; }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[q][e] = -INFINITY;
+            }
+        }
+        float wm = m;
+        int wa = am;
+        warp_argmax(wm, wa);
+        if (lane == 0) { rv[wid] = wm; ri[wid] = wa; }
+        __syncthreads();
+        float M = rv[0];
+        int A = ri[0];
+        for (int q = 1; q < 8; ++q)
+            if (rv[q] > M || (rv[q] == M && ri[q] < A)) { M = rv[q]; A = ri[q]; }
+        __syncthreads();
+        float s = 0.f;
+        if (invT > 0.f) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s += exp_e((v[q][e] - M) * invT);
+        }
+        s = warp_sum(s);
+        if (lane == 0) rv[wid] = s;
+        __syncthreads();
+        if (tid == 0) {
+            float t = 0.f;
+            for (int q = 0; q < 8; ++q) t += rv[q];
+            const size_t o = (size_t)j * w.nChunks + c;
+            w.cm[o] = M;
+            w.cs[o] = t;
+            w.ca[o] = A;
+        }
+        __syncthreads();
+    }
+}
+
+// Row statistics from the chunk partials of compacted row j (one warp).
+__device__ __forceinline__ void row_stats(const VerifyWs &w, int j, float invT, float &M, float &Z,
+                                          int &A) {
+    const int lane = threadIdx.x & 31;
+    const float *cm = w.cm + (size_t)j * w.nChunks;
+    const float *cs = w.cs + (size_t)j * w.nChunks;
+    const int32_t *ca = w.ca + (size_t)j * w.nChunks;
+    float m = -INFINITY;
+    int a = 0x7fffffff;
+    for (int c = lane; c < w.nChunks; c += 32)
+        if (cm[c] > m || (cm[c] == m && ca[c] < a)) { m = cm[c]; a = ca[c]; }
+    warp_argmax(m, a);
+    float z = 0.f;
+    if (invT > 0.f)
+        for (int c = lane; c < w.nChunks; c += 32) z += cs[c] * exp_e((cm[c] - m) * invT);
+    z = warp_sum(z);
+    M = m; Z = z; A = a;
+}
+
+// Inverse-CDF draw from target row j (compacted index; request b, position
+// k) with row stats (M, Z): prefix over the chunk sums, then the chosen chunk
+// rescanned in index order.  Whole block; returns the token.
+template <typename T>
+__device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, int j, int b, int k,
+                                 int G, int V, float M, float Z, float invT, float u, float *red,
+                                 int *redi) {
+    const int tid = threadIdx.x;
+    const float *cm = w.cm + (size_t)j * w.nChunks;
+    const float *cs = w.cs + (size_t)j * w.nChunks;
+    const float target = u * Z;
+    // Prefix over chunk sums (nChunks <= 128 for V <= 2^20; kRowThreads >= that).
+    float wc = tid < w.nChunks ? cs[tid] * exp_e((cm[tid] - M) * invT) : 0.f;
+    float tot;
+    float inc = block_incl_scan(wc, red, &tot);
+    int cs_ = (tid < w.nChunks && inc > target) ? tid : 0x7fffffff;
+    cs_ = block_min_i(cs_, redi);
+    if (cs_ == 0x7fffffff) {
+        int lc = (tid < w.nChunks && wc > 0.f) ? tid : -1;
+        cs_ = -block_min_i(-lc, redi);
+        if (cs_ < 0) cs_ = w.nChunks - 1;
+    }
+    __shared__ float excl_s;
+    if (tid == cs_) excl_s = inc - wc;
+    __syncthreads();
+    float rem = target - excl_s;
+    const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
+    const int c0 = cs_ * kChunk, c1 = min(V, c0 + kChunk);
+    int found = 0x7fffffff, lastpos = -1;
+    for (int q = 0; q < 4; ++q) {
+        const int i = c0 + (q * kRowThreads + tid) * 8;
+        float v[8];
+        float e[8];
+        float run = 0.f;
+        if (i < c1) load8(row, i, c1, v);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            e[t] = (i < c1 && i + t < c1) ? exp_e((v[t] - M) * invT) : 0.f;
+            run += e[t];
+            if (e[t] > 0.f) lastpos = i + t;
+        }
+        float rt;
+        float incl = block_incl_scan(run, red, &rt);
+        float p = incl - run;
+        int f = 0x7fffffff;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            p += e[t];
+            if (f == 0x7fffffff && e[t] > 0.f && p > rem) f = i + t;
+        }
+        f = block_min_i(f, redi);
+        if (f != 0x7fffffff) { found = f; break; }
+        rem -= rt;
+    }
+    if (found == 0x7fffffff) {
+        found = -block_min_i(-lastpos, redi);
+        if (found < 0) found = c1 - 1;
+    }
+    return found;
+}
+
+// ----------------------------------------------------------------- decide
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) verify_decide(
+    const T *__restrict__ Tlog, const int32_t *__restrict__ x, const float *__restrict__ pd_x,
+    const float *__restrict__ temp, const float *__restrict__ u_accept,
+    const float *__restrict__ u_final, const int32_t *__restrict__ ell, int B, int G, int V,
+    VerifyWs w, int32_t *__restrict__ acc_out, int32_t *__restrict__ tokens_out,
+    int32_t *__restrict__ nout_out, float *__restrict__ pt_x_out) {
+    __shared__ float rM[17], rZ[17];
+    __shared__ int rA[17];
+    __shared__ float red[33];
+    __shared__ int redi[33];
+    __shared__ int A_s;
+    const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float Tb = sane_temp(temp[b], w.hdr);
+    const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
+    int lb = ell[b];
+    lb = lb < 0 ? 0 : (lb > G ? G : lb);
+    const int j0 = w.row_off[b];
+    for (int k = wid; k <= lb; k += kRowThreads / 32) {
+        float M, Z;
+        int A;
+        row_stats(w, j0 + k, invT, M, Z, A);
+        if (lane == 0) { rM[k] = M; rZ[k] = Z; rA[k] = A; }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int A = 0;
+        bool rejected = false;
+        for (int k = 0; k < G; ++k) {
+            const size_t o = (size_t)b * G + k;
+            float pt = -1.f;
+            if (k < lb) {
+                const int xk = clamp_token(x[o], V, w.hdr);
+                bool acc;
+                if (Tb == 0.f) {
+                    acc = (rA[k] == xk);
+                    pt = acc ? 1.f : 0.f;
+                } else {
+                    const float t = to_f32(Tlog[((size_t)b * (G + 1) + k) * V + xk]);
+                    pt = exp_e((t - rM[k]) * invT) / rZ[k];
+                    acc = u_accept[o] < pt / pd_x[o];
+                }
+                if (!rejected) {
+                    if (acc) ++A; else rejected = true;
+                }
+            }
+            if (pt_x_out != nullptr) pt_x_out[o] = pt;
+        }
+        A_s = A;
+        acc_out[b] = A;
+        nout_out[b] = A + 1;
+        int32_t *tok = tokens_out + (size_t)b * (G + 1);
+        for (int q = 0; q <= G; ++q) tok[q] = q < A ? x[(size_t)b * G + q] : -1;
+        if (Tb == 0.f) {
+            tok[A] = (rA[A] >= 0 && rA[A] < V) ? rA[A] : 0;
+        } else if (A < lb) {  // queue the rejected row for the residual draw
+            const int slot = atomicAdd(&w.hdr->pad[1], 1u);
+            w.res_b[slot] = b;
+            w.res_k[slot] = A;
+            w.res_mt[slot] = rM[A];
+            w.res_zt[slot] = rZ[A];
+        }
+    }
+    __syncthreads();
+    const int A = A_s;
+    if (Tb > 0.f && A == lb) {  // bonus (fresh token when nothing was admitted)
+        const int y = sample_target_row(Tlog, w, j0 + lb, b, lb, G, V, rM[lb], rZ[lb], invT,
+                                        u_final[b], red, redi);
+        if (tid == 0) tokens_out[(size_t)b * (G + 1) + A] = y;
+    }
+}
+
+// ----------------------------------------------------------------- residual
+// q = max(0, p_t - p_d) tile sums for the queued rows; p_d rebuilt from
+// L + U[x_{k-1}] W (CUDA-core tile GEMM) and the drafting stats.
+template <typename T>
+__global__ void __launch_bounds__(256) residual_tile_simt(
+    const T *__restrict__ Tlog, const T *__restrict__ L, const T *__restrict__ U,
+    const T *__restrict__ Wt, const int32_t *__restrict__ x0, const int32_t *__restrict__ x,
+    const float *__restrict__ rowmax, const float *__restrict__ rowsum,
+    const float *__restrict__ temp, int G, int V, int r, VerifyWs w) {
+    __shared__ float Es[kResRows][33];
+    __shared__ int prev_s[kResRows], b_s[kResRows], k_s[kResRows];
+    __shared__ float red[8][kResRows];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int nres = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[1]);
+    const int row0 = blockIdx.y * kResRows;
+    if (row0 >= nres) return;
+    const int tile = blockIdx.x;
+    const int col = tile * kResCols + tid;
+    const bool colok = col < V;
+    if (tid < kResRows) {
+        int s = row0 + tid, b = 0, k = 0, p = 0;
+        if (s < nres) {
+            b = w.res_b[s];
+            k = w.res_k[s];
+            p = (k == 0) ? x0[b] : x[(size_t)b * G + k - 1];
+            p = min(max(p, 0), V - 1);
+        }
+        b_s[tid] = b; k_s[tid] = k; prev_s[tid] = p;
+    }
+    float acc[kResRows];
+#pragma unroll
+    for (int j = 0; j < kResRows; ++j) acc[j] = 0.f;
+    for (int k0 = 0; k0 < r; k0 += 32) {
+        __syncthreads();
+        for (int e = tid; e < kResRows * 32; e += blockDim.x) {
+            int rr = e >> 5, kk = e & 31;
+            float v = 0.f;
+            if (row0 + rr < nres && k0 + kk < r) v = ld_elem(U, (size_t)prev_s[rr] * r + k0 + kk);
+            Es[rr][kk] = v;
+        }
+        __syncthreads();
+        float wv[32];
+#pragma unroll
+        for (int kk = 0; kk < 32; ++kk)
+            wv[kk] = (colok && k0 + kk < r) ? ld_elem(Wt, (size_t)col * r + k0 + kk) : 0.f;
+#pragma unroll
+        for (int j = 0; j < kResRows; ++j) {
+            float a = acc[j];
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) a = fmaf(Es[j][kk], wv[kk], a);
+            acc[j] = a;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kResRows; ++j) {
+        const int s = row0 + j;
+        float q = 0.f;
+        if (s < nres && colok) {
+            const int b = b_s[j], k = k_s[j];
+            const float Tb = fmaxf(temp[b], 0.f);
+            const float invT = 1.f / Tb;
+            const size_t ro = (size_t)b * G + k;
+            const float l = ld_elem(L, ro * V + col);
+            const float pd = exp_e(((l - rowmax[ro]) + acc[j]) * invT) / rowsum[ro];
+            const float t = ld_elem(Tlog, ((size_t)b * (G + 1) + k) * V + col);
+            const float pt = exp_e((t - w.res_mt[s]) * invT) / w.res_zt[s];
+            q = fmaxf(pt - pd, 0.f);
+        }
+        q = warp_sum(q);
+        if (lane == 0) red[wid][j] = q;
+    }
+    __syncthreads();
+    if (tid < kResRows && row0 + tid < nres) {
+        float s = 0.f;
+        for (int q = 0; q < 8; ++q) s += red[q][tid];
+        w.rp[(size_t)(row0 + tid) * w.nResTiles + tile] = s;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) residual_final(
+    const T *__restrict__ Tlog, const T *__restrict__ L, const T *__restrict__ U,
+    const T *__restrict__ Wt, const int32_t *__restrict__ x0, const int32_t *__restrict__ x,
+    const float *__restrict__ rowmax, const float *__restrict__ rowsum,
+    const float *__restrict__ temp, const float *__restrict__ u_final, int G, int V, int r,
+    VerifyWs w, int32_t *__restrict__ tokens_out) {
+    extern __shared__ float res_smem[];
+    float *pref = res_smem;               // [nResTiles]
+    float *urow = res_smem + w.nResTiles; // [r]
+    __shared__ float red[33];
+    __shared__ int redi[33];
+    __shared__ float carry_s;
+    const int s = blockIdx.x, tid = threadIdx.x;
+    const int nres = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[1]);
+    if (s >= nres) return;
+    const int b = w.res_b[s], k = w.res_k[s];
+    const float Tb = fmaxf(temp[b], 0.f), invT = 1.f / Tb;
+    const size_t ro = (size_t)b * G + k;
+    const float Md = rowmax[ro], Zd = rowsum[ro], Mt = w.res_mt[s], Zt = w.res_zt[s];
+    const float *tp = w.rp + (size_t)s * w.nResTiles;
+    if (tid == 0) carry_s = 0.f;
+    __syncthreads();
+    for (int t0 = 0; t0 < w.nResTiles; t0 += blockDim.x) {
+        const int t = t0 + tid;
+        float v = t < w.nResTiles ? tp[t] : 0.f;
+        float tot;
+        float inc = block_incl_scan(v, red, &tot);
+        const float c = carry_s;
+        if (t < w.nResTiles) pref[t] = c + inc;
+        __syncthreads();
+        if (tid == 0) carry_s = c + tot;
+        __syncthreads();
+    }
+    const float Q = carry_s;
+    const float u = u_final[b];
+    int y;
+    if (!(Q > 0.f)) {  // empty residual: draw from p_t of the rejected row
+        y = sample_target_row(Tlog, w, w.row_off[b] + k, b, k, G, V, Mt, Zt, invT, u, red, redi);
+    } else {
+        const float target = u * Q;
+        int ts = 0x7fffffff;
+        for (int t = tid; t < w.nResTiles; t += blockDim.x)
+            if (pref[t] > target) ts = min(ts, t);
+        ts = block_min_i(ts, redi);
+        if (ts == 0x7fffffff) {
+            int lt = -1;
+            for (int t = tid; t < w.nResTiles; t += blockDim.x)
+                if (tp[t] > 0.f) lt = max(lt, t);
+            ts = -block_min_i(-lt, redi);
+            if (ts < 0) ts = w.nResTiles - 1;
+        }
+        const float rem = target - (ts > 0 ? pref[ts - 1] : 0.f);
+        const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
+        for (int q = tid; q < r; q += blockDim.x) urow[q] = ld_elem(U, (size_t)prev * r + q);
+        __syncthreads();
+        const int c0 = ts * kResCols;
+        float qv = 0.f;
+        const int col = c0 + tid;
+        if (tid < kResCols && col < V) {
+            float dl = 0.f;
+            for (int q = 0; q < r; ++q) dl = fmaf(urow[q], ld_elem(Wt, (size_t)col * r + q), dl);
+            const float pd = exp_e(((ld_elem(L, ro * V + col) - Md) + dl) * invT) / Zd;
+            const float pt = exp_e((ld_elem(Tlog, ((size_t)b * (G + 1) + k) * V + col) - Mt) * invT) / Zt;
+            qv = fmaxf(pt - pd, 0.f);
+        }
+        float tot;
+        float inc = block_incl_scan(qv, red, &tot);
+        int ys = (tid < kResCols && col < V && qv > 0.f && inc > rem) ? col : 0x7fffffff;
+        ys = block_min_i(ys, redi);
+        if (ys == 0x7fffffff) {
+            int lc = (qv > 0.f) ? col : -1;
+            ys = -block_min_i(-lc, redi);
+            if (ys < 0) ys = min(c0 + kResCols, V) - 1;
+        }
+        y = ys;
+    }
+    if (tid == 0) tokens_out[(size_t)b * (G + 1) + k] = y;
+}
+
+// ----------------------------------------------------------------- host
+template <typename T>
+static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaStream_t st) {
+    const T *Tl = static_cast<const T *>(a.Tlog);
+    verify_plan<<<1, 1024, 0, st>>>(a.ell, a.B, a.G, w);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int maxwork = a.B * (a.G + 1) * w.nChunks;
+    const int grid = max(1, min(maxwork, sms * 8));
+    verify_rows<T><<<grid, kRowThreads, 0, st>>>(Tl, a.temp, a.G, a.V, w);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    verify_decide<T><<<a.B, kRowThreads, 0, st>>>(Tl, a.x, a.pd_x, a.temp, a.u_accept, a.u_final, a.ell,
+                                                  a.B, a.G, a.V, w, a.acc_out, a.tokens_out,
+                                                  a.nout_out, a.pt_x_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dim3 rg(w.nResTiles, (a.B + kResRows - 1) / kResRows);
+    residual_tile_simt<T><<<rg, 256, 0, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
+                                              static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax,
+                                              a.rowsum, a.temp, a.G, a.V, a.r, w);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t smem = sizeof(float) * ((size_t)w.nResTiles + a.r);
+    auto fin = residual_final<T>;
+    if (smem > 48 * 1024) {
+        if ((e = cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+    }
+    fin<<<a.B, kRowThreads, smem, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
+                                       static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax, a.rowsum,
+                                       a.temp, a.u_final, a.G, a.V, a.r, w, a.tokens_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st) {
+    VerifyWs w = carve_verify_ws(ws, a.B, a.G, a.V);
+    if (a.dtype == DSPARK_BF16) return launch_verify_t<__nv_bfloat16>(a, w, st);
+    return launch_verify_t<float>(a, w, st);
+}
+
+}  // namespace dspark

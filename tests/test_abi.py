@@ -1,0 +1,113 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/dspark.h declares, and rejects bad arguments on the host with the
+documented status codes (no CUDA call is reached on these paths)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from speculative_decoding_draft_rank_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dspark.h")
+
+FAKE = ctypes.c_void_p(0x100000)      # never dereferenced: every call below fails host checks first
+FAKE_WS = ctypes.c_void_p(0x200000)   # 256-byte aligned
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(dspark_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_exports_match_header(lib):
+    declared = _declared()
+    assert declared, "no declarations parsed"
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r" T (dspark_\w+)$", out, re.M))
+    assert set(declared) <= exported, set(declared) - exported
+    assert set(_lib.EXPORTS) == set(declared)
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_version(lib):
+    assert "sm_100a" in _lib.version()
+
+
+def test_workspace_queries(lib):
+    assert _lib.dspark_draft_workspace_size(256, 5, 129280, 256, _lib.DSPARK_BF16) > 0
+    assert _lib.dspark_verify_workspace_size(256, 5, 129280, 256, _lib.DSPARK_BF16) > 0
+    assert _lib.dspark_schedule_workspace_size(1024, 8) > 0
+    assert _lib.dspark_draft_workspace_size(0, 5, 1000, 16, 0) == 0
+    assert _lib.dspark_draft_workspace_size(4, 17, 1000, 16, 0) == 0
+    assert _lib.dspark_draft_workspace_size(4, 5, 1, 16, 0) == 0
+    assert _lib.dspark_draft_workspace_size(4, 5, 1000, 24, _lib.DSPARK_BF16) == 0  # r % 16
+    assert _lib.dspark_schedule_workspace_size(4096, 16) == 0                    # B*G > 16384
+
+
+def _draft(lib, B=4, G=5, V=1024, r=16, dtype=0, ws=FAKE_WS, ws_bytes=1 << 30, null=None):
+    args = [FAKE] * 6
+    if null is not None:
+        args[null] = None
+    return lib.dspark_draft_markov(*args, B, G, V, r, dtype, ws, ws_bytes, FAKE, FAKE, FAKE, FAKE, None)
+
+
+def test_draft_argument_checks(lib):
+    assert _draft(lib, B=0) == 1
+    assert _draft(lib, G=0) == 1
+    assert _draft(lib, G=17) == 1
+    assert _draft(lib, V=1) == 1
+    assert _draft(lib, r=24, dtype=1) == 1
+    assert _draft(lib, dtype=7) == 2
+    for k in range(6):
+        assert _draft(lib, null=k) == 1
+    assert _draft(lib, ws=None) == 3
+    assert _draft(lib, ws=ctypes.c_void_p(0x200010)) == 3          # misaligned
+    assert _draft(lib, ws_bytes=16) == 3                           # too small
+
+
+def test_schedule_and_confidence_checks(lib):
+    f = lib.dspark_schedule
+    assert f(FAKE, 4, 5, FAKE, FAKE, 0, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1  # P = 0
+    assert f(FAKE, 4, 5, FAKE, FAKE, 65, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 9, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1  # mode
+    assert f(FAKE, 4096, 8, FAKE, FAKE, 2, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 1, None, 1 << 20, FAKE, FAKE, FAKE, None, None) == 3
+    g = lib.dspark_confidence
+    assert g(FAKE, FAKE, ctypes.c_float(0), None, 4, 5, 0, 0, FAKE, FAKE, None) == 1   # d = 0
+    assert g(FAKE, FAKE, ctypes.c_float(0), None, 4, 5, 8, 3, FAKE, FAKE, None) == 2   # dtype
+    assert g(None, FAKE, ctypes.c_float(0), None, 4, 5, 8, 0, FAKE, FAKE, None) == 1
+
+
+def test_verify_argument_checks(lib):
+    f = lib.dspark_verify
+    ok = [FAKE] * 13
+    assert f(*ok, 4, 5, 1024, 16, 0, None, 1 << 30, FAKE, FAKE, FAKE, None, None) == 3
+    bad = list(ok)
+    bad[12] = None
+    assert f(*bad, 4, 5, 1024, 16, 0, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 1
+    assert f(*ok, 4, 5, 1024, 16, 0, FAKE_WS, 1 << 30, None, FAKE, FAKE, None, None) == 1
+
+
+def test_injected_failure(lib, monkeypatch):
+    """Host-side fault injection: the named entry point returns the given
+    status without enqueuing any work."""
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_draft_markov=4")
+    assert _draft(lib) == 4
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_schedule=5")
+    assert lib.dspark_schedule(FAKE, 4, 5, FAKE, FAKE, 2, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None,
+                               None) == 5
+    with pytest.raises(_lib.DsparkError) as ei:
+        _lib._call("dspark_schedule", FAKE, 4, 5, FAKE, FAKE, 2, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE,
+                   None, None)
+    assert ei.value.status == 5

@@ -53,8 +53,8 @@ def test_draft_matches_torch_softmax_and_cdf(T):
             lo = C[x - 1] if x > 0 else 0.0
             assert lo <= u[b, i] < C[x] + 1e-15
             assert res.pd[b, i] == pytest.approx(float(p[x]), rel=1e-12, abs=1e-300)
-            assert res.rowmax[b, i] == pytest.approx(float(z.max()), rel=1e-13)
-            assert np.log(res.rowsum[b, i]) + res.rowmax[b, i] == pytest.approx(
+            assert res.rowmax[b, i] == pytest.approx(float(z.max()) * T, rel=1e-13)
+            assert np.log(res.rowsum[b, i]) + res.rowmax[b, i] / T == pytest.approx(
                 float(torch.logsumexp(z, 0)), rel=1e-12)
             prev = x
 

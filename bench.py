@@ -1,0 +1,366 @@
+"""Benchmark of one DSpark round (drafting, confidence, Algorithm-1 scheduling,
+verification) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload headline]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+A step is one round over one batch of synthetic requests (the headline
+workload: B=256, G=5, V=129280, r=256, d=4096, bf16).  The round is captured
+once in a CUDA graph and replayed; L2 is flushed (a 256 MiB write) before
+every timed replay, outside the timed events.  Under torchrun every rank runs
+its own engine on its own batch (weak scaling, no collective on the data
+path); the reported time is the max over ranks.
+
+Prints one JSON line: value = verified draft tokens/s (sum over ranks of the
+admitted draft tokens per round / round time), plus the round's fraction of
+the HBM roofline, the dominant stage's roofline, the oracle's CPU baseline,
+an end-to-end number through host buffers and the clocks seen.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verified draft tokens/s, B=256 γ=5 V=129280, as % of HBM roofline"
+UNIT = "verified draft tokens/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _workload(name):
+    from speculative_decoding_draft_rank_b200 import workloads as wl
+    table = {"tiny": wl.tiny, "qwen_vocab": wl.qwen_vocab, "headline": wl.headline,
+             "saturated": wl.saturated}
+    if name.startswith("long_block_g"):
+        return wl.long_block(int(name[len("long_block_g"):]))
+    return table[name]()
+
+
+def algorithmic_bytes(w, ell_sum):
+    """Bytes a round must move at least once: draft logits, the transition
+    factor W once, the gathered U rows, the hidden states, and the target
+    rows of the admitted prefixes plus one bonus/final row per request."""
+    es = 2 if w.dtype == "bf16" else 4
+    B, G, V, r, d = w.B, w.G, w.V, w.r, w.d
+    parts = {
+        "draft_logits": B * G * V * es,
+        "transition_W": r * V * es,
+        "U_rows": B * G * r * es,
+        "hidden": B * G * d * es,
+        "target_rows": (ell_sum + B) * V * es,
+    }
+    return parts
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample(w, inp, n_req, seed=0):
+    """Time the fp64 oracle (as it stands, one thread) on a bounded sample of
+    the round: confidence and scheduling for the whole batch, drafting and
+    verification for n_req requests.  Returns (verified tokens in the sample,
+    seconds)."""
+    from oracle import oracle
+    from speculative_decoding_draft_rank_b200 import synth
+    rng = np.random.default_rng(seed)
+    idx = np.sort(rng.choice(w.B, size=min(n_req, w.B), replace=False))
+    sub = synth.select_requests(inp, idx)
+    t0 = time.perf_counter()
+    _, S = oracle.confidence(inp.h, inp.w, inp.bias)
+    sch = oracle.schedule(S, w.knots_n, w.knots_t, w.budget, w.mode)
+    dr = oracle.draft(sub.L, sub.U, sub.W, sub.x0, sub.temp, sub.u_draft.astype(np.float64))
+    oracle.verify(sub.Tlog, sub.L, sub.U, sub.W, sub.x0, dr.x, sub.temp, sub.u_accept.astype(np.float64),
+                  sub.u_final.astype(np.float64), sch.ell[idx])
+    dt = time.perf_counter() - t0
+    return int(sch.ell[idx].sum()), dt, len(idx)
+
+
+def run_reference(args):
+    """The reference arm: the oracle on the host cores, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = _workload(args.workload)
+    inp = w.inputs()
+    n_req = args.reference_requests
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, max(1, n_req // 8), seed=1)
+    toks, secs = 0, 0.0
+    for s in range(args.steps):
+        t, dt, n = oracle_sample(w, inp, n_req, seed=100 + s)
+        toks += t
+        secs += dt
+    value = toks / secs if secs > 0 else 0.0
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "G": w.G, "V": w.V, "r": w.r, "d": w.d},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{n_req} requests per step (draft+verify), whole-batch confidence+schedule"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="headline")
+    ap.add_argument("--oracle-requests", type=int, default=64,
+                    help="requests drafted+verified by the oracle for the CPU baseline leg")
+    ap.add_argument("--reference-requests", type=int, default=8,
+                    help="requests per step of the reference arm (the oracle)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_draft_rank_b200.round import DeviceRound
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = _workload(args.workload)
+    w.seed = rank  # every engine drafts its own batch
+    inp = w.inputs()
+    dr = DeviceRound(inp, w.knots_n, w.knots_t, w.budget, w.mode, device=dev, pinned_host=True)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    # Warm up eagerly once (library attributes, lazy module loads), then capture.
+    with torch.cuda.stream(stream):
+        dr.run(stream)
+    torch.cuda.synchronize()
+    from speculative_decoding_draft_rank_b200 import _lib
+    t, o = dr.t, dr.o
+    stages = [
+        lambda: _lib.dspark_draft_markov(t["L"], t["U"], t["Wt"], t["x0"], t["temp"], t["u_draft"], dr.ws,
+                                         o["x"], o["pd_x"], o["rowmax"], o["rowsum"]),
+        lambda: _lib.dspark_confidence(t["h"], t["w"], float(inp.bias), t["tau"], o["c"], o["S"]),
+        lambda: _lib.dspark_schedule(o["S"], t["knots_n"], t["knots_t"], dr.budget, dr.mode, dr.ws, o["ell"],
+                                     o["n_adm"], o["theta"], o["order"]),
+        lambda: _lib.dspark_verify(t["Tlog"], t["L"], t["U"], t["Wt"], t["x0"], o["x"], o["pd_x"], o["rowmax"],
+                                   o["rowsum"], t["temp"], t["u_accept"], t["u_final"], o["ell"], dr.ws,
+                                   o["acc"], o["tokens"], o["nout"], o["pt_x"]),
+    ]
+    graph = torch.cuda.CUDAGraph()          # the whole round: the timed unit
+    with torch.cuda.graph(graph, stream=stream):
+        for f in stages:
+            f()
+    stage_graphs = []                       # one graph per stage: the breakdown
+    for f in stages:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            f()
+        stage_graphs.append(g)
+
+    launches_per_round = 1 + 2 * w.G + 1 + 1 + 5
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            graph.replay()
+    torch.cuda.synchronize()
+    barrier()
+
+    step_ms, stage_ms = [], [[] for _ in range(4)]
+    ell_sum = int(dr.o["ell"].sum().item())
+    nout_sum = int(dr.o["nout"].sum().item())
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier()
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                flush.zero_()
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                e1.synchronize()
+                step_ms.append(e0.elapsed_time(e1))
+        torch.cuda.synchronize()
+        barrier()
+    # Stage breakdown (not the headline): each stage's graph between events.
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.steps // 2)):
+            flush.zero_()
+            for j, g in enumerate(stage_graphs):
+                ev[j].record(stream)
+                g.replay()
+            ev[4].record(stream)
+            ev[4].synchronize()
+            for j in range(4):
+                stage_ms[j].append(ev[j].elapsed_time(ev[j + 1]))
+    torch.cuda.synchronize()
+    status = dr.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x}")
+
+    ms = statistics.mean(step_ms)
+    if world > 1:
+        tt = torch.tensor([ms, float(ell_sum), float(nout_sum)], device=dev, dtype=torch.float64)
+        gathered = [torch.zeros_like(tt) for _ in range(world)]
+        dist.all_gather(gathered, tt)
+        ms = max(float(g[0]) for g in gathered)
+        ell_tot = sum(float(g[1]) for g in gathered)
+        nout_tot = sum(float(g[2]) for g in gathered)
+    else:
+        ell_tot, nout_tot = float(ell_sum), float(nout_sum)
+    value = ell_tot / (ms * 1e-3)
+
+    # End to end through the public API: per-round inputs from pinned host
+    # memory, the round, and the emitted tokens back to pinned host memory.
+    e2e_ms = []
+    per_round_inputs = ("L", "Tlog", "h", "x0", "temp", "u_draft", "u_accept", "u_final")
+    h2d = sum(dr.host[k].numel() * dr.host[k].element_size() for k in per_round_inputs)
+    d2h = dr.d2h_bytes()
+    with torch.cuda.stream(stream):
+        for i in range(max(2, args.steps // 2) + 1):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for k in per_round_inputs:
+                dr.t[k].copy_(dr.host[k], non_blocking=True)
+            dr.run(stream)
+            dr.download(stream)
+            e1.record(stream)
+            stream.synchronize()
+            if i > 0:
+                e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+    if world > 1:
+        tt = torch.tensor([e2e], device=dev, dtype=torch.float64)
+        gathered = [torch.zeros_like(tt) for _ in range(world)]
+        dist.all_gather(gathered, tt)
+        e2e = max(float(g[0]) for g in gathered)
+
+    hbm_gbs, bf16_tf, peak_kind = _peaks()
+    parts = algorithmic_bytes(w, ell_sum)
+    round_bytes = sum(parts.values())
+    stage_means = [statistics.mean(s) for s in stage_ms]
+    dom = int(np.argmax(stage_means))
+    stage_names = ["draft", "confidence", "schedule", "verify"]
+    stage_bytes = [parts["draft_logits"] + parts["transition_W"] + parts["U_rows"], parts["hidden"],
+                   w.B * w.G * 8, parts["target_rows"]]
+    ach = stage_bytes[dom] / (stage_means[dom] * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, one batch per rank)",
+        "config": {"workload": w.name, "B": w.B, "G": w.G, "V": w.V, "r": w.r, "d": w.d,
+                   "l2_flush": "256 MiB write before every timed round", "graph_replay": True,
+                   "parallelism": f"{world} independent engines"},
+        "round": {"admitted_draft_tokens": ell_sum, "emitted_tokens": nout_sum,
+                  "rounds_per_s": world * 1e3 / ms, "emitted_tokens_per_s": nout_tot / (ms * 1e-3),
+                  "algorithmic_bytes": round_bytes,
+                  "hbm_roofline_frac": (round_bytes / (ms * 1e-3) / 1e9) / hbm_gbs,
+                  "stage_ms": dict(zip(stage_names, stage_means))},
+        "roofline": {"kernel": f"{stage_names[dom]} stage", "bound": "hbm", "achieved": ach,
+                     "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs, "traffic": None,
+                     "peak_source": peak_kind},
+        "e2e": {"value": ell_tot / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
+        "gpu_launches": launches_per_round * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        t, secs, n = oracle_sample(w, inp, args.oracle_requests)
+        line["cpu_baseline"] = {"value": t / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+                                "sample": f"{n} of {w.B} requests drafted+verified, whole-batch "
+                                          f"confidence+schedule, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line))
+    graph.reset()
+    for g in stage_graphs:
+        g.reset()
+    del graph, stage_graphs
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -17,7 +17,8 @@ dspark_status check_common(int B, int G, int V, int r, int dtype) {
     if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
     if (B < 1 || B > 4096 || G < 1 || G > 16 || V < 2 || V > (1 << 20) || r < 1 || r > 512)
         return DSPARK_ERR_INVALID_ARG;
-    if (dtype == DSPARK_BF16 && (r % 16) != 0) return DSPARK_ERR_INVALID_ARG;
+    // bf16 rows are moved by TMA: 16-byte row pitches for the logits and factors.
+    if (dtype == DSPARK_BF16 && ((r % 16) != 0 || (V % 8) != 0)) return DSPARK_ERR_INVALID_ARG;
     return DSPARK_OK;
 }
 

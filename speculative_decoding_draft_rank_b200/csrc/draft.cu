@@ -226,28 +226,31 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
         const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
         for (int k = tid; k < r; k += blockDim.x) urow[k] = ld_elem(U, (size_t)prev * r + k);
         __syncthreads();
+        // tpc threads (consecutive lanes) share one column's dot product.
         const int c0 = ts * TN;
+        const int tpc = blockDim.x / TN;
+        const int cj = tid / tpc, part = tid % tpc;
+        const int col = c0 + cj;
+        const bool mine = part == 0 && col < V;
+        float dl = 0.f;
+        if (col < V)
+            for (int k = part; k < r; k += tpc) dl = fmaf(urow[k], ld_elem(Wt, (size_t)col * r + k), dl);
+        for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
         float e = 0.f;
-        const int col = c0 + tid;
-        if (tid < TN && col < V) {
-            float dl = 0.f;
-            for (int k = 0; k < r; ++k) dl = fmaf(urow[k], ld_elem(Wt, (size_t)col * r + k), dl);
-            float l = ld_elem(L, ro * V + col);
-            e = exp_e(((l - M) + dl) * invT);
-        }
+        if (mine) e = exp_e(((ld_elem(L, ro * V + col) - M) + dl) * invT);
         float tot;
         float inc = block_incl_scan(e, red, &tot);
-        int xs = (tid < TN && col < V && inc > rem) ? col : 0x7fffffff;
+        int xs = (mine && inc > rem) ? col : 0x7fffffff;
         xs = block_min_i(xs, redi);
         if (xs == 0x7fffffff) {  // the tile's recomputed mass fell short: last positive
-            int lc = (e > 0.f) ? col : -1;
+            int lc = (mine && e > 0.f) ? col : -1;
             xs = -block_min_i(-lc, redi);
             if (xs < 0) xs = min(c0 + TN, V) - 1;
         }
         x = xs;
         // p_d(x) from the recomputed value of the chosen column.
         __shared__ float ex_s;
-        if (col == x) ex_s = e;
+        if (mine && col == x) ex_s = e;
         __syncthreads();
         pd = ex_s / Z;
     }
@@ -341,15 +344,3 @@ cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
 
 }  // namespace dspark
 
-namespace dspark {
-// Interim bf16 tile launcher on CUDA cores (same tile width as the tensor-core kernel).
-cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
-    static_assert(kTcTileN == kSimtCols, "interim path shares the tile width");
-    dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
-    draft_tile_simt<__nv_bfloat16><<<grid, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16 *>(a.L), static_cast<const __nv_bfloat16 *>(a.U),
-        static_cast<const __nv_bfloat16 *>(a.Wt), a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos,
-        w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
-    return cudaGetLastError();
-}
-}  // namespace dspark

@@ -8,8 +8,8 @@ namespace dspark {
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Column-tile width of the bf16 (tensor-core) drafting and residual kernels.
-constexpr int kTcTileN = 256;
+// Columns per partial (max, sum, argmax) of the bf16 tensor-core drafting kernel.
+constexpr int kTcTileN = 64;
 
 // ----------------------------------------------------------------- drafting
 struct DraftArgs {

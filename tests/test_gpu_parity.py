@@ -43,7 +43,8 @@ PROFILE = (np.array([0, 20, 60], np.int32), np.array([10.0, 11.0, 14.0]))
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("B,G,V,r,d", [(37, 5, 5000, 32, 96), (9, 3, 1283, 16, 40), (64, 8, 3072, 64, 256)])
+@pytest.mark.parametrize("B,G,V,r,d", [(37, 5, 5000, 32, 96), (9, 3, 1288, 16, 40), (64, 8, 3072, 64, 256),
+                                       (130, 4, 9000, 256, 128), (200, 2, 2056, 80, 64)])
 def test_round_parity_small(dtype, B, G, V, r, d):
     temps = np.tile(np.float32([1.0, 0.0, 0.6, 1.2]), B)[:B]
     inp, dr = _round(B, G, V, r, d, dtype, seed=B + V, knots_n=PROFILE[0], knots_t=PROFILE[1], temps=temps)
@@ -65,7 +66,8 @@ def test_verify_everything_and_nothing(dtype):
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_tiny_vocab_and_single_request(dtype):
-    for (B, G, V) in [(1, 1, 2), (3, 2, 7), (1, 16, 300)]:
+    shapes = [(1, 1, 2), (3, 2, 7), (1, 16, 300)] if dtype == "f32" else [(1, 1, 8), (3, 2, 16), (1, 16, 304)]
+    for (B, G, V) in shapes:
         inp, dr = _round(B, G, V, 16, 8, dtype, seed=V, knots_n=np.array([0], np.int32),
                          knots_t=np.array([1.0]), hot=1)
         _check_round(inp, dr, np.array([0], np.int32), np.array([1.0]), -1, 1)

@@ -150,8 +150,11 @@ __global__ void gather_rows_bf16(const __nv_bfloat16 *__restrict__ U, const int3
 }
 
 // ---------------------------------------------------------------------------
-// Finalize: one CTA (kFinThreads threads) per request row.
-constexpr int kFinThreads = 512;
+// Finalize: one CTA of kFinThreads threads per request row.  Thread t owns the
+// contiguous tiles [t K, t K + K): one block max, one block scan of the
+// threads' scaled tile sums, then the thread whose range holds u Z walks its
+// K tiles to the crossing tile, which the block recomputes column by column.
+constexpr int kFinThreads = 256;
 
 template <typename T>
 __global__ void __launch_bounds__(kFinThreads) draft_finalize(
@@ -164,28 +167,33 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
     __nv_bfloat16 *__restrict__ Enext, WsHeader *hdr)
 {
     extern __shared__ float fin_smem[];
-    float *pref = fin_smem;                 // [nTiles] inclusive tile prefixes
-    float *urow = fin_smem + nTiles;        // [r] U[x_{i-1}] row
+    float *urow = fin_smem;                 // [r] U[x_{i-1}] row
     __shared__ float red[33];
     __shared__ int redi[33];
-    __shared__ float carry_s;
+    __shared__ int ts_s;
+    __shared__ float rem_s, ex_s;
 
     const int b = blockIdx.x, tid = threadIdx.x;
     const size_t ro = (size_t)b * G + pos;
     const float *pm = part_m + (size_t)b * nTiles;
     const float *ps = part_s + (size_t)b * nTiles;
     const float Tb = sane_temp(temp[b], hdr);
+    const int K = (nTiles + blockDim.x - 1) / blockDim.x;
+    const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
+
+    // Start fetching the previous token's U row; it is only needed for T > 0.
+    const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
 
     float m = -INFINITY;
-    for (int t = tid; t < nTiles; t += blockDim.x) m = fmaxf(m, pm[t]);
+    for (int t = t0; t < t1; ++t) m = fmaxf(m, pm[t]);
     const float M = block_max(m, red);
 
     int x;
     float pd, Z;
     if (Tb == 0.f) {
         int first = 0x7fffffff;
-        for (int t = tid; t < nTiles; t += blockDim.x)
-            if (pm[t] == M) first = min(first, t);
+        for (int t = t0; t < t1; ++t)
+            if (pm[t] == M) { first = t; break; }
         first = block_min_i(first, redi);
         if (first >= nTiles) first = 0;  // no tile matched (non-finite inputs)
         x = part_a[(size_t)b * nTiles + first];
@@ -193,53 +201,51 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
         pd = 1.f;
         Z = 1.f;
     } else {
-        const float invT = 1.f / Tb;
-        // Inclusive prefix over the scaled tile sums, in tile order.
-        if (tid == 0) carry_s = 0.f;
-        __syncthreads();
-        for (int t0 = 0; t0 < nTiles; t0 += blockDim.x) {
-            int t = t0 + tid;
-            float w = t < nTiles ? ps[t] * exp_e((pm[t] - M) * invT) : 0.f;
-            float tot;
-            float inc = block_incl_scan(w, red, &tot);
-            float c = carry_s;
-            if (t < nTiles) pref[t] = c + inc;
-            __syncthreads();
-            if (tid == 0) carry_s = c + tot;
-            __syncthreads();
-        }
-        Z = carry_s;
-        const float target = u_draft[ro] * Z;
-        int ts = 0x7fffffff;
-        for (int t = tid; t < nTiles; t += blockDim.x)
-            if (pref[t] > target) ts = min(ts, t);
-        ts = block_min_i(ts, redi);
-        if (ts == 0x7fffffff) {  // rounding left u Z at the top: last tile with mass
-            int lt = -1;
-            for (int t = tid; t < nTiles; t += blockDim.x)
-                if (ps[t] > 0.f) lt = max(lt, t);
-            ts = -block_min_i(-lt, redi);
-            if (ts < 0) ts = nTiles - 1;
-        }
-        const float rem = target - (ts > 0 ? pref[ts - 1] : 0.f);
-        // Recompute the chosen tile: Delta on CUDA cores for its TN columns.
-        const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
+        const float cexp = kLog2e / Tb;
         for (int k = tid; k < r; k += blockDim.x) urow[k] = ld_elem(U, (size_t)prev * r + k);
+        float loc = 0.f;
+        for (int t = t0; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
+        float tot;
+        const float incl = block_incl_scan(loc, red, &tot);   // also publishes urow
+        Z = tot;
+        const float target = u_draft[ro] * Z;
+        const float before = incl - loc;
+        // The first thread whose inclusive prefix passes u Z owns the crossing
+        // (the last thread with mass if rounding left u Z at the top).
+        int owner = (incl > target && loc > 0.f) ? tid : 0x7fffffff;
+        owner = block_min_i(owner, redi);
+        if (owner == 0x7fffffff) {
+            owner = -block_min_i(loc > 0.f ? -tid : 1, redi);
+            if (owner < 0) owner = 0;
+        }
+        if (tid == owner) {
+            float run = before, run_last = before;
+            int ts = -1, last = t1 - 1;
+            for (int t = t0; t < t1; ++t) {
+                const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
+                if (run + wt > target) { ts = t; break; }
+                if (wt > 0.f) { last = t; run_last = run; }
+                run += wt;
+            }
+            if (ts < 0) { ts = last; run = run_last; }
+            ts_s = max(ts, 0);
+            rem_s = target - run;
+        }
         __syncthreads();
-        // tpc threads (consecutive lanes) share one column's dot product.
+        const int ts = ts_s;
+        const float rem = rem_s;
+        // Recompute the chosen tile: tpc consecutive threads share one column.
         const int c0 = ts * TN;
         const int tpc = blockDim.x / TN;
-        const int cj = tid / tpc, part = tid % tpc;
-        const int col = c0 + cj;
+        const int col = c0 + tid / tpc, part = tid % tpc;
         const bool mine = part == 0 && col < V;
         float dl = 0.f;
-        if (col < V)
-            for (int k = part; k < r; k += tpc) dl = fmaf(urow[k], ld_elem(Wt, (size_t)col * r + k), dl);
+        if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
         for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
         float e = 0.f;
-        if (mine) e = exp_e(((ld_elem(L, ro * V + col) - M) + dl) * invT);
-        float tot;
-        float inc = block_incl_scan(e, red, &tot);
+        if (mine) e = fast_exp2(((ld_elem(L, ro * V + col) - M) + dl) * cexp);
+        float ttot;
+        const float inc = block_incl_scan(e, red, &ttot);
         int xs = (mine && inc > rem) ? col : 0x7fffffff;
         xs = block_min_i(xs, redi);
         if (xs == 0x7fffffff) {  // the tile's recomputed mass fell short: last positive
@@ -248,8 +254,8 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
             if (xs < 0) xs = min(c0 + TN, V) - 1;
         }
         x = xs;
-        // p_d(x) from the recomputed value of the chosen column.
-        __shared__ float ex_s;
+        if (tid == 0) ex_s = 0.f;
+        __syncthreads();
         if (mine && col == x) ex_s = e;
         __syncthreads();
         pd = ex_s / Z;
@@ -302,7 +308,7 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
 template <typename T>
 static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st,
                                    __nv_bfloat16 *Enext) {
-    size_t smem = sizeof(float) * ((size_t)w.nTiles + a.r);
+    size_t smem = sizeof(float) * (size_t)a.r;
     auto kern = draft_finalize<T>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -58,6 +58,20 @@ struct VerifyArgs {
     float *pt_x_out;
 };
 size_t verify_ws_bytes(int B, int G, int V, int r, int dtype);
+
+// Residual pass of bf16 verification on the tensor cores: rows are the
+// queued rejections (count on the device), A operand their gathered U rows.
+struct ResidualTcArgs {
+    const void *Wt;
+    const __nv_bfloat16 *E, *L, *Tlog;
+    const float *temp, *rowmax, *rowsum, *res_mt, *res_zt;
+    const int32_t *res_b, *res_k;
+    const uint32_t *nrows;
+    int B, G, V, r, nParts;
+    float *rp;
+    WsHeader *hdr;
+};
+cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st);
 cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st);
 
 }  // namespace dspark

@@ -25,13 +25,16 @@
 //               recomputed and scanned to the replacement token.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tc.cuh"
 
 namespace dspark {
 
 constexpr int kChunk = 8192;          // columns per row work item
 constexpr int kRowThreads = 256;      // threads of the row and decide kernels
 constexpr int kResRows = 32;          // queued rows per residual tile CTA
-constexpr int kResCols = 256;         // columns per residual tile
+constexpr int kResCols = 256;         // columns per residual tile (fp32, CUDA cores)
+
+__host__ __device__ inline int res_cols(int dtype) { return dtype == DSPARK_BF16 ? kTcTileN : kResCols; }
 
 struct VerifyWs {
     WsHeader *hdr;             // pad[0] = row count, pad[1] = residual count
@@ -43,13 +46,15 @@ struct VerifyWs {
     int32_t *res_k;            // [B] rejected position (0-based)
     float *res_mt, *res_zt;    // [B] target row max / Z of the rejected row
     float *rp;                 // [B*nResTiles] residual tile sums
-    int nChunks, nResTiles;
+    __nv_bfloat16 *E;          // [round_up(B,128), r] gathered U rows of the queue (bf16)
+    int nChunks, nResTiles, resCols;
 };
 
-static VerifyWs carve_verify_ws(void *ws, int B, int G, int V) {
+static VerifyWs carve_verify_ws(void *ws, int B, int G, int V, int r, int dtype) {
     VerifyWs w;
     w.nChunks = (V + kChunk - 1) / kChunk;
-    w.nResTiles = (V + kResCols - 1) / kResCols;
+    w.resCols = res_cols(dtype);
+    w.nResTiles = (V + w.resCols - 1) / w.resCols;
     const size_t R = (size_t)B * (G + 1);
     char *p = static_cast<char *>(ws);
     w.hdr = reinterpret_cast<WsHeader *>(p); p += sizeof(WsHeader);
@@ -63,14 +68,18 @@ static VerifyWs carve_verify_ws(void *ws, int B, int G, int V) {
     w.res_mt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
     w.res_zt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
     w.rp = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * w.nResTiles);
+    w.E = nullptr;
+    if (dtype == DSPARK_BF16) w.E = reinterpret_cast<__nv_bfloat16 *>(p);
     return w;
 }
 
-size_t verify_ws_bytes(int B, int G, int V, int, int) {
-    const int nChunks = (V + kChunk - 1) / kChunk, nResTiles = (V + kResCols - 1) / kResCols;
+size_t verify_ws_bytes(int B, int G, int V, int r, int dtype) {
+    const int nChunks = (V + kChunk - 1) / kChunk, rc = res_cols(dtype), nResTiles = (V + rc - 1) / rc;
     const size_t R = (size_t)B * (G + 1);
-    return sizeof(WsHeader) + align256(4 * R) + align256(4 * (B + 1)) + 3 * align256(4 * R * nChunks) +
-           4 * align256(4 * (size_t)B) + align256(4 * (size_t)B * nResTiles);
+    size_t bytes = sizeof(WsHeader) + align256(4 * R) + align256(4 * (B + 1)) + 3 * align256(4 * R * nChunks) +
+                   4 * align256(4 * (size_t)B) + align256(4 * (size_t)B * nResTiles);
+    if (dtype == DSPARK_BF16) bytes += align256(2 * (size_t)round_up(B, 128) * r);
+    return bytes;
 }
 
 // Eight consecutive elements starting at index i of a row (bounds-checked;
@@ -136,68 +145,237 @@ __global__ void verify_plan(const int32_t *__restrict__ ell, int B, int G, Verif
 }
 
 // ----------------------------------------------------------------- rows
+// One work item = one 8192-column chunk of one admitted target row.  Each
+// thread owns 32 columns (4 groups of 8 contiguous columns), loads them with
+// 16-byte streaming loads one item ahead of the one it reduces, and keeps an
+// online (max, sum of exp((t - max) / T)); the greedy argmax is only tracked
+// for T = 0 rows.  One block merge per item writes the chunk partial.
+template <typename T>
+__device__ __forceinline__ void rows_load(const T *__restrict__ Tlog, const VerifyWs &w, int G, int V, int item,
+                                          float (&v)[4][8]) {
+    const int j = item / w.nChunks, c = item - j * w.nChunks;
+    const int rk = w.rows[j], b = rk >> 5, k = rk & 31;
+    const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
+    const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int i = c0 + (q * kRowThreads + threadIdx.x) * 8;
+        if (i < c1) {
+            load8(row, i, c1, v[q]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[q][e] = -INFINITY;
+        }
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__ Tlog,
                                                            const float *__restrict__ temp, int G,
                                                            int V, VerifyWs w) {
-    __shared__ float rv[8];
-    __shared__ int ri[8];
+    __shared__ float rm[8], rs[8];
+    __shared__ int ra[8];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
     const int nwork = nrows * w.nChunks;
-    for (int item = blockIdx.x; item < nwork; item += gridDim.x) {
+    int item = blockIdx.x;
+    if (item >= nwork) return;
+    float cur[4][8], nxt[4][8];
+    rows_load(Tlog, w, G, V, item, cur);
+    for (; item < nwork; item += gridDim.x) {
+        const int next = item + gridDim.x;
+        if (next < nwork) rows_load(Tlog, w, G, V, next, nxt);
         const int j = item / w.nChunks, c = item - j * w.nChunks;
-        const int rk = w.rows[j], b = rk >> 5, k = rk & 31;
+        const int b = w.rows[j] >> 5;
         float Tb = temp[b];
         Tb = Tb >= 0.f ? Tb : 0.f;
-        const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
-        const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
-        const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
-        float v[4][8];
+        const float cexp = Tb > 0.f ? kLog2e / Tb : 0.f;
         float m = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m = fmaxf(m, cur[q][e]);
         int am = 0x7fffffff;
+        float s = 0.f;
+        if (Tb == 0.f) {   // whole item is one row: the branch is block-uniform
+#pragma unroll
+            for (int q = 3; q >= 0; --q)
+#pragma unroll
+                for (int e = 7; e >= 0; --e)
+                    if (cur[q][e] == m) am = c * kChunk + (q * kRowThreads + tid) * 8 + e;
+        } else if (m > -INFINITY) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s += fast_exp2((cur[q][e] - m) * cexp);
+        }
+        // Warp merge of (m, s, argmax), then across the 8 warps.
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, m, o);
+            const float os = __shfl_xor_sync(0xffffffffu, s, o);
+            const int oa = __shfl_xor_sync(0xffffffffu, am, o);
+            const float nm = fmaxf(m, om);
+            if (cexp > 0.f)
+                s = (m > -INFINITY ? s * fast_exp2((m - nm) * cexp) : 0.f) +
+                    (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
+            if (om > m || (om == m && oa < am)) am = oa;
+            m = nm;
+        }
+        if (lane == 0) { rm[wid] = m; rs[wid] = s; ra[wid] = am; }
+        __syncthreads();
+        if (tid == 0) {
+            float M = rm[0];
+            int A = ra[0];
+            for (int q = 1; q < 8; ++q)
+                if (rm[q] > M || (rm[q] == M && ra[q] < A)) { M = rm[q]; A = ra[q]; }
+            float S = 0.f;
+            if (cexp > 0.f)
+                for (int q = 0; q < 8; ++q)
+                    if (rm[q] > -INFINITY) S += rs[q] * fast_exp2((rm[q] - M) * cexp);
+            const size_t o = (size_t)j * w.nChunks + c;
+            w.cm[o] = M;
+            w.cs[o] = S;
+            w.ca[o] = A;
+        }
+        __syncthreads();
+        if (next < nwork) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) cur[q][e] = nxt[q][e];
+        }
+    }
+}
+
+// bf16 rows: each chunk is one contiguous 16-byte-aligned run, so thread 0
+// streams the CTA's work items into a 3-stage shared-memory ring with bulk
+// async copies (evict-first), keeping up to three 16 KB chunks in flight per
+// CTA while the block reduces the oldest.  Waits are bounded.
+constexpr int kRowStages = 3;
+
+__global__ void __launch_bounds__(kRowThreads) verify_rows_bulk(const __nv_bfloat16 *__restrict__ Tlog,
+                                                                const float *__restrict__ temp, int G, int V,
+                                                                VerifyWs w) {
+    extern __shared__ __align__(128) unsigned char rows_smem[];
+    __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(rows_smem);   // [kRowStages][kChunk]
+    __shared__ __align__(8) uint64_t full[kRowStages];
+    __shared__ float rm[8], rs[8];
+    __shared__ int ra[8];
+    __shared__ int abort_s;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
+    const int nwork = nrows * w.nChunks;
+    if ((int)blockIdx.x >= nwork) return;
+    const int my_items = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    auto issue = [&](int k) {  // k-th item of this CTA into stage k % kRowStages
+        const int item = blockIdx.x + k * gridDim.x;
+        const int j = item / w.nChunks, c = item - j * w.nChunks;
+        const int rk = w.rows[j], b = rk >> 5, kk = rk & 31;
+        const int c0 = c * kChunk, n = min(V, c0 + kChunk) - c0;
+        const __nv_bfloat16 *src = Tlog + ((size_t)b * (G + 1) + kk) * V + c0;
+        uint64_t *bar = &full[k % kRowStages];
+        tc::mbar_arrive_expect_tx(bar, (uint32_t)n * 2);
+        asm volatile(
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+            " [%0], [%1], %2, [%3], %4;" ::"r"(tc::smem_u32(stage + (size_t)(k % kRowStages) * kChunk)),
+            "l"(src), "r"(n * 2), "r"(tc::smem_u32(bar)), "l"(tc::policy_evict_first())
+            : "memory");
+    };
+    if (tid == 0) {
+        for (int q = 0; q < kRowStages; ++q) tc::mbar_init(&full[q], 1);
+        tc::fence_barrier_init();
+        abort_s = 0;
+        for (int k = 0; k < kRowStages && k < my_items; ++k) issue(k);
+    }
+    __syncthreads();
+    for (int k = 0; k < my_items; ++k) {
+        const int item = blockIdx.x + k * gridDim.x;
+        const int j = item / w.nChunks, c = item - j * w.nChunks;
+        const int b = w.rows[j] >> 5;
+        float Tb = temp[b];
+        Tb = Tb >= 0.f ? Tb : 0.f;
+        const float cexp = Tb > 0.f ? kLog2e / Tb : 0.f;
+        const int c0 = c * kChunk, n = min(V, c0 + kChunk) - c0;
+        const bool ok = tc::mbar_wait_bounded(&full[k % kRowStages], (k / kRowStages) & 1, &abort_s,
+                                              2000000000LL);
+        if (!__syncthreads_and(ok)) {
+            if (tid == 0) flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
+            break;
+        }
+        const __nv_bfloat16 *st = stage + (size_t)(k % kRowStages) * kChunk;
+        float v[4][8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int i = c0 + (q * kRowThreads + tid) * 8;
-            if (i < c1) {
-                load8(row, i, c1, v[q]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    if (v[q][e] > m) { m = v[q][e]; am = i + e; }
+            const int i = (q * kRowThreads + tid) * 8;
+            if (i < n) {
+                const uint4 r4 = *reinterpret_cast<const uint4 *>(st + i);
+                v[q][0] = bf16lo(r4.x); v[q][1] = bf16hi(r4.x); v[q][2] = bf16lo(r4.y); v[q][3] = bf16hi(r4.y);
+                v[q][4] = bf16lo(r4.z); v[q][5] = bf16hi(r4.z); v[q][6] = bf16lo(r4.w); v[q][7] = bf16hi(r4.w);
             } else {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) v[q][e] = -INFINITY;
             }
         }
-        float wm = m;
-        int wa = am;
-        warp_argmax(wm, wa);
-        if (lane == 0) { rv[wid] = wm; ri[wid] = wa; }
-        __syncthreads();
-        float M = rv[0];
-        int A = ri[0];
-        for (int q = 1; q < 8; ++q)
-            if (rv[q] > M || (rv[q] == M && ri[q] < A)) { M = rv[q]; A = ri[q]; }
-        __syncthreads();
+        float m = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m = fmaxf(m, v[q][e]);
+        int am = 0x7fffffff;
         float s = 0.f;
-        if (invT > 0.f) {
+        if (Tb == 0.f) {   // the item is one row: block-uniform branch
+#pragma unroll
+            for (int q = 3; q >= 0; --q)
+#pragma unroll
+                for (int e = 7; e >= 0; --e)
+                    if (v[q][e] == m) am = c0 + (q * kRowThreads + tid) * 8 + e;
+        } else if (m > -INFINITY) {
 #pragma unroll
             for (int q = 0; q < 4; ++q)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) s += exp_e((v[q][e] - M) * invT);
+                for (int e = 0; e < 8; ++e) s += fast_exp2((v[q][e] - m) * cexp);
         }
-        s = warp_sum(s);
-        if (lane == 0) rv[wid] = s;
-        __syncthreads();
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, m, o);
+            const float os = __shfl_xor_sync(0xffffffffu, s, o);
+            const int oa = __shfl_xor_sync(0xffffffffu, am, o);
+            const float nm = fmaxf(m, om);
+            if (cexp > 0.f)
+                s = (m > -INFINITY ? s * fast_exp2((m - nm) * cexp) : 0.f) +
+                    (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
+            if (om > m || (om == m && oa < am)) am = oa;
+            m = nm;
+        }
+        if (lane == 0) { rm[wid] = m; rs[wid] = s; ra[wid] = am; }
+        __syncthreads();   // also: every thread is done with this stage
         if (tid == 0) {
-            float t = 0.f;
-            for (int q = 0; q < 8; ++q) t += rv[q];
+            float M = rm[0];
+            int A = ra[0];
+            for (int q = 1; q < 8; ++q)
+                if (rm[q] > M || (rm[q] == M && ra[q] < A)) { M = rm[q]; A = ra[q]; }
+            float S = 0.f;
+            if (cexp > 0.f)
+                for (int q = 0; q < 8; ++q)
+                    if (rm[q] > -INFINITY) S += rs[q] * fast_exp2((rm[q] - M) * cexp);
             const size_t o = (size_t)j * w.nChunks + c;
             w.cm[o] = M;
-            w.cs[o] = t;
+            w.cs[o] = S;
             w.ca[o] = A;
+            if (k + kRowStages < my_items) {
+                tc::fence_proxy_async_smem();
+                issue(k + kRowStages);
+            }
         }
-        __syncthreads();
+    }
+    // Copies still in flight after a timeout must land before the CTA exits.
+    if (tid == 0 && abort_s) {
+        int none = 0;
+        for (int k = 0; k < my_items && k < kRowStages; ++k) {
+            const int kk = my_items - 1 - k;
+            tc::mbar_wait_bounded(&full[kk % kRowStages], (kk / kRowStages) & 1, &none, 500000000LL);
+        }
     }
 }
 
@@ -284,7 +462,8 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
 // ----------------------------------------------------------------- decide
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) verify_decide(
-    const T *__restrict__ Tlog, const int32_t *__restrict__ x, const float *__restrict__ pd_x,
+    const T *__restrict__ Tlog, const T *__restrict__ U, const int32_t *__restrict__ x0, int r,
+    const int32_t *__restrict__ x, const float *__restrict__ pd_x,
     const float *__restrict__ temp, const float *__restrict__ u_accept,
     const float *__restrict__ u_final, const int32_t *__restrict__ ell, int B, int G, int V,
     VerifyWs w, int32_t *__restrict__ acc_out, int32_t *__restrict__ tokens_out,
@@ -293,7 +472,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     __shared__ int rA[17];
     __shared__ float red[33];
     __shared__ int redi[33];
-    __shared__ int A_s;
+    __shared__ int A_s, slot_s;
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float Tb = sane_temp(temp[b], w.hdr);
     const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
@@ -308,6 +487,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     }
     __syncthreads();
     if (tid == 0) {
+        slot_s = -1;
         int A = 0;
         bool rejected = false;
         for (int k = 0; k < G; ++k) {
@@ -343,10 +523,17 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
             w.res_k[slot] = A;
             w.res_mt[slot] = rM[A];
             w.res_zt[slot] = rZ[A];
+            slot_s = slot;
         }
     }
     __syncthreads();
     const int A = A_s;
+    if (w.E != nullptr && slot_s >= 0) {  // A-operand row U[x_{k*-1}] of the queued rejection
+        const int prev = min(max((A == 0) ? x0[b] : x[(size_t)b * G + A - 1], 0), V - 1);
+        const uint4 *src = reinterpret_cast<const uint4 *>(U + (size_t)prev * r);
+        uint4 *dst = reinterpret_cast<uint4 *>(w.E + (size_t)slot_s * r);
+        for (int q = tid; q < r / 8; q += blockDim.x) dst[q] = src[q];
+    }
     if (Tb > 0.f && A == lb) {  // bonus (fresh token when nothing was admitted)
         const int y = sample_target_row(Tlog, w, j0 + lb, b, lb, G, V, rM[lb], rZ[lb], invT,
                                         u_final[b], red, redi);
@@ -489,24 +676,29 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
         const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
         for (int q = tid; q < r; q += blockDim.x) urow[q] = ld_elem(U, (size_t)prev * r + q);
         __syncthreads();
-        const int c0 = ts * kResCols;
+        // tpc consecutive threads share one column's dot product.
+        const int TN = w.resCols;
+        const int c0 = ts * TN;
+        const int tpc = blockDim.x / TN;
+        const int col = c0 + tid / tpc, part = tid % tpc;
+        const bool mine = part == 0 && col < V;
+        float dl = 0.f;
+        if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
+        for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
         float qv = 0.f;
-        const int col = c0 + tid;
-        if (tid < kResCols && col < V) {
-            float dl = 0.f;
-            for (int q = 0; q < r; ++q) dl = fmaf(urow[q], ld_elem(Wt, (size_t)col * r + q), dl);
+        if (mine) {
             const float pd = exp_e(((ld_elem(L, ro * V + col) - Md) + dl) * invT) / Zd;
             const float pt = exp_e((ld_elem(Tlog, ((size_t)b * (G + 1) + k) * V + col) - Mt) * invT) / Zt;
             qv = fmaxf(pt - pd, 0.f);
         }
         float tot;
         float inc = block_incl_scan(qv, red, &tot);
-        int ys = (tid < kResCols && col < V && qv > 0.f && inc > rem) ? col : 0x7fffffff;
+        int ys = (mine && qv > 0.f && inc > rem) ? col : 0x7fffffff;
         ys = block_min_i(ys, redi);
         if (ys == 0x7fffffff) {
-            int lc = (qv > 0.f) ? col : -1;
+            int lc = (mine && qv > 0.f) ? col : -1;
             ys = -block_min_i(-lc, redi);
-            if (ys < 0) ys = min(c0 + kResCols, V) - 1;
+            if (ys < 0) ys = min(c0 + TN, V) - 1;
         }
         y = ys;
     }
@@ -524,18 +716,36 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int maxwork = a.B * (a.G + 1) * w.nChunks;
-    const int grid = max(1, min(maxwork, sms * 8));
-    verify_rows<T><<<grid, kRowThreads, 0, st>>>(Tl, a.temp, a.G, a.V, w);
+    if (a.dtype == DSPARK_BF16) {
+        const size_t smem = (size_t)kRowStages * kChunk * 2;
+        if ((e = cudaFuncSetAttribute(verify_rows_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        const int grid = max(1, min(maxwork, sms * 4));
+        verify_rows_bulk<<<grid, kRowThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp,
+                                                          a.G, a.V, w);
+    } else {
+        const int grid = max(1, min(maxwork, sms * 8));
+        verify_rows<T><<<grid, kRowThreads, 0, st>>>(Tl, a.temp, a.G, a.V, w);
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    verify_decide<T><<<a.B, kRowThreads, 0, st>>>(Tl, a.x, a.pd_x, a.temp, a.u_accept, a.u_final, a.ell,
+    verify_decide<T><<<a.B, kRowThreads, 0, st>>>(Tl, static_cast<const T *>(a.U), a.x0, a.r, a.x, a.pd_x,
+                                                  a.temp, a.u_accept, a.u_final, a.ell,
                                                   a.B, a.G, a.V, w, a.acc_out, a.tokens_out,
                                                   a.nout_out, a.pt_x_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dim3 rg(w.nResTiles, (a.B + kResRows - 1) / kResRows);
-    residual_tile_simt<T><<<rg, 256, 0, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
-                                              static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax,
-                                              a.rowsum, a.temp, a.G, a.V, a.r, w);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.dtype == DSPARK_BF16) {
+        ResidualTcArgs ra{a.Wt, w.E, static_cast<const __nv_bfloat16 *>(a.L),
+                          static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp, a.rowmax, a.rowsum, w.res_mt,
+                          w.res_zt, w.res_b, w.res_k, &w.hdr->pad[1], a.B, a.G, a.V, a.r, w.nResTiles, w.rp, w.hdr};
+        if ((e = launch_residual_tile_tc(ra, st)) != cudaSuccess) return e;
+    } else {
+        dim3 rg(w.nResTiles, (a.B + kResRows - 1) / kResRows);
+        residual_tile_simt<T><<<rg, 256, 0, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
+                                                  static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax,
+                                                  a.rowsum, a.temp, a.G, a.V, a.r, w);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     const size_t smem = sizeof(float) * ((size_t)w.nResTiles + a.r);
     auto fin = residual_final<T>;
     if (smem > 48 * 1024) {
@@ -550,7 +760,7 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
 }
 
 cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st) {
-    VerifyWs w = carve_verify_ws(ws, a.B, a.G, a.V);
+    VerifyWs w = carve_verify_ws(ws, a.B, a.G, a.V, a.r, a.dtype);
     if (a.dtype == DSPARK_BF16) return launch_verify_t<__nv_bfloat16>(a, w, st);
     return launch_verify_t<float>(a, w, st);
 }

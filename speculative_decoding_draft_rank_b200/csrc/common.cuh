@@ -41,6 +41,15 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p) {
     return r;
 }
 
+// Read-only 16-byte load through L1 (neighbouring pieces of a line hit L1).
+__device__ __forceinline__ uint4 ld_nc16(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 

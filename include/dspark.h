@@ -179,6 +179,39 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
                             float *pt_x_out, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Drafting without a workspace, for callers that cannot allocate device
+ * memory when they draft: e.g. a plugin of an inference engine that receives
+ * only its inputs and outputs at enqueue time (the engine planned all memory
+ * ahead and offers no allocator), or a latency-critical serving loop that must
+ * not call cudaMalloc, which can synchronise the whole device.  The paper has
+ * no counterpart to this entry point; it is an engineering variant of
+ * dspark_draft_markov with identical arguments and results, minus the
+ * workspace.
+ *
+ * Its scratch lives in a file-scope device array of
+ * dspark_draft_noalloc_max_scratch() bytes (8 MiB) that every GPU which loads
+ * this library holds until the process exits.  Rounds whose drafting
+ * workspace (dspark_draft_workspace_size) would exceed that size are rejected
+ * with DSPARK_ERR_WORKSPACE before any work is enqueued; the headline shape
+ * B = 256, V = 129280, r = 256 needs about 6.3 MB.  No call allocates: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  Every call reuses the same array, which keeps the previous call's
+ * contents: the call clears the status word it needs to start at zero, and
+ * the rest is written before it is read.  Calls that may overlap on the GPU
+ * (other streams, other host threads) race on the array and must be
+ * serialised by the caller.  Device-side data errors are clamped as in
+ * dspark_draft_markov but are not reported back. */
+size_t dspark_draft_noalloc_max_scratch(void);
+dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const void *Wt,
+                                          const int32_t *x0, const float *temp,
+                                          const float *u_draft, int B, int G, int V, int r,
+                                          int dtype, int32_t *x_out, float *pd_x_out,
+                                          float *rowmax_out, float *rowsum_out, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Device status word of a workspace: dspark_get_device_status synchronises
  * `stream`, then copies the word to *status_out (0 = no data error since the
  * last clear).  dspark_clear_device_status enqueues a reset of the word. */

@@ -26,7 +26,8 @@ DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
 EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov", "dspark_confidence",
            "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
-           "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status")
+           "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
+           "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc")
 
 
 class DsparkError(RuntimeError):
@@ -67,6 +68,10 @@ def load() -> ctypes.CDLL:
     lib.dspark_get_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.dspark_clear_device_status.restype = _i
     lib.dspark_clear_device_status.argtypes = [_vp, _vp]
+    lib.dspark_draft_noalloc_max_scratch.restype = _sz
+    lib.dspark_draft_noalloc_max_scratch.argtypes = []
+    lib.dspark_draft_markov_noalloc.restype = _i
+    lib.dspark_draft_markov_noalloc.argtypes = [_vp] * 6 + [_i] * 5 + [_vp] * 5
     _lib = lib
     return lib
 
@@ -123,6 +128,19 @@ def dspark_draft_markov(L, U, Wt, x0, temp, u_draft, ws, x_out, pd_x_out, rowmax
     _call("dspark_draft_markov", _ptr(L), _ptr(U), _ptr(Wt), _ptr(x0), _ptr(temp), _ptr(u_draft), B, G, V,
           r, _dtype(L), _ptr(ws), ws.numel() * ws.element_size(), _ptr(x_out), _ptr(pd_x_out),
           _ptr(rowmax_out), _ptr(rowsum_out), _stream(stream))
+
+
+def dspark_draft_noalloc_max_scratch() -> int:
+    return int(load().dspark_draft_noalloc_max_scratch())
+
+
+def dspark_draft_markov_noalloc(L, U, Wt, x0, temp, u_draft, x_out, pd_x_out, rowmax_out, rowsum_out,
+                                stream=None):
+    """Drafting with the library's own fixed scratch instead of a workspace."""
+    B, G, V = L.shape
+    r = U.shape[1]
+    _call("dspark_draft_markov_noalloc", _ptr(L), _ptr(U), _ptr(Wt), _ptr(x0), _ptr(temp), _ptr(u_draft), B,
+          G, V, r, _dtype(L), _ptr(x_out), _ptr(pd_x_out), _ptr(rowmax_out), _ptr(rowsum_out), _stream(stream))
 
 
 def dspark_confidence(h, w, bias, tau, c_out, S_out, stream=None):

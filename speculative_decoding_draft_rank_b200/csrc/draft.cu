@@ -15,8 +15,7 @@
 //   finalize      one CTA per row: combines the tile partials into (max, Z),
 //                 finds the tile where u Z falls by a prefix scan over the
 //                 tile sums, recomputes that one tile's values and scans it to
-//                 the sampled token; writes x_i, p_d(x_i), max, Z and, for the
-//                 tensor-core kernel, the next position's gathered U row.
+//                 the sampled token; writes x_i, p_d(x_i), max and Z.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -138,18 +137,6 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
 }
 
 // ---------------------------------------------------------------------------
-// Gather E[b] = U[x0[b]] (bf16 rows) for the tensor-core kernel's first position.
-__global__ void gather_rows_bf16(const __nv_bfloat16 *__restrict__ U, const int32_t *__restrict__ tok,
-                                 int B, int V, int r, __nv_bfloat16 *__restrict__ E, WsHeader *hdr)
-{
-    int b = blockIdx.x;
-    int t = clamp_token(tok[b], V, hdr);
-    const uint4 *src = reinterpret_cast<const uint4 *>(U + (size_t)t * r);
-    uint4 *dst = reinterpret_cast<uint4 *>(E + (size_t)b * r);
-    for (int j = threadIdx.x; j < r / 8; j += blockDim.x) dst[j] = src[j];
-}
-
-// ---------------------------------------------------------------------------
 // Finalize: one CTA of kFinThreads threads per request row.  Thread t owns the
 // contiguous tiles [t K, t K + K): one block max, one block scan of the
 // threads' scaled tile sums, then the thread whose range holds u Z walks its
@@ -163,8 +150,7 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
     const float *__restrict__ u_draft, int B, int G, int V, int r, int pos, int nTiles, int TN,
     const float *__restrict__ part_m, const float *__restrict__ part_s,
     const int32_t *__restrict__ part_a, int32_t *__restrict__ x_out, float *__restrict__ pd_out,
-    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out,
-    __nv_bfloat16 *__restrict__ Enext, WsHeader *hdr)
+    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out, WsHeader *hdr)
 {
     extern __shared__ float fin_smem[];
     float *urow = fin_smem;                 // [r] U[x_{i-1}] row
@@ -239,11 +225,12 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
         const int tpc = blockDim.x / TN;
         const int col = c0 + tid / tpc, part = tid % tpc;
         const bool mine = part == 0 && col < V;
+        const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
         float dl = 0.f;
         if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
         for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
         float e = 0.f;
-        if (mine) e = fast_exp2(((ld_elem(L, ro * V + col) - M) + dl) * cexp);
+        if (mine) e = fast_exp2(((lval - M) + dl) * cexp);
         float ttot;
         const float inc = block_incl_scan(e, red, &ttot);
         int xs = (mine && inc > rem) ? col : 0x7fffffff;
@@ -266,12 +253,6 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
         rowmax_out[ro] = M;
         rowsum_out[ro] = Z;
     }
-    if (Enext != nullptr) {  // next position's A-operand row for the tensor-core kernel
-        const uint4 *src = reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(U) +
-                                                           (size_t)x * r);
-        uint4 *dst = reinterpret_cast<uint4 *>(Enext + (size_t)b * r);
-        for (int j = tid; j < r / 8; j += blockDim.x) dst[j] = src[j];
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -286,7 +267,6 @@ size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_m
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_s
     bytes += align256(sizeof(int32_t) * (size_t)B * nt);  // part_a
-    if (dtype == DSPARK_BF16) bytes += align256(sizeof(__nv_bfloat16) * (size_t)round_up(B, 128) * r);  // E
     return bytes;
 }
 
@@ -299,54 +279,44 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     w.part_m = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
     w.part_s = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
     w.part_a = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (size_t)B * nt);
-    w.E = nullptr;
-    if (dtype == DSPARK_BF16) w.E = reinterpret_cast<__nv_bfloat16 *>(p);
     w.nTiles = (int)nt;
     return w;
 }
 
 template <typename T>
-static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st,
-                                   __nv_bfloat16 *Enext) {
+static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
     size_t smem = sizeof(float) * (size_t)a.r;
     auto kern = draft_finalize<T>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
     }
-    kern<<<a.B, kFinThreads, smem, st>>>(
-        static_cast<const T *>(a.L), static_cast<const T *>(a.U), static_cast<const T *>(a.Wt), a.x0,
-        a.temp, a.u_draft, a.B, a.G, a.V, a.r, pos, w.nTiles, draft_tile_cols(a.dtype), w.part_m,
-        w.part_s, w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out, Enext, w.hdr);
+    kern<<<a.B, kFinThreads, smem, st>>>(static_cast<const T *>(a.L), static_cast<const T *>(a.U),
+                                         static_cast<const T *>(a.Wt), a.x0, a.temp, a.u_draft, a.B, a.G, a.V,
+                                         a.r, pos, w.nTiles, draft_tile_cols(a.dtype), w.part_m, w.part_s,
+                                         w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out, w.hdr);
     return cudaGetLastError();
 }
 
 cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
     DraftWs w = carve_draft_ws(ws, a.B, a.V, a.r, a.dtype);
     cudaError_t e;
-    if (a.dtype == DSPARK_F32) {
-        dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
-        for (int pos = 0; pos < a.G; ++pos) {
+    for (int pos = 0; pos < a.G; ++pos) {
+        if (a.dtype == DSPARK_F32) {
+            dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
             draft_tile_simt<float><<<grid, 256, 0, st>>>(
                 static_cast<const float *>(a.L), static_cast<const float *>(a.U),
                 static_cast<const float *>(a.Wt), a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos,
                 w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            if ((e = launch_finalize<float>(a, w, pos, st, nullptr)) != cudaSuccess) return e;
+            if ((e = launch_finalize<float>(a, w, pos, st)) != cudaSuccess) return e;
+        } else {
+            // bf16: tensor-core tile kernel (its A rows are U[previous token]).
+            if ((e = launch_draft_tile_tc(a, w, pos, st)) != cudaSuccess) return e;
+            if ((e = launch_finalize<__nv_bfloat16>(a, w, pos, st)) != cudaSuccess) return e;
         }
-        return cudaSuccess;
-    }
-    // bf16: tensor-core tile kernel, A operand gathered into w.E.
-    gather_rows_bf16<<<a.B, 64, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.U), a.x0, a.B, a.V, a.r,
-                                         w.E, w.hdr);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    for (int pos = 0; pos < a.G; ++pos) {
-        if ((e = launch_draft_tile_tc(a, w, pos, st)) != cudaSuccess) return e;
-        __nv_bfloat16 *En = (pos + 1 < a.G) ? w.E : nullptr;
-        if ((e = launch_finalize<__nv_bfloat16>(a, w, pos, st, En)) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }
 
 }  // namespace dspark
-

@@ -7,22 +7,29 @@
 // draft-generation figure): Delta_i = E_i W with E_i[b] = U[x_{i-1}[b]], added
 // to the backbone logits L[i] before the temperature softmax.
 //
-// Persistent, warp-specialised CTA (one per SM), 320 threads, 512 TMEM columns:
-//   warp 0      TMA producer of the B operand: per 128-column tile the
-//               transition-factor tile Wt[n0:n0+128, :] through a ring of
-//               k-block stages (128-byte swizzle, evict-last: W is reused by
-//               every position and m-block).
-//   warp 1      TMEM owner and MMA issuer: 128 x 128 x 16 bf16 MMAs with the A
-//               operand read from TMEM (the CTA's 128 gathered U rows, written
-//               there once) into one of two fp32 accumulators.
-//   warps 2-9   epilogue: first they copy the A rows into TMEM (lane = row),
-//               then each thread owns one row and one 64-column half of every
-//               tile: Delta from TMEM, its row's logits straight from global
-//               memory (loaded one tile ahead), and the 64-column partials.
-// Shared memory only carries the B ring, so the MMA's operand fetch does not
-// compete with the logit stream.  Delta never leaves the SM.  Every mbarrier
-// wait is bounded by a clock budget; on expiry the CTA raises a timeout bit in
-// the status word, drains its own copies and MMAs, frees TMEM and returns.
+// Persistent, warp-specialised CTA (one per SM), 608 threads, 512 TMEM columns.
+// A CTA owns 128 rows and walks 256-column tiles; one 128 x 256 x 16 MMA per
+// K step (a chain of MMAs into one accumulator costs about the same per
+// instruction for N = 128 and N = 256 on this part, so the wide tile doubles
+// tensor throughput).
+//   warp 0      TMA producer of the B operand: the transition-factor tile
+//               Wt[n0:n0+256, :] one 64-deep k-block at a time through a ring
+//               (128-byte swizzle, evict-last: W is reused by every position
+//               and M-block).
+//   warp 1      TMEM owner and MMA issuer: 128 x 256 x 16 bf16 MMAs, A and B
+//               from shared memory, into one of two 256-column fp32
+//               accumulators.
+//   warp 2      TMA producer of the logits L[:, i, :] in 128 x 64 segments
+//               (128-byte swizzle, evict-first; drafting only).
+//   warps 3-18  epilogue: first they write the A operand -- the 128 rows
+//               U[previous token] -- into shared memory in the swizzled
+//               K-major layout; then warp e owns TMEM lane quarter (warp % 4)
+//               and the 64-column segment (e / 4) of every tile: Delta from
+//               TMEM plus the logits from the segment give the 64-column
+//               partials (max, lowest argmax, sum of exp((y - max) / T)).
+// Delta never leaves the SM.  Every mbarrier wait is bounded by a clock
+// budget; on expiry the CTA raises a timeout bit in the status word, drains
+// its own copies and MMAs, frees TMEM and returns.
 #include <algorithm>
 
 #include "common.cuh"
@@ -33,19 +40,37 @@ namespace dspark {
 
 namespace {
 
-constexpr int kM = 128;            // rows (requests) per CTA
-constexpr int kBN = 128;           // MMA N: columns per tile
-constexpr int kPartN = 64;         // partial granularity: columns per epilogue warp
-constexpr int kKB = 64;            // bf16 elements per 128-byte k-block
-constexpr int kStageBytes = kBN * 128;        // one k-block of the B tile
-constexpr int kStages = 8;                    // B ring depth (two tiles at r = 256)
-constexpr int kThreads = 320;
-constexpr int kEpiWarp0 = 2;       // first epilogue warp
-constexpr int kTmemCols = 512;     // A (r/2 columns, <= 256) + two 128-column accumulators
-constexpr int kAccCol0 = 256;
-constexpr long long kWaitBudget = 4000000000LL;  // ~2 s of SM clock
+constexpr int kM = 128;             // rows (requests) per CTA
+constexpr int kBN = 256;            // MMA N: columns per tile
+constexpr int kSeg = 64;            // columns per logit segment = per partial
+constexpr int kSegs = kBN / kSeg;   // 4
+constexpr int kKB = 64;             // bf16 elements per 128-byte k-block
+constexpr int kABlockBytes = kM * 128;     // one k-block of A (16 KB)
+constexpr int kStageBytes = kBN * 128;     // one k-block of B (32 KB)
+constexpr int kSegBytes = kM * kSeg * 2;   // one logit segment (16 KB)
+constexpr int kEpiWarp0 = 3;
+constexpr int kEpiWarps = 16;
+constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;   // 608
+constexpr int kTmemCols = 2 * kBN;                        // two accumulators
+constexpr long long kWaitBudget = 4000000000LL;          // ~2 s of SM clock
 
-constexpr uint32_t kSmemBytes = kStages * kStageBytes + 256 + 1024;  // ring + barriers + base alignment
+struct TcLayout {
+    int nkb, sB, sL;
+    uint32_t a_off, b_off, l_off, bar_off, total;
+};
+
+__host__ __device__ inline TcLayout tc_layout(int r) {
+    TcLayout t;
+    t.nkb = (r + kKB - 1) / kKB;
+    t.sB = t.nkb <= 4 ? 3 : 2;       // B ring depth
+    t.sL = t.nkb <= 4 ? 4 : 2;       // logit segment ring depth
+    t.a_off = 0;
+    t.b_off = t.a_off + t.nkb * kABlockBytes;
+    t.l_off = t.b_off + t.sB * kStageBytes;
+    t.bar_off = t.l_off + t.sL * kSegBytes;
+    t.total = t.bar_off + 256 + 1024;   // barriers, base alignment
+    return t;
+}
 
 // Epilogue modes: drafting partials, or residual mass for verification.
 enum { kEpiDraft = 0, kEpiResidual = 1 };
@@ -54,7 +79,9 @@ struct TcEpi {
     const float *temp;
     int B, G, V, pos, nParts;
     WsHeader *hdr;
-    const __nv_bfloat16 *E;   // [round_up(B,128), r] A-operand rows
+    const __nv_bfloat16 *U;   // [V, r]: A-operand rows are U[previous token]
+    const int32_t *x0;        // [B] last committed tokens
+    const int32_t *x;         // [B, G] draft tokens (drafting: earlier positions of this call)
     const __nv_bfloat16 *L;   // drafting and residual: backbone logits [B, G, V]
     // drafting: 64-column partials per request row
     float *part_m, *part_s;
@@ -69,20 +96,27 @@ struct TcEpi {
 };
 
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_constant__ CUtensorMap mapW, int r,
+__global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_constant__ CUtensorMap mapW,
+                                                              const __grid_constant__ CUtensorMap mapL, int r,
                                                               int nTilesN, const TcEpi ep)
 {
     extern __shared__ unsigned char smem_raw[];
+    const TcLayout lay = tc_layout(r);
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     unsigned char *base = smem_raw + (((raw_u32 + 1023) & ~1023u) - raw_u32);
-    unsigned char *sB = base;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(base + kStages * kStageBytes);
-    uint64_t *a_full = bars;                       // 8 epilogue-warp arrivals: A is in TMEM
-    uint64_t *b_full = bars + 1;                   // kStages
-    uint64_t *b_empty = b_full + kStages;          // kStages
-    uint64_t *acc_full = b_empty + kStages;        // 2
-    uint64_t *acc_empty = acc_full + 2;            // 2
-    uint64_t *drain = acc_empty + 2;               // 1
+    unsigned char *sA = base + lay.a_off;
+    unsigned char *sB = base + lay.b_off;
+    unsigned char *sL = base + lay.l_off;
+    const int SB = lay.sB, SL = lay.sL, nkb = lay.nkb;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar_off);
+    uint64_t *a_full = bars;                 // 16 epilogue-warp arrivals: A is in shared memory
+    uint64_t *b_full = a_full + 1;           // SB
+    uint64_t *b_empty = b_full + SB;         // SB
+    uint64_t *l_full = b_empty + SB;         // SL
+    uint64_t *l_empty = l_full + SL;         // SL (4 warps, one per lane quarter)
+    uint64_t *acc_full = l_empty + SL;       // 2
+    uint64_t *acc_empty = acc_full + 2;      // 2 (16 warps)
+    uint64_t *drain = acc_empty + 2;         // 1
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
@@ -94,15 +128,15 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     const int m0 = mb * kM;
     const int first_tile = blockIdx.x / nMB;
     const int tile_step = ((int)gridDim.x - mb + nMB - 1) / nMB;
-    const int nkb = (r + kKB - 1) / kKB;
     // Residual rows are counted on the device: m-blocks past the count leave now.
     const int nrows = (MODE == kEpiResidual) ? (int)*reinterpret_cast<const volatile uint32_t *>(ep.nrows) : B;
     if (m0 >= nrows) return;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(a_full, 8);
-        for (int s = 0; s < kStages; ++s) { tc::mbar_init(&b_full[s], 1); tc::mbar_init(&b_empty[s], 1); }
-        for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], 8); }
+        tc::mbar_init(a_full, kEpiWarps);
+        for (int q = 0; q < SB; ++q) { tc::mbar_init(&b_full[q], 1); tc::mbar_init(&b_empty[q], 1); }
+        for (int q = 0; q < SL; ++q) { tc::mbar_init(&l_full[q], 1); tc::mbar_init(&l_empty[q], 4); }
+        for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], kEpiWarps); }
         tc::mbar_init(drain, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
@@ -126,8 +160,8 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 const int n0 = t * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % kStages;
-                    if (!tc::mbar_wait_bounded(&b_empty[s], ((g / kStages) & 1) ^ 1, abort_flag, kWaitBudget)) {
+                    const int s = g % SB;
+                    if (!tc::mbar_wait_bounded(&b_empty[s], ((g / SB) & 1) ^ 1, abort_flag, kWaitBudget)) {
                         ok = false;
                         break;
                     }
@@ -140,9 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 // this thread issued so that none lands after the CTA exits.
                 int dummy = 0;
                 volatile int *no_abort = &dummy;
-                for (int q = 0; q < kStages && g - 1 - q >= 0; ++q) {
+                for (int q = 0; q < SB && g - 1 - q >= 0; ++q) {
                     const int gg = g - 1 - q;
-                    tc::mbar_wait_bounded(&b_full[gg % kStages], (gg / kStages) & 1, no_abort, kWaitBudget / 4);
+                    tc::mbar_wait_bounded(&b_full[gg % SB], (gg / SB) & 1, no_abort, kWaitBudget / 4);
                 }
                 flag_status(hdr, DSPARK_DEV_TIMEOUT);
             }
@@ -151,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16_f32(kM, kBN);
-            const uint32_t b_addr = tc::smem_u32(sB);
+            const uint32_t a_addr = tc::smem_u32(sA), b_addr = tc::smem_u32(sB);
             bool ok = tc::mbar_wait_bounded(a_full, 0, abort_flag, kWaitBudget);
             tc::tc_fence_after();
             int g = 0, j = 0;
@@ -162,19 +196,19 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     break;
                 }
                 tc::tc_fence_after();
-                const uint32_t d = tmem_base + kAccCol0 + ab * kBN;
+                const uint32_t d = tmem_base + ab * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
-                    const int s = g % kStages;
-                    if (!tc::mbar_wait_bounded(&b_full[s], (g / kStages) & 1, abort_flag, kWaitBudget)) {
+                    const int s = g % SB;
+                    if (!tc::mbar_wait_bounded(&b_full[s], (g / SB) & 1, abort_flag, kWaitBudget)) {
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kKB / 16; ++kk) {
-                        const uint32_t a = tmem_base + kb * (kKB / 2) + kk * 8;   // 16 bf16 = 8 columns
+                        const uint64_t ad = tc::sw128_desc(a_addr + kb * kABlockBytes + kk * 32);
                         const uint64_t bd = tc::sw128_desc(b_addr + s * kStageBytes + kk * 32);
-                        tc::mma_bf16_ts(d, a, bd, idesc, (kb | kk) != 0);
+                        tc::mma_bf16(d, ad, bd, idesc, (kb | kk) != 0);
                     }
                     tc::mma_commit(&b_empty[s]);
                 }
@@ -187,33 +221,77 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             tc::mbar_wait_bounded(drain, 0, &dummy, kWaitBudget / 4);
             if (!ok) flag_status(hdr, DSPARK_DEV_TIMEOUT);
         }
-    } else {
-        const int ew = warp - kEpiWarp0;
-        const int quarter = warp & 3;          // TMEM lane quarter this warp may access
-        const int half = ew >> 2;              // which 64-column half of every tile
-        const int row = quarter * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        // ---------------------------------------------- A operand into TMEM
-        // Row m0 + row of E; this warp writes the k-blocks kb = half, half+2, ...
-        // (zeros past r), 32 columns per k-block.
-        {
-            const __nv_bfloat16 *erow = ep.E + (size_t)(m0 + row) * r;
-            for (int kb = half; kb < nkb; kb += 2) {
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t v[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int k = kb * kKB + h2 * 32 + q * 8;
-                        uint4 x = make_uint4(0, 0, 0, 0);
-                        if (k < r) x = ld_nc16(erow + k);
-                        v[q * 4 + 0] = x.x; v[q * 4 + 1] = x.y; v[q * 4 + 2] = x.z; v[q * 4 + 3] = x.w;
+    } else if (warp == 2) {
+        // ------------------------------------------------------ logit producer
+        if (MODE == kEpiDraft && lane == 0) {
+            tc::prefetch_tmap(&mapL);
+            const uint64_t stream = tc::policy_evict_first();
+            int g = 0;
+            bool ok = true;
+            for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
+                for (int sg = 0; sg < kSegs; ++sg, ++g) {
+                    const int q = g % SL;
+                    if (!tc::mbar_wait_bounded(&l_empty[q], ((g / SL) & 1) ^ 1, abort_flag, kWaitBudget)) {
+                        ok = false;
+                        break;
                     }
-                    tc::tmem_st16(tmem_base + lane_addr + kb * (kKB / 2) + h2 * 16, v);
+                    tc::mbar_arrive_expect_tx(&l_full[q], kSegBytes);
+                    tc::tma_load_3d(sL + q * kSegBytes, &mapL, &l_full[q], t * kBN + sg * kSeg, ep.pos, m0, stream);
                 }
             }
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
+            if (!ok) {
+                int dummy = 0;
+                volatile int *no_abort = &dummy;
+                for (int q = 0; q < SL && g - 1 - q >= 0; ++q) {
+                    const int gg = g - 1 - q;
+                    tc::mbar_wait_bounded(&l_full[gg % SL], (gg / SL) & 1, no_abort, kWaitBudget / 4);
+                }
+                flag_status(hdr, DSPARK_DEV_TIMEOUT);
+            }
+        }
+    } else {
+        const int ew = warp - kEpiWarp0;       // 0..15
+        const int quarter = warp & 3;          // TMEM lane quarter this warp may access
+        const int sg = ew >> 2;                // 64-column segment of every tile (0..3)
+        const int row = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        // ---------------------------------------------- A operand into smem
+        // Row m0 + row is U[previous token] of that row (the previous draft
+        // token, x0 at the first position, or for a queued rejection the token
+        // before it).  This warp writes k-blocks kb = sg, sg + 4, ... of its
+        // 32 rows in the 128-byte-swizzled K-major layout (zeros past r).
+        {
+            int prev = 0;
+            if (MODE == kEpiDraft) {
+                const int b = m0 + row;
+                if (b < B) {
+                    prev = (ep.pos == 0) ? ep.x0[b] : ep.x[(size_t)b * ep.G + ep.pos - 1];
+                    if (prev < 0 || prev >= V) {
+                        if (ep.pos == 0) flag_status(hdr, DSPARK_DEV_TOKEN_RANGE);
+                        prev = prev < 0 ? 0 : V - 1;
+                    }
+                }
+            } else {
+                const int sidx = m0 + row;
+                if (sidx < nrows) {
+                    const int b = ep.res_b[sidx], k = ep.res_k[sidx];
+                    prev = (k == 0) ? ep.x0[b] : ep.x[(size_t)b * ep.G + k - 1];
+                    prev = min(max(prev, 0), V - 1);
+                }
+            }
+            const __nv_bfloat16 *urow = ep.U + (size_t)prev * r;
+            for (int kb = sg; kb < nkb; kb += kSegs) {
+                uint4 v[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int k = kb * kKB + c * 8;
+                    v[c] = (k < r) ? ld_nc16(urow + k) : make_uint4(0, 0, 0, 0);
+                }
+                unsigned char *dst = sA + kb * kABlockBytes + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + ((c ^ (row & 7)) << 4)) = v[c];
+            }
+            tc::fence_proxy_async_smem();   // generic writes -> tensor-core reads
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(a_full);
         }
@@ -222,8 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             // One online pass per 32-column chunk: y = L + Delta, chunk max,
             // then the running sum of exp((y - max) / T), rescaled when the
             // max grows.  The lowest argmax is tracked only in warps holding a
-            // greedy row.  The row's logits for the next tile are loaded
-            // before waiting on this tile's accumulator.
+            // greedy row.
             const int b = m0 + row;
             const bool rowok = b < B;
             float invT = 0.f;
@@ -234,55 +311,53 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             const float cexp = invT * kLog2e;      // exp((y - m) / T) = 2^((y - m) * cexp)
             const bool warp_greedy = __any_sync(0xffffffffu, rowok && invT == 0.f);
             const bool warp_soft = __any_sync(0xffffffffu, rowok && invT > 0.f);
-            const __nv_bfloat16 *lrow = ep.L + ((size_t)(rowok ? b : 0) * ep.G + ep.pos) * V;
-            uint4 lq[8];
-            auto load_l = [&](int t) {
-                const int cb = t * kBN + half * kPartN;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int c8 = cb + u * 8;
-                    lq[u] = (rowok && c8 < V) ? ld_nc16(lrow + c8) : make_uint4(0, 0, 0, 0);
-                }
-            };
-            if (first_tile < nTilesN) load_l(first_tile);
             int j = 0;
             for (int t = first_tile; t < nTilesN; t += tile_step, ++j) {
                 const int ab = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                uint4 cur[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) cur[u] = lq[u];
-                if (t + tile_step < nTilesN) load_l(t + tile_step);
+                const int gl = j * kSegs + sg, q = gl % SL;
                 // Every lane waits; the vote keeps the warp converged for the
                 // warp-collective TMEM loads below even if the budget runs out.
-                const bool ok = tc::mbar_wait_bounded(&acc_full[ab], ph, abort_flag, kWaitBudget);
+                bool ok = tc::mbar_wait_bounded(&l_full[q], (gl / SL) & 1, abort_flag, kWaitBudget);
+                ok = ok && tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc::tc_fence_after();
-                const uint32_t taddr = tmem_base + lane_addr + kAccCol0 + ab * kBN + half * kPartN;
-                const int cbase = t * kBN + half * kPartN;
-                const bool whole = cbase + kPartN <= V;   // no column of this half lies past V
+                // This thread's 64 logits: one 128-byte row of the swizzled segment.
+                const unsigned char *lsrc = sL + q * kSegBytes + row * 128;
+                uint4 cur[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    cur[u] = *reinterpret_cast<const uint4 *>(lsrc + ((u ^ (row & 7)) << 4));
+                const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
+                const int cbase = t * kBN + sg * kSeg;
+                const bool whole = cbase + kSeg <= V;   // no column of this segment lies past V
                 float m = -INFINITY, s = 0.f;
                 int am = 0x7fffffff;
 #pragma unroll
-                for (int c = 0; c < kPartN / 32; ++c) {
+                for (int c = 0; c < kSeg / 32; ++c) {
                     float y[32];
                     tc::tmem_ld32(taddr + c * 32, y);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const uint4 q = cur[c * 4 + u];
-                        y[u * 8 + 0] += bf16lo(q.x); y[u * 8 + 1] += bf16hi(q.x);
-                        y[u * 8 + 2] += bf16lo(q.y); y[u * 8 + 3] += bf16hi(q.y);
-                        y[u * 8 + 4] += bf16lo(q.z); y[u * 8 + 5] += bf16hi(q.z);
-                        y[u * 8 + 6] += bf16lo(q.w); y[u * 8 + 7] += bf16hi(q.w);
+                        const uint4 qv = cur[c * 4 + u];
+                        y[u * 8 + 0] += bf16lo(qv.x); y[u * 8 + 1] += bf16hi(qv.x);
+                        y[u * 8 + 2] += bf16lo(qv.y); y[u * 8 + 3] += bf16hi(qv.y);
+                        y[u * 8 + 4] += bf16lo(qv.z); y[u * 8 + 5] += bf16hi(qv.z);
+                        y[u * 8 + 6] += bf16lo(qv.w); y[u * 8 + 7] += bf16hi(qv.w);
                     }
                     if (!whole) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             if (cbase + c * 32 + e >= V) y[e] = -INFINITY;
                     }
-                    float cm = y[0];
+                    // Tree max (short dependency chains).
+                    float t16[16];
 #pragma unroll
-                    for (int e = 1; e < 32; ++e) cm = fmaxf(cm, y[e]);
+                    for (int e = 0; e < 16; ++e) t16[e] = fmaxf(y[e], y[e + 16]);
+#pragma unroll
+                    for (int wdt = 8; wdt > 0; wdt >>= 1)
+#pragma unroll
+                        for (int e = 0; e < wdt; ++e) t16[e] = fmaxf(t16[e], t16[e + wdt]);
+                    const float cm = t16[0];
                     if (warp_greedy && cm > m) {
                         int ix = 0x7fffffff;
 #pragma unroll
@@ -292,17 +367,22 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     }
                     const float mn = fmaxf(m, cm);
                     if (warp_soft) {
-                        float acc = 0.f;
+                        float a4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sums
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) acc += fast_exp2((y[e] - mn) * cexp);
+                        for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2((y[e] - mn) * cexp);
+                        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
                         s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + acc;
                     }
                     m = mn;
                 }
                 tc::tc_fence_before();
+                tc::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
-                const int p = t * (kBN / kPartN) + half;
+                if (lane == 0) {
+                    tc::mbar_arrive(&acc_empty[ab]);
+                    tc::mbar_arrive(&l_empty[q]);
+                }
+                const int p = t * kSegs + sg;
                 if (rowok && p < nParts) {
                     const size_t o = (size_t)b * nParts + p;
                     ep.part_m[o] = m;
@@ -330,33 +410,27 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             int j = 0;
             for (int t = first_tile; t < nTilesN; t += tile_step, ++j) {
                 const int ab = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                const int cbase = t * kBN + half * kPartN;
-                // Issue this row's logit loads before waiting on the accumulator.
-                uint4 lq[8], tq[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int c8 = cbase + u * 8;
-                    if (rowok && c8 < V) {
-                        lq[u] = ld_nc16(Lrow + c8);
-                        tq[u] = ld_nc16(Trow + c8);
-                    } else {
-                        lq[u] = make_uint4(0, 0, 0, 0);
-                        tq[u] = make_uint4(0, 0, 0, 0);
-                    }
-                }
-                const bool ok = tc::mbar_wait_bounded(&acc_full[ab], ph, abort_flag, kWaitBudget);
+                const int cbase = t * kBN + sg * kSeg;
+                const bool ok = tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc::tc_fence_after();
-                const uint32_t taddr = tmem_base + lane_addr + kAccCol0 + ab * kBN + half * kPartN;
+                const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
                 float qs = 0.f;
 #pragma unroll
-                for (int c = 0; c < kPartN / 32; ++c) {
+                for (int c = 0; c < kSeg / 32; ++c) {
+                    uint4 lq[4], tq[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c8 = cbase + c * 32 + u * 8;
+                        const bool in = rowok && c8 < V;
+                        lq[u] = in ? ld_nc16(Lrow + c8) : make_uint4(0, 0, 0, 0);
+                        tq[u] = in ? ld_nc16(Trow + c8) : make_uint4(0, 0, 0, 0);
+                    }
                     float d[32];
                     tc::tmem_ld32(taddr + c * 32, d);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const uint4 a = lq[c * 4 + u], bq = tq[c * 4 + u];
+                        const uint4 a = lq[u], bq = tq[u];
                         const float l8[8] = {bf16lo(a.x), bf16hi(a.x), bf16lo(a.y), bf16hi(a.y),
                                              bf16lo(a.z), bf16hi(a.z), bf16lo(a.w), bf16hi(a.w)};
                         const float t8[8] = {bf16lo(bq.x), bf16hi(bq.x), bf16lo(bq.y), bf16hi(bq.y),
@@ -373,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 tc::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
-                const int p = t * (kBN / kPartN) + half;
+                const int p = t * kSegs + sg;
                 if (rowok && p < nParts) ep.rp[(size_t)sidx * nParts + p] = qs;
             }
         }
@@ -412,7 +486,7 @@ bool map_factor(CUtensorMap *m, const void *Wt, int V, int r) {
     if (fn == nullptr) return false;
     cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)V};
     cuuint64_t strides[1] = {(cuuint64_t)r * 2};
-    cuuint32_t box[2] = {kKB, kBN};
+    cuuint32_t box[2] = {kKB, kBN};   // 64 x 256: one k-block of a 256-column tile
     cuuint32_t es[2] = {1, 1};
     CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(Wt), dims, strides, box, es,
                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -420,12 +494,29 @@ bool map_factor(CUtensorMap *m, const void *Wt, int V, int r) {
     return res == CUDA_SUCCESS;
 }
 
+// Tensor map of the logits L [B, G, V] (bf16) as a 3-D tensor (V, G, B):
+// 64-column x 1 x 128-row boxes, 128-byte swizzle, out-of-range reads as zero.
+bool map_logits(CUtensorMap *m, const void *L, int B, int G, int V) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)V, (cuuint64_t)G, (cuuint64_t)B};
+    cuuint64_t strides[2] = {(cuuint64_t)V * 2, (cuuint64_t)G * V * 2};
+    cuuint32_t box[3] = {kSeg, 1, kM};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(L), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS;
+}
+
 template <int MODE>
 cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, cudaStream_t st) {
-    CUtensorMap mW;
+    CUtensorMap mW, mL;
     if (!map_factor(&mW, Wt, ep.V, r)) return cudaErrorInvalidValue;
+    if (!map_logits(&mL, ep.L, ep.B, ep.G, ep.V)) return cudaErrorInvalidValue;
+    const TcLayout lay = tc_layout(r);
     cudaError_t e = cudaFuncSetAttribute(markov_tile_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)lay.total);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -434,7 +525,7 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, cudaStream_
     const int nMB = (ep.B + kM - 1) / kM;
     int grid = std::min(sms, nMB * nTilesN);
     grid = std::max(grid, nMB);
-    markov_tile_tc<MODE><<<grid, kThreads, kSmemBytes, st>>>(mW, r, nTilesN, ep);
+    markov_tile_tc<MODE><<<grid, kThreads, lay.total, st>>>(mW, mL, r, nTilesN, ep);
     return cudaGetLastError();
 }
 
@@ -443,7 +534,8 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, cudaStream_
 cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
     TcEpi ep{};
     ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.pos = pos; ep.nParts = w.nTiles; ep.hdr = w.hdr;
-    ep.E = w.E; ep.L = static_cast<const __nv_bfloat16 *>(a.L);
+    ep.U = static_cast<const __nv_bfloat16 *>(a.U); ep.x0 = a.x0; ep.x = a.x_out;
+    ep.L = static_cast<const __nv_bfloat16 *>(a.L);
     ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
     return launch_markov_tc<kEpiDraft>(a.Wt, a.r, ep, st);
 }
@@ -451,7 +543,7 @@ cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, 
 cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st) {
     TcEpi ep{};
     ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.pos = 0; ep.nParts = a.nParts; ep.hdr = a.hdr;
-    ep.E = a.E; ep.L = a.L;
+    ep.U = a.U; ep.x0 = a.x0; ep.x = a.x; ep.L = a.L;
     ep.nrows = a.nrows; ep.res_b = a.res_b; ep.res_k = a.res_k; ep.res_mt = a.res_mt; ep.res_zt = a.res_zt;
     ep.rowmax = a.rowmax; ep.rowsum = a.rowsum; ep.Tlog = a.Tlog; ep.rp = a.rp;
     return launch_markov_tc<kEpiResidual>(a.Wt, a.r, ep, st);

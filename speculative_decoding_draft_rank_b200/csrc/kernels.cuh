@@ -25,7 +25,6 @@ struct DraftWs {
     WsHeader *hdr;
     float *part_m, *part_s;
     int32_t *part_a;
-    __nv_bfloat16 *E;   // [round_up(B,128), r] gathered U rows (bf16 only)
     int nTiles;
 };
 
@@ -63,7 +62,8 @@ size_t verify_ws_bytes(int B, int G, int V, int r, int dtype);
 // queued rejections (count on the device), A operand their gathered U rows.
 struct ResidualTcArgs {
     const void *Wt;
-    const __nv_bfloat16 *E, *L, *Tlog;
+    const __nv_bfloat16 *U, *L, *Tlog;
+    const int32_t *x0, *x;
     const float *temp, *rowmax, *rowsum, *res_mt, *res_zt;
     const int32_t *res_b, *res_k;
     const uint32_t *nrows;

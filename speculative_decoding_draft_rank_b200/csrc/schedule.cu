@@ -7,11 +7,10 @@
 // token k never looks at information from after x_k is drawn).
 //
 // One CTA of 1024 threads does the whole stage:
-//   1. keys ~bits(S) (ascending = S descending, valid since S >= 0) and
-//      position-major candidate ids i*B + b are sorted by a stable LSD radix
-//      sort in shared memory (8 passes of 4 bits; each thread owns a
-//      contiguous chunk, per-thread digit counts are scanned digit-major so
-//      equal keys keep their id order);
+//   1. 64-bit keys (~bits(S) above the position-major candidate id i*B + b)
+//      are sorted ascending by a bitonic sort in shared memory; the keys are
+//      unique, so this is the stable sort by S descending with ties going to
+//      the lower id;
 //   2. fp64 block scan of the sorted survivals gives V_n = B + sum_{j<n} S_(j);
 //   3. every candidate n evaluates the stop test
 //      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index
@@ -25,8 +24,6 @@ namespace dspark {
 constexpr int kSchedThreads = 1024;
 constexpr int kSchedMaxN = 16384;
 constexpr int kSchedMaxP = 64;
-constexpr int kRadixBits = 4;
-constexpr int kRadixBins = 1 << kRadixBits;
 
 // Piecewise-linear profile through (kn[j], kt[j]) continued with the last slope.
 __device__ __forceinline__ double profile_at(const int *kn, const double *kt, int P, double n) {
@@ -47,15 +44,12 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 {
     extern __shared__ __align__(16) unsigned char sched_smem[];
     const int N = B * G;
-    uint32_t *keys = reinterpret_cast<uint32_t *>(sched_smem);                  // [N]
-    uint16_t *ids = reinterpret_cast<uint16_t *>(keys + kSchedMaxN);            // [N]
-    uint16_t *cnt = ids + kSchedMaxN;                                          // [bins][threads]
-    int *ell_s = reinterpret_cast<int *>(cnt);                                 // reused after sorting
+    unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [n2]
+    int *ell_s = reinterpret_cast<int *>(keys + kSchedMaxN);                          // [B]
     __shared__ int kn_s[kSchedMaxP];
     __shared__ double kt_s[kSchedMaxP];
     __shared__ int red_i[33];
     __shared__ double red_d[33];
-    __shared__ int tot_s[33];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
@@ -78,74 +72,42 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
         return;
     }
 
-    // Keys and ids in position-major order (id = i*B + b).
-    for (int id = tid; id < N; id += blockDim.x) {
-        const int i = id / B, b = id - i * B;
-        float s = S[(size_t)b * G + i];
-        if (!(s >= 0.f)) s = 0.f;  // NaN or negative survival ranks last
-        keys[id] = ~__float_as_uint(s);
-        ids[id] = (uint16_t)id;
+    // Unique 64-bit keys: ~bits(S) (ascending = S descending, valid for
+    // S >= 0) above the position-major id, so an ascending sort is the stable
+    // sort by S descending.  Padding keys sort last.
+    int n2 = 1;
+    while (n2 < N) n2 <<= 1;
+    for (int id = tid; id < n2; id += blockDim.x) {
+        unsigned long long k = ~0ull;
+        if (id < N) {
+            const int i = id / B, b = id - i * B;
+            float s = S[(size_t)b * G + i];
+            if (!(s >= 0.f)) s = 0.f;  // NaN or negative survival ranks last
+            k = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)id;
+        }
+        keys[id] = k;
     }
     __syncthreads();
-
-    const int cpt = (N + blockDim.x - 1) / blockDim.x;  // chunk per thread (<= 16)
-    const int c0 = min(N, tid * cpt), c1 = min(N, c0 + cpt);
-    constexpr int kMaxChunk = kSchedMaxN / kSchedThreads;
-    for (int shift = 0; shift < 32; shift += kRadixBits) {
-        uint32_t kr[kMaxChunk];
-        uint32_t ir[kMaxChunk];
-#pragma unroll
-        for (int d = 0; d < kRadixBins; ++d) cnt[d * blockDim.x + tid] = 0;
-#pragma unroll
-        for (int j = 0; j < kMaxChunk; ++j) {
-            if (c0 + j < c1) {
-                kr[j] = keys[c0 + j];
-                ir[j] = ids[c0 + j];
-                cnt[((kr[j] >> shift) & (kRadixBins - 1)) * blockDim.x + tid]++;
+    // Bitonic sort in shared memory: one compare-exchange per pair per stage.
+    for (int k = 2; k <= n2; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < (n2 >> 1); i += blockDim.x) {
+                const int lo = 2 * i - (i & (j - 1)), hi = lo + j;
+                const bool up = (lo & k) == 0;
+                const unsigned long long a = keys[lo], c = keys[hi];
+                if ((a > c) == up) { keys[lo] = c; keys[hi] = a; }
             }
+            __syncthreads();
         }
-        __syncthreads();
-        // Exclusive scan of cnt in (digit, thread) order: thread t scans the
-        // kRadixBins consecutive entries starting at kRadixBins * t.
-        uint16_t *mine = cnt + tid * kRadixBins;
-        int s = 0;
-#pragma unroll
-        for (int j = 0; j < kRadixBins; ++j) s += mine[j];
-        const int ws = warp_incl_scan_i(s);
-        if (lane == 31) tot_s[wid] = ws;
-        __syncthreads();
-        if (wid == 0) {
-            int t = lane < (int)(blockDim.x >> 5) ? tot_s[lane] : 0;
-            t = warp_incl_scan_i(t);
-            tot_s[lane] = t;
-        }
-        __syncthreads();
-        int run = ws - s + (wid > 0 ? tot_s[wid - 1] : 0);
-#pragma unroll
-        for (int j = 0; j < kRadixBins; ++j) {  // offsets reach N <= 16384: fits 16 bits
-            const int c = mine[j];
-            mine[j] = (uint16_t)run;
-            run += c;
-        }
-        __syncthreads();
-        // Stable scatter: each thread walks its chunk in order, bumping its
-        // own column of offsets.
-#pragma unroll
-        for (int j = 0; j < kMaxChunk; ++j) {
-            if (c0 + j < c1) {
-                uint16_t &o = cnt[((kr[j] >> shift) & (kRadixBins - 1)) * blockDim.x + tid];
-                const int p = o;
-                o = (uint16_t)(p + 1);
-                keys[p] = kr[j];
-                ids[p] = (uint16_t)ir[j];
-            }
-        }
-        __syncthreads();
     }
 
-    // fp64 prefix of the sorted survivals: V_n = B + sum_{j<n} S_(j).
+    // fp64 prefix of the sorted survivals: V_n = B + sum_{j<n} S_(j).  Thread t
+    // owns the contiguous ranks [c0, c1).
+    const int cpt = (N + blockDim.x - 1) / blockDim.x;
+    const int c0 = min(N, tid * cpt), c1 = min(N, c0 + cpt);
+    auto surv = [&](int n) { return (double)__uint_as_float(~(unsigned)(keys[n] >> 32)); };
     double run = 0.0;
-    for (int n = c0; n < c1; ++n) run += (double)__uint_as_float(~keys[n]);
+    for (int n = c0; n < c1; ++n) run += surv(n);
     const double wsum = warp_incl_scan_d(run);
     if (lane == 31) red_d[wid] = wsum;
     __syncthreads();
@@ -161,7 +123,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     {
         double Vn = Vbase;
         for (int n = c0; n < c1 && n < limit; ++n) {
-            const double sn = (double)__uint_as_float(~keys[n]);
+            const double sn = surv(n);
             const double t0 = profile_at(kn_s, kt_s, P, (double)n);
             const double t1 = profile_at(kn_s, kt_s, P, (double)(n + 1));
             if ((Vn + sn) * t0 < Vn * t1) { first_stop = n; break; }
@@ -178,14 +140,14 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     __syncthreads();
     if (c0 < c1 && ((nadm >= c0 && nadm < c1) || (nadm == N && c1 == N))) {
         double Vn = Vbase;
-        for (int n = c0; n < nadm && n < c1; ++n) Vn += (double)__uint_as_float(~keys[n]);
+        for (int n = c0; n < nadm && n < c1; ++n) Vn += surv(n);
         Vadm_s = Vn;
     }
     for (int b = tid; b < B; b += blockDim.x) ell_s[b] = 0;
     __syncthreads();
-    for (int n = tid; n < nadm; n += blockDim.x) atomicAdd(&ell_s[ids[n] % B], 1);
+    for (int n = tid; n < nadm; n += blockDim.x) atomicAdd(&ell_s[(int)(unsigned)keys[n] % B], 1);
     if (order_out != nullptr)
-        for (int n = tid; n < N; n += blockDim.x) order_out[n] = ids[n];
+        for (int n = tid; n < N; n += blockDim.x) order_out[n] = (int)(unsigned)keys[n];
     __syncthreads();
     for (int b = tid; b < B; b += blockDim.x) ell_out[b] = ell_s[b];
     if (tid == 0) {
@@ -200,10 +162,7 @@ cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n
                             const double *knots_t, int P, int budget, int mode, void *,
                             int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
                             int32_t *order_out, cudaStream_t st) {
-    const size_t smem = sizeof(uint32_t) * kSchedMaxN + sizeof(uint16_t) * kSchedMaxN +
-                        sizeof(uint16_t) * kRadixBins * kSchedThreads;
-    static_assert(sizeof(uint16_t) * kRadixBins * kSchedThreads >= sizeof(int) * 4096,
-                  "the count table doubles as the per-request counters");
+    const size_t smem = sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096;
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;

@@ -46,7 +46,6 @@ struct VerifyWs {
     int32_t *res_k;            // [B] rejected position (0-based)
     float *res_mt, *res_zt;    // [B] target row max / Z of the rejected row
     float *rp;                 // [B*nResTiles] residual tile sums
-    __nv_bfloat16 *E;          // [round_up(B,128), r] gathered U rows of the queue (bf16)
     int nChunks, nResTiles, resCols;
 };
 
@@ -68,8 +67,6 @@ static VerifyWs carve_verify_ws(void *ws, int B, int G, int V, int r, int dtype)
     w.res_mt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
     w.res_zt = reinterpret_cast<float *>(p); p += align256(sizeof(float) * B);
     w.rp = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * w.nResTiles);
-    w.E = nullptr;
-    if (dtype == DSPARK_BF16) w.E = reinterpret_cast<__nv_bfloat16 *>(p);
     return w;
 }
 
@@ -78,7 +75,6 @@ size_t verify_ws_bytes(int B, int G, int V, int r, int dtype) {
     const size_t R = (size_t)B * (G + 1);
     size_t bytes = sizeof(WsHeader) + align256(4 * R) + align256(4 * (B + 1)) + 3 * align256(4 * R * nChunks) +
                    4 * align256(4 * (size_t)B) + align256(4 * (size_t)B * nResTiles);
-    if (dtype == DSPARK_BF16) bytes += align256(2 * (size_t)round_up(B, 128) * r);
     return bytes;
 }
 
@@ -472,7 +468,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     __shared__ int rA[17];
     __shared__ float red[33];
     __shared__ int redi[33];
-    __shared__ int A_s, slot_s;
+    __shared__ int A_s;
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float Tb = sane_temp(temp[b], w.hdr);
     const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
@@ -487,7 +483,6 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     }
     __syncthreads();
     if (tid == 0) {
-        slot_s = -1;
         int A = 0;
         bool rejected = false;
         for (int k = 0; k < G; ++k) {
@@ -523,17 +518,10 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
             w.res_k[slot] = A;
             w.res_mt[slot] = rM[A];
             w.res_zt[slot] = rZ[A];
-            slot_s = slot;
         }
     }
     __syncthreads();
     const int A = A_s;
-    if (w.E != nullptr && slot_s >= 0) {  // A-operand row U[x_{k*-1}] of the queued rejection
-        const int prev = min(max((A == 0) ? x0[b] : x[(size_t)b * G + A - 1], 0), V - 1);
-        const uint4 *src = reinterpret_cast<const uint4 *>(U + (size_t)prev * r);
-        uint4 *dst = reinterpret_cast<uint4 *>(w.E + (size_t)slot_s * r);
-        for (int q = tid; q < r / 8; q += blockDim.x) dst[q] = src[q];
-    }
     if (Tb > 0.f && A == lb) {  // bonus (fresh token when nothing was admitted)
         const int y = sample_target_row(Tlog, w, j0 + lb, b, lb, G, V, rM[lb], rZ[lb], invT,
                                         u_final[b], red, redi);
@@ -724,19 +712,19 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
         const int grid = max(1, min(maxwork, sms * 4));
         verify_rows_bulk<<<grid, kRowThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp,
                                                           a.G, a.V, w);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         const int grid = max(1, min(maxwork, sms * 8));
         verify_rows<T><<<grid, kRowThreads, 0, st>>>(Tl, a.temp, a.G, a.V, w);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    verify_decide<T><<<a.B, kRowThreads, 0, st>>>(Tl, static_cast<const T *>(a.U), a.x0, a.r, a.x, a.pd_x,
-                                                  a.temp, a.u_accept, a.u_final, a.ell,
-                                                  a.B, a.G, a.V, w, a.acc_out, a.tokens_out,
-                                                  a.nout_out, a.pt_x_out);
+    verify_decide<T><<<a.B, kRowThreads, 0, st>>>(Tl, static_cast<const T *>(a.U), a.x0, a.r, a.x, a.pd_x, a.temp,
+                                                  a.u_accept, a.u_final, a.ell, a.B, a.G, a.V, w, a.acc_out,
+                                                  a.tokens_out, a.nout_out, a.pt_x_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.dtype == DSPARK_BF16) {
-        ResidualTcArgs ra{a.Wt, w.E, static_cast<const __nv_bfloat16 *>(a.L),
-                          static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp, a.rowmax, a.rowsum, w.res_mt,
+        ResidualTcArgs ra{a.Wt, static_cast<const __nv_bfloat16 *>(a.U), static_cast<const __nv_bfloat16 *>(a.L),
+                          static_cast<const __nv_bfloat16 *>(a.Tlog), a.x0, a.x, a.temp, a.rowmax, a.rowsum, w.res_mt,
                           w.res_zt, w.res_b, w.res_k, &w.hdr->pad[1], a.B, a.G, a.V, a.r, w.nResTiles, w.rp, w.hdr};
         if ((e = launch_residual_tile_tc(ra, st)) != cudaSuccess) return e;
     } else {
@@ -754,8 +742,8 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
             return e;
     }
     fin<<<a.B, kRowThreads, smem, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
-                                       static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax, a.rowsum,
-                                       a.temp, a.u_final, a.G, a.V, a.r, w, a.tokens_out);
+                                       static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax, a.rowsum, a.temp,
+                                       a.u_final, a.G, a.V, a.r, w, a.tokens_out);
     return cudaGetLastError();
 }
 

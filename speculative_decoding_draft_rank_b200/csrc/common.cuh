@@ -210,6 +210,47 @@ __device__ __forceinline__ int block_min_i(int v, int *smem) {
     return r;
 }
 
+// ---------------------------------------------------------------------------
+// One-barrier block reductions.  Every warp publishes its partial into its own
+// entry of `slots` (blockDim/32 entries); after a single barrier each thread
+// folds all entries in warp order, so every thread gets the same value.  A
+// call site must own its `slots` array (no other call writes it while a slow
+// warp may still read), which is what removes the trailing barrier.
+__device__ __forceinline__ float block_max1(float v, float *slots) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_max(v);
+    if (lane == 0) slots[wid] = v;
+    __syncthreads();
+    float r = slots[0];
+    for (int w = 1; w < nw; ++w) r = fmaxf(r, slots[w]);
+    return r;
+}
+__device__ __forceinline__ int block_min1(int v, int *slots) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    v = warp_min_i(v);
+    if (lane == 0) slots[wid] = v;
+    __syncthreads();
+    int r = slots[0];
+    for (int w = 1; w < nw; ++w) r = min(r, slots[w]);
+    return r;
+}
+__device__ __forceinline__ int block_max1_i(int v, int *slots) { return -block_min1(-v, slots); }
+// Inclusive block scan in thread order; *total = block sum (same fold order
+// in every thread).
+__device__ __forceinline__ float block_scan1(float v, float *slots, float *total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const float s = warp_incl_scan(v);
+    if (lane == 31) slots[wid] = s;
+    __syncthreads();
+    float before = 0.f, tot = 0.f;
+    for (int w = 0; w < nw; ++w) {
+        if (w == wid) before = tot;
+        tot += slots[w];
+    }
+    *total = tot;
+    return before + s;
+}
+
 // Clamp a token id to [0, V), flagging the status word when it was outside.
 __device__ __forceinline__ int clamp_token(int t, int V, WsHeader *h) {
     if (t < 0 || t >= V) {

@@ -138,10 +138,13 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
 
 // ---------------------------------------------------------------------------
 // Finalize: one CTA of kFinThreads threads per request row.  Thread t owns the
-// contiguous tiles [t K, t K + K): one block max, one block scan of the
-// threads' scaled tile sums, then the thread whose range holds u Z walks its
-// K tiles to the crossing tile, which the block recomputes column by column.
+// contiguous partials [t K, t K + K) and loads them (with the previous token
+// and its U row) before any barrier, so the stage costs a few dependent
+// memory round trips: one block max, one block scan of the threads' scaled
+// partial sums, then the thread whose range holds u Z walks its partials to
+// the crossing one, whose columns the block recomputes and scans.
 constexpr int kFinThreads = 256;
+constexpr int kFinChunk = 8;   // partials per thread held in registers
 
 template <typename T>
 __global__ void __launch_bounds__(kFinThreads) draft_finalize(
@@ -154,102 +157,125 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
 {
     extern __shared__ float fin_smem[];
     float *urow = fin_smem;                 // [r] U[x_{i-1}] row
-    __shared__ float red[33];
-    __shared__ int redi[33];
+    __shared__ float s_max[32], s_loc[32], s_col[32];
+    __shared__ int s_own[32], s_own2[32], s_x[32], s_x2[32];
     __shared__ int ts_s;
-    __shared__ float rem_s, ex_s;
+    __shared__ float rem_s;
 
-    const int b = blockIdx.x, tid = threadIdx.x;
+    const int b = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
     const size_t ro = (size_t)b * G + pos;
     const float *pm = part_m + (size_t)b * nTiles;
     const float *ps = part_s + (size_t)b * nTiles;
-    const float Tb = sane_temp(temp[b], hdr);
-    const int K = (nTiles + blockDim.x - 1) / blockDim.x;
+    const int K = (nTiles + nthr - 1) / nthr;
     const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
 
-    // Start fetching the previous token's U row; it is only needed for T > 0.
+    // Every load that depends on nothing else goes out first.
+    float cm[kFinChunk], cs[kFinChunk];
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) {
+        const bool in = t0 + q < t1;
+        cm[q] = in ? pm[t0 + q] : -INFINITY;
+        cs[q] = in ? ps[t0 + q] : 0.f;
+    }
+    const float Tb = sane_temp(temp[b], hdr);
+    const float u = u_draft[ro];
     const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
+    // The previous token's U row (r <= 512 = 2 x kFinThreads), kept in
+    // registers until after the first barrier.
+    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
+    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
 
     float m = -INFINITY;
-    for (int t = t0; t < t1; ++t) m = fmaxf(m, pm[t]);
-    const float M = block_max(m, red);
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) m = fmaxf(m, cm[q]);
+    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, pm[t]);   // very large vocabularies only
+    const float M = block_max1(m, s_max);
 
-    int x;
-    float pd, Z;
-    if (Tb == 0.f) {
+    if (Tb == 0.f) {   // greedy row (block-uniform): lowest argmax over the partials
         int first = 0x7fffffff;
-        for (int t = t0; t < t1; ++t)
-            if (pm[t] == M) { first = t; break; }
-        first = block_min_i(first, redi);
-        if (first >= nTiles) first = 0;  // no tile matched (non-finite inputs)
-        x = part_a[(size_t)b * nTiles + first];
-        if (x < 0 || x >= V) x = 0;
-        pd = 1.f;
-        Z = 1.f;
-    } else {
-        const float cexp = kLog2e / Tb;
-        for (int k = tid; k < r; k += blockDim.x) urow[k] = ld_elem(U, (size_t)prev * r + k);
-        float loc = 0.f;
-        for (int t = t0; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
-        float tot;
-        const float incl = block_incl_scan(loc, red, &tot);   // also publishes urow
-        Z = tot;
-        const float target = u_draft[ro] * Z;
-        const float before = incl - loc;
-        // The first thread whose inclusive prefix passes u Z owns the crossing
-        // (the last thread with mass if rounding left u Z at the top).
-        int owner = (incl > target && loc > 0.f) ? tid : 0x7fffffff;
-        owner = block_min_i(owner, redi);
-        if (owner == 0x7fffffff) {
-            owner = -block_min_i(loc > 0.f ? -tid : 1, redi);
-            if (owner < 0) owner = 0;
+        for (int t = t1 - 1; t >= t0 + kFinChunk; --t)
+            if (pm[t] == M) first = t;
+#pragma unroll
+        for (int q = kFinChunk - 1; q >= 0; --q)
+            if (t0 + q < t1 && cm[q] == M) first = t0 + q;
+        first = block_min1(first, s_own);
+        if (tid == 0) {
+            if (first >= nTiles) first = 0;  // no partial matched (non-finite inputs)
+            int x = part_a[(size_t)b * nTiles + first];
+            if (x < 0 || x >= V) x = 0;
+            x_out[ro] = x;
+            pd_out[ro] = 1.f;
+            rowmax_out[ro] = M;
+            rowsum_out[ro] = 1.f;
         }
-        if (tid == owner) {
-            float run = before, run_last = before;
-            int ts = -1, last = t1 - 1;
-            for (int t = t0; t < t1; ++t) {
-                const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
-                if (run + wt > target) { ts = t; break; }
+        return;
+    }
+
+    const float cexp = kLog2e / Tb;
+    float loc = 0.f;
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
+    for (int t = t0 + kFinChunk; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
+    if (tid < r) urow[tid] = uv0;
+    if (tid + nthr < r) urow[tid + nthr] = uv1;
+    float Z;
+    const float incl = block_scan1(loc, s_loc, &Z);   // also publishes urow
+    const float target = u * Z;
+    // The first thread whose inclusive prefix passes u Z owns the crossing
+    // (the last thread with mass if rounding left u Z at the top).
+    int owner = block_min1((incl > target && loc > 0.f) ? tid : 0x7fffffff, s_own);
+    if (owner == 0x7fffffff) owner = max(0, block_max1_i(loc > 0.f ? tid : -1, s_own2));
+    if (tid == owner) {
+        float run = incl - loc, run_last = run;
+        int ts = -1, last = t1 - 1;
+#pragma unroll
+        for (int q = 0; q < kFinChunk; ++q) {
+            if (ts < 0 && t0 + q < t1) {
+                const float wt = cs[q] * fast_exp2((cm[q] - M) * cexp);
+                if (run + wt > target) {
+                    ts = t0 + q;
+                } else {
+                    if (wt > 0.f) { last = t0 + q; run_last = run; }
+                    run += wt;
+                }
+            }
+        }
+        for (int t = t0 + kFinChunk; t < t1 && ts < 0; ++t) {
+            const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
+            if (run + wt > target) {
+                ts = t;
+            } else {
                 if (wt > 0.f) { last = t; run_last = run; }
                 run += wt;
             }
-            if (ts < 0) { ts = last; run = run_last; }
-            ts_s = max(ts, 0);
-            rem_s = target - run;
         }
-        __syncthreads();
-        const int ts = ts_s;
-        const float rem = rem_s;
-        // Recompute the chosen tile: tpc consecutive threads share one column.
-        const int c0 = ts * TN;
-        const int tpc = blockDim.x / TN;
-        const int col = c0 + tid / tpc, part = tid % tpc;
-        const bool mine = part == 0 && col < V;
-        const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
-        float dl = 0.f;
-        if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
-        for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
-        float e = 0.f;
-        if (mine) e = fast_exp2(((lval - M) + dl) * cexp);
-        float ttot;
-        const float inc = block_incl_scan(e, red, &ttot);
-        int xs = (mine && inc > rem) ? col : 0x7fffffff;
-        xs = block_min_i(xs, redi);
-        if (xs == 0x7fffffff) {  // the tile's recomputed mass fell short: last positive
-            int lc = (mine && e > 0.f) ? col : -1;
-            xs = -block_min_i(-lc, redi);
-            if (xs < 0) xs = min(c0 + TN, V) - 1;
-        }
-        x = xs;
-        if (tid == 0) ex_s = 0.f;
-        __syncthreads();
-        if (mine && col == x) ex_s = e;
-        __syncthreads();
-        pd = ex_s / Z;
+        if (ts < 0) { ts = last; run = run_last; }
+        ts_s = max(ts, 0);
+        rem_s = target - run;
     }
-    if (tid == 0) {
-        x_out[ro] = x;
-        pd_out[ro] = pd;
+    __syncthreads();
+    const int ts = ts_s;
+    const float rem = rem_s;
+    // Recompute the chosen partial's columns: tpc consecutive threads share one column.
+    const int c0 = ts * TN;
+    const int tpc = nthr / TN;
+    const int col = c0 + tid / tpc, part = tid % tpc;
+    const bool mine = part == 0 && col < V;
+    const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
+    float dl = 0.f;
+    if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
+    for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    const float e = mine ? fast_exp2(((lval - M) + dl) * cexp) : 0.f;
+    float ttot;
+    const float inc = block_scan1(e, s_col, &ttot);
+    int xs = block_min1((mine && inc > rem) ? col : 0x7fffffff, s_x);
+    if (xs == 0x7fffffff) {  // the recomputed mass fell short: last positive column
+        xs = block_max1_i((mine && e > 0.f) ? col : -1, s_x2);
+        if (xs < 0) xs = min(c0 + TN, V) - 1;
+    }
+    if (mine && col == xs) {
+        x_out[ro] = xs;
+        pd_out[ro] = e / Z;
         rowmax_out[ro] = M;
         rowsum_out[ro] = Z;
     }

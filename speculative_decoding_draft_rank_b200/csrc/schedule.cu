@@ -8,9 +8,12 @@
 //
 // One CTA of 1024 threads does the whole stage:
 //   1. 64-bit keys (~bits(S) above the position-major candidate id i*B + b)
-//      are sorted ascending by a bitonic sort in shared memory; the keys are
-//      unique, so this is the stable sort by S descending with ties going to
-//      the lower id;
+//      are sorted ascending by a bitonic sort; the keys are unique, so this
+//      is the stable sort by S descending with ties going to the lower id.
+//      Compare-exchange stages with a partner distance of 64 or more go
+//      through shared memory, one barrier each; a warp holds each 64-key
+//      chunk in registers (two keys per lane) for the stages below that and
+//      exchanges with shuffles;
 //   2. fp64 block scan of the sorted survivals gives V_n = B + sum_{j<n} S_(j);
 //   3. every candidate n evaluates the stop test
 //      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index
@@ -35,6 +38,23 @@ __device__ __forceinline__ double profile_at(const int *kn, const double *kt, in
     }
     const double slope = (kt[lo + 1] - kt[lo]) / (double)(kn[lo + 1] - kn[lo]);
     return kt[lo] + (n - (double)kn[lo]) * slope;
+}
+
+// One bitonic compare-exchange stage (block size k, partner distance j <= 32)
+// on the 64-key chunk a warp holds: lane l has keys e0 = base + 2l and e0 + 1.
+__device__ __forceinline__ void bitonic_warp_step(unsigned long long &v0, unsigned long long &v1, int e0, int k,
+                                                  int j) {
+    const bool up = (e0 & k) == 0;   // the same for e0 and e0 + 1 (k >= 2)
+    if (j == 1) {
+        if ((v0 > v1) == up) { const unsigned long long t = v0; v0 = v1; v1 = t; }
+        return;
+    }
+    const int lane = threadIdx.x & 31, o = j >> 1;   // partner keys sit in lane ^ (j / 2), same slot
+    const unsigned long long o0 = __shfl_xor_sync(0xffffffffu, v0, o);
+    const unsigned long long o1 = __shfl_xor_sync(0xffffffffu, v1, o);
+    const bool keep_min = ((lane & o) == 0) == up;
+    v0 = keep_min ? (v0 < o0 ? v0 : o0) : (v0 > o0 ? v0 : o0);
+    v1 = keep_min ? (v1 < o1 ? v1 : o1) : (v1 > o1 ? v1 : o1);
 }
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
@@ -75,7 +95,7 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     // Unique 64-bit keys: ~bits(S) (ascending = S descending, valid for
     // S >= 0) above the position-major id, so an ascending sort is the stable
     // sort by S descending.  Padding keys sort last.
-    int n2 = 1;
+    int n2 = 64;
     while (n2 < N) n2 <<= 1;
     for (int id = tid; id < n2; id += blockDim.x) {
         unsigned long long k = ~0ull;
@@ -88,9 +108,19 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
         keys[id] = k;
     }
     __syncthreads();
-    // Bitonic sort in shared memory: one compare-exchange per pair per stage.
-    for (int k = 2; k <= n2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
+    const int nchunks = n2 >> 6, nwarps = blockDim.x >> 5;
+    // Block sizes 2..64: every stage stays inside one 64-key chunk.
+    for (int c = wid; c < nchunks; c += nwarps) {
+        const int e0 = c * 64 + 2 * lane;
+        unsigned long long v0 = keys[e0], v1 = keys[e0 + 1];
+        for (int k = 2; k <= 64; k <<= 1)
+            for (int j = k >> 1; j > 0; j >>= 1) bitonic_warp_step(v0, v1, e0, k, j);
+        keys[e0] = v0;
+        keys[e0 + 1] = v1;
+    }
+    __syncthreads();
+    for (int k = 128; k <= n2; k <<= 1) {
+        for (int j = k >> 1; j >= 64; j >>= 1) {
             for (int i = tid; i < (n2 >> 1); i += blockDim.x) {
                 const int lo = 2 * i - (i & (j - 1)), hi = lo + j;
                 const bool up = (lo & k) == 0;
@@ -99,6 +129,14 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
             }
             __syncthreads();
         }
+        for (int c = wid; c < nchunks; c += nwarps) {
+            const int e0 = c * 64 + 2 * lane;
+            unsigned long long v0 = keys[e0], v1 = keys[e0 + 1];
+            for (int j = 32; j > 0; j >>= 1) bitonic_warp_step(v0, v1, e0, k, j);
+            keys[e0] = v0;
+            keys[e0 + 1] = v1;
+        }
+        __syncthreads();
     }
 
     // fp64 prefix of the sorted survivals: V_n = B + sum_{j<n} S_(j).  Thread t

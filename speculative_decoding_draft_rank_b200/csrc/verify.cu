@@ -396,63 +396,67 @@ __device__ __forceinline__ void row_stats(const VerifyWs &w, int j, float invT, 
 
 // Inverse-CDF draw from target row j (compacted index; request b, position
 // k) with row stats (M, Z): prefix over the chunk sums, then the chosen chunk
-// rescanned in index order.  Whole block; returns the token.
+// rescanned in index order, each thread owning 32 consecutive columns loaded
+// at once.  Whole block (kRowThreads threads); returns the token.
 template <typename T>
 __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, int j, int b, int k,
-                                 int G, int V, float M, float Z, float invT, float u, float *red,
-                                 int *redi) {
+                                 int G, int V, float M, float Z, float invT, float u) {
+    __shared__ float s_c[32], s_e[32];
+    __shared__ int s_i0[32], s_i1[32], s_i2[32], s_i3[32];
+    __shared__ float excl_s;
+    __shared__ int col_s;
     const int tid = threadIdx.x;
     const float *cm = w.cm + (size_t)j * w.nChunks;
     const float *cs = w.cs + (size_t)j * w.nChunks;
     const float target = u * Z;
     // Prefix over chunk sums (nChunks <= 128 for V <= 2^20; kRowThreads >= that).
-    float wc = tid < w.nChunks ? cs[tid] * exp_e((cm[tid] - M) * invT) : 0.f;
+    const float wc = tid < w.nChunks ? cs[tid] * exp_e((cm[tid] - M) * invT) : 0.f;
     float tot;
-    float inc = block_incl_scan(wc, red, &tot);
-    int cs_ = (tid < w.nChunks && inc > target) ? tid : 0x7fffffff;
-    cs_ = block_min_i(cs_, redi);
-    if (cs_ == 0x7fffffff) {
-        int lc = (tid < w.nChunks && wc > 0.f) ? tid : -1;
-        cs_ = -block_min_i(-lc, redi);
-        if (cs_ < 0) cs_ = w.nChunks - 1;
+    const float inc = block_scan1(wc, s_c, &tot);
+    int ch = block_min1((tid < w.nChunks && inc > target) ? tid : 0x7fffffff, s_i0);
+    if (ch == 0x7fffffff) {
+        ch = block_max1_i((tid < w.nChunks && wc > 0.f) ? tid : -1, s_i1);
+        if (ch < 0) ch = w.nChunks - 1;
     }
-    __shared__ float excl_s;
-    if (tid == cs_) excl_s = inc - wc;
+    if (tid == ch) excl_s = inc - wc;
     __syncthreads();
-    float rem = target - excl_s;
+    const float rem = target - excl_s;
     const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
-    const int c0 = cs_ * kChunk, c1 = min(V, c0 + kChunk);
-    int found = 0x7fffffff, lastpos = -1;
+    const int c0 = ch * kChunk, c1 = min(V, c0 + kChunk);
+    const int i0 = c0 + tid * 32;   // this thread's 32 consecutive columns
+    float e[32];
+    float run = 0.f;
+#pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const int i = c0 + (q * kRowThreads + tid) * 8;
         float v[8];
-        float e[8];
-        float run = 0.f;
+        const int i = i0 + q * 8;
         if (i < c1) load8(row, i, c1, v);
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-            e[t] = (i < c1 && i + t < c1) ? exp_e((v[t] - M) * invT) : 0.f;
-            run += e[t];
-            if (e[t] > 0.f) lastpos = i + t;
+            e[q * 8 + t] = (i + t < c1) ? exp_e((v[t] - M) * invT) : 0.f;
+            run += e[q * 8 + t];
         }
-        float rt;
-        float incl = block_incl_scan(run, red, &rt);
+    }
+    float rt;
+    const float incl = block_scan1(run, s_e, &rt);
+    int owner = block_min1((incl > rem && run > 0.f) ? tid : 0x7fffffff, s_i2);
+    if (owner == 0x7fffffff) owner = max(0, block_max1_i(run > 0.f ? tid : -1, s_i3));
+    if (tid == owner) {
         float p = incl - run;
-        int f = 0x7fffffff;
+        int f = -1, lastpos = -1;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            p += e[t];
-            if (f == 0x7fffffff && e[t] > 0.f && p > rem) f = i + t;
+        for (int t = 0; t < 32; ++t) {
+            if (f < 0 && e[t] > 0.f) {
+                lastpos = i0 + t;
+                p += e[t];
+                if (p > rem) f = i0 + t;
+            }
         }
-        f = block_min_i(f, redi);
-        if (f != 0x7fffffff) { found = f; break; }
-        rem -= rt;
+        if (f < 0) f = lastpos >= 0 ? lastpos : c1 - 1;
+        col_s = f;
     }
-    if (found == 0x7fffffff) {
-        found = -block_min_i(-lastpos, redi);
-        if (found < 0) found = c1 - 1;
-    }
-    return found;
+    __syncthreads();
+    return col_s;
 }
 
 // ----------------------------------------------------------------- decide
@@ -466,14 +470,26 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     int32_t *__restrict__ nout_out, float *__restrict__ pt_x_out) {
     __shared__ float rM[17], rZ[17];
     __shared__ int rA[17];
-    __shared__ float red[33];
-    __shared__ int redi[33];
+    __shared__ int acc_s[16];
     __shared__ int A_s;
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float Tb = sane_temp(temp[b], w.hdr);
     const float invT = Tb > 0.f ? 1.f / Tb : 0.f;
     int lb = ell[b];
     lb = lb < 0 ? 0 : (lb > G ? G : lb);
+    // Thread k < G fetches what the accept test of position k needs before
+    // the row statistics are in.
+    const size_t o = (size_t)b * G + tid;
+    int xk = 0;
+    float tk = 0.f, uk = 0.f, pdk = 1.f;
+    if (tid < lb) {
+        xk = clamp_token(x[o], V, w.hdr);
+        if (Tb > 0.f) {
+            tk = to_f32(Tlog[((size_t)b * (G + 1) + tid) * V + xk]);
+            uk = u_accept[o];
+            pdk = pd_x[o];
+        }
+    }
     const int j0 = w.row_off[b];
     for (int k = wid; k <= lb; k += kRowThreads / 32) {
         float M, Z;
@@ -482,37 +498,29 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
         if (lane == 0) { rM[k] = M; rZ[k] = Z; rA[k] = A; }
     }
     __syncthreads();
+    if (tid < G) {
+        float pt = -1.f;
+        int acc = 0;
+        if (tid < lb) {
+            if (Tb == 0.f) {
+                acc = rA[tid] == xk;
+                pt = acc ? 1.f : 0.f;
+            } else {
+                pt = exp_e((tk - rM[tid]) * invT) / rZ[tid];
+                acc = uk < pt / pdk;
+            }
+        }
+        acc_s[tid] = acc;
+        if (pt_x_out != nullptr) pt_x_out[o] = pt;
+    }
+    __syncthreads();
     if (tid == 0) {
         int A = 0;
-        bool rejected = false;
-        for (int k = 0; k < G; ++k) {
-            const size_t o = (size_t)b * G + k;
-            float pt = -1.f;
-            if (k < lb) {
-                const int xk = clamp_token(x[o], V, w.hdr);
-                bool acc;
-                if (Tb == 0.f) {
-                    acc = (rA[k] == xk);
-                    pt = acc ? 1.f : 0.f;
-                } else {
-                    const float t = to_f32(Tlog[((size_t)b * (G + 1) + k) * V + xk]);
-                    pt = exp_e((t - rM[k]) * invT) / rZ[k];
-                    acc = u_accept[o] < pt / pd_x[o];
-                }
-                if (!rejected) {
-                    if (acc) ++A; else rejected = true;
-                }
-            }
-            if (pt_x_out != nullptr) pt_x_out[o] = pt;
-        }
+        while (A < lb && acc_s[A]) ++A;   // the first rejection discards the rest
         A_s = A;
         acc_out[b] = A;
         nout_out[b] = A + 1;
-        int32_t *tok = tokens_out + (size_t)b * (G + 1);
-        for (int q = 0; q <= G; ++q) tok[q] = q < A ? x[(size_t)b * G + q] : -1;
-        if (Tb == 0.f) {
-            tok[A] = (rA[A] >= 0 && rA[A] < V) ? rA[A] : 0;
-        } else if (A < lb) {  // queue the rejected row for the residual draw
+        if (Tb > 0.f && A < lb) {  // queue the rejected row for the residual draw
             const int slot = atomicAdd(&w.hdr->pad[1], 1u);
             w.res_b[slot] = b;
             w.res_k[slot] = A;
@@ -522,11 +530,15 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     }
     __syncthreads();
     const int A = A_s;
-    if (Tb > 0.f && A == lb) {  // bonus (fresh token when nothing was admitted)
-        const int y = sample_target_row(Tlog, w, j0 + lb, b, lb, G, V, rM[lb], rZ[lb], invT,
-                                        u_final[b], red, redi);
-        if (tid == 0) tokens_out[(size_t)b * (G + 1) + A] = y;
-    }
+    // Token A: the greedy target token, the bonus draw from p_t at row lb
+    // (a fresh token when nothing was admitted), or -1 until the residual
+    // draw replaces it.
+    int fin = -1;
+    if (Tb == 0.f)
+        fin = (rA[A] >= 0 && rA[A] < V) ? rA[A] : 0;
+    else if (A == lb)   // block-uniform
+        fin = sample_target_row(Tlog, w, j0 + lb, b, lb, G, V, rM[lb], rZ[lb], invT, u_final[b]);
+    if (tid <= G) tokens_out[(size_t)b * (G + 1) + tid] = tid < A ? x[(size_t)b * G + tid] : (tid == A ? fin : -1);
 }
 
 // ----------------------------------------------------------------- residual
@@ -608,6 +620,12 @@ __global__ void __launch_bounds__(256) residual_tile_simt(
     }
 }
 
+// Replacement token of a queued rejection: thread t owns the contiguous tile
+// sums [t K, t K + K) (loaded before any barrier), one block scan gives Q and
+// the thread whose range holds u Q, which walks its sums to the crossing
+// tile; the block recomputes that tile's q values and scans them.
+constexpr int kResChunk = 8;   // tile sums per thread held in registers
+
 template <typename T>
 __global__ void __launch_bounds__(kRowThreads) residual_final(
     const T *__restrict__ Tlog, const T *__restrict__ L, const T *__restrict__ U,
@@ -616,76 +634,96 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
     const float *__restrict__ temp, const float *__restrict__ u_final, int G, int V, int r,
     VerifyWs w, int32_t *__restrict__ tokens_out) {
     extern __shared__ float res_smem[];
-    float *pref = res_smem;               // [nResTiles]
-    float *urow = res_smem + w.nResTiles; // [r]
-    __shared__ float red[33];
-    __shared__ int redi[33];
-    __shared__ float carry_s;
-    const int s = blockIdx.x, tid = threadIdx.x;
+    float *urow = res_smem;   // [r]
+    __shared__ float s_loc[32], s_col[32];
+    __shared__ int s_own[32], s_own2[32], s_y[32], s_y2[32];
+    __shared__ int ts_s;
+    __shared__ float rem_s;
+    const int s = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
     const int nres = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[1]);
     if (s >= nres) return;
+    const int nT = w.nResTiles;
+    const float *tp = w.rp + (size_t)s * nT;
+    const int K = (nT + nthr - 1) / nthr;
+    const int t0 = min(nT, tid * K), t1 = min(nT, t0 + K);
+    float cq[kResChunk];
+#pragma unroll
+    for (int q = 0; q < kResChunk; ++q) cq[q] = t0 + q < t1 ? tp[t0 + q] : 0.f;
     const int b = w.res_b[s], k = w.res_k[s];
-    const float Tb = fmaxf(temp[b], 0.f), invT = 1.f / Tb;
     const size_t ro = (size_t)b * G + k;
+    const float Tb = fmaxf(temp[b], 0.f), invT = 1.f / Tb;
     const float Md = rowmax[ro], Zd = rowsum[ro], Mt = w.res_mt[s], Zt = w.res_zt[s];
-    const float *tp = w.rp + (size_t)s * w.nResTiles;
-    if (tid == 0) carry_s = 0.f;
-    __syncthreads();
-    for (int t0 = 0; t0 < w.nResTiles; t0 += blockDim.x) {
-        const int t = t0 + tid;
-        float v = t < w.nResTiles ? tp[t] : 0.f;
-        float tot;
-        float inc = block_incl_scan(v, red, &tot);
-        const float c = carry_s;
-        if (t < w.nResTiles) pref[t] = c + inc;
-        __syncthreads();
-        if (tid == 0) carry_s = c + tot;
-        __syncthreads();
-    }
-    const float Q = carry_s;
     const float u = u_final[b];
+    const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
+    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
+    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+    float loc = 0.f;
+#pragma unroll
+    for (int q = 0; q < kResChunk; ++q) loc += cq[q];
+    for (int t = t0 + kResChunk; t < t1; ++t) loc += tp[t];   // very large vocabularies only
+    if (tid < r) urow[tid] = uv0;
+    if (tid + nthr < r) urow[tid + nthr] = uv1;
+    float Q;
+    const float incl = block_scan1(loc, s_loc, &Q);   // also publishes urow
     int y;
-    if (!(Q > 0.f)) {  // empty residual: draw from p_t of the rejected row
-        y = sample_target_row(Tlog, w, w.row_off[b] + k, b, k, G, V, Mt, Zt, invT, u, red, redi);
+    if (!(Q > 0.f)) {  // empty residual (block-uniform): draw from p_t of the rejected row
+        y = sample_target_row(Tlog, w, w.row_off[b] + k, b, k, G, V, Mt, Zt, invT, u);
     } else {
         const float target = u * Q;
-        int ts = 0x7fffffff;
-        for (int t = tid; t < w.nResTiles; t += blockDim.x)
-            if (pref[t] > target) ts = min(ts, t);
-        ts = block_min_i(ts, redi);
-        if (ts == 0x7fffffff) {
-            int lt = -1;
-            for (int t = tid; t < w.nResTiles; t += blockDim.x)
-                if (tp[t] > 0.f) lt = max(lt, t);
-            ts = -block_min_i(-lt, redi);
-            if (ts < 0) ts = w.nResTiles - 1;
+        int owner = block_min1((incl > target && loc > 0.f) ? tid : 0x7fffffff, s_own);
+        if (owner == 0x7fffffff) owner = max(0, block_max1_i(loc > 0.f ? tid : -1, s_own2));
+        if (tid == owner) {
+            float run = incl - loc, run_last = run;
+            int ts = -1, last = t1 - 1;
+#pragma unroll
+            for (int q = 0; q < kResChunk; ++q) {
+                if (ts < 0 && t0 + q < t1) {
+                    if (run + cq[q] > target) {
+                        ts = t0 + q;
+                    } else {
+                        if (cq[q] > 0.f) { last = t0 + q; run_last = run; }
+                        run += cq[q];
+                    }
+                }
+            }
+            for (int t = t0 + kResChunk; t < t1 && ts < 0; ++t) {
+                const float wt = tp[t];
+                if (run + wt > target) {
+                    ts = t;
+                } else {
+                    if (wt > 0.f) { last = t; run_last = run; }
+                    run += wt;
+                }
+            }
+            if (ts < 0) { ts = last; run = run_last; }
+            ts_s = max(ts, 0);
+            rem_s = target - run;
         }
-        const float rem = target - (ts > 0 ? pref[ts - 1] : 0.f);
-        const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
-        for (int q = tid; q < r; q += blockDim.x) urow[q] = ld_elem(U, (size_t)prev * r + q);
         __syncthreads();
+        const int ts = ts_s;
+        const float rem = rem_s;
         // tpc consecutive threads share one column's dot product.
         const int TN = w.resCols;
         const int c0 = ts * TN;
-        const int tpc = blockDim.x / TN;
+        const int tpc = nthr / TN;
         const int col = c0 + tid / tpc, part = tid % tpc;
         const bool mine = part == 0 && col < V;
+        const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;
+        const float tval = mine ? ld_elem(Tlog, ((size_t)b * (G + 1) + k) * V + col) : 0.f;
         float dl = 0.f;
         if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
         for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
         float qv = 0.f;
         if (mine) {
-            const float pd = exp_e(((ld_elem(L, ro * V + col) - Md) + dl) * invT) / Zd;
-            const float pt = exp_e((ld_elem(Tlog, ((size_t)b * (G + 1) + k) * V + col) - Mt) * invT) / Zt;
+            const float pd = exp_e(((lval - Md) + dl) * invT) / Zd;
+            const float pt = exp_e((tval - Mt) * invT) / Zt;
             qv = fmaxf(pt - pd, 0.f);
         }
         float tot;
-        float inc = block_incl_scan(qv, red, &tot);
-        int ys = (mine && qv > 0.f && inc > rem) ? col : 0x7fffffff;
-        ys = block_min_i(ys, redi);
+        const float inc = block_scan1(qv, s_col, &tot);
+        int ys = block_min1((mine && qv > 0.f && inc > rem) ? col : 0x7fffffff, s_y);
         if (ys == 0x7fffffff) {
-            int lc = (mine && qv > 0.f) ? col : -1;
-            ys = -block_min_i(-lc, redi);
+            ys = block_max1_i((mine && qv > 0.f) ? col : -1, s_y2);
             if (ys < 0) ys = min(c0 + TN, V) - 1;
         }
         y = ys;
@@ -734,7 +772,7 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
                                                   a.rowsum, a.temp, a.G, a.V, a.r, w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    const size_t smem = sizeof(float) * ((size_t)w.nResTiles + a.r);
+    const size_t smem = sizeof(float) * (size_t)a.r;
     auto fin = residual_final<T>;
     if (smem > 48 * 1024) {
         if ((e = cudaFuncSetAttribute(fin, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=

@@ -153,17 +153,25 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
     const float *__restrict__ u_draft, int B, int G, int V, int r, int pos, int nTiles, int TN,
     const float *__restrict__ part_m, const float *__restrict__ part_s,
     const int32_t *__restrict__ part_a, int32_t *__restrict__ x_out, float *__restrict__ pd_out,
-    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out, WsHeader *hdr)
+    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out, __nv_bfloat16 *__restrict__ E,
+    WsHeader *hdr)
 {
     extern __shared__ float fin_smem[];
     float *urow = fin_smem;                 // [r] U[x_{i-1}] row
     __shared__ float s_max[32], s_loc[32], s_col[32];
     __shared__ int s_own[32], s_own2[32], s_x[32], s_x2[32];
-    __shared__ int ts_s;
+    __shared__ int ts_s, xg_s;
     __shared__ float rem_s;
 
     const int b = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
     const size_t ro = (size_t)b * G + pos;
+    // bf16 rounds: the sampled token's U row is staged in E[b] for the next
+    // position's tensor-core pass (16-byte pieces; r is a multiple of 16).
+    auto stage_next = [&](int x) {
+        if (E != nullptr && pos + 1 < G)
+            for (int q = tid; q < r / 8; q += nthr)
+                reinterpret_cast<uint4 *>(E + (size_t)b * r)[q] = ld_nc16(U + (size_t)x * r + q * 8);
+    };
     const float *pm = part_m + (size_t)b * nTiles;
     const float *ps = part_s + (size_t)b * nTiles;
     const int K = (nTiles + nthr - 1) / nthr;
@@ -207,6 +215,11 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
             pd_out[ro] = 1.f;
             rowmax_out[ro] = M;
             rowsum_out[ro] = 1.f;
+            xg_s = x;
+        }
+        if (E != nullptr && pos + 1 < G) {
+            __syncthreads();
+            stage_next(xg_s);
         }
         return;
     }
@@ -279,6 +292,7 @@ __global__ void __launch_bounds__(kFinThreads) draft_finalize(
         rowmax_out[ro] = M;
         rowsum_out[ro] = Z;
     }
+    stage_next(xs);
 }
 
 // ---------------------------------------------------------------------------
@@ -293,6 +307,7 @@ size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_m
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_s
     bytes += align256(sizeof(int32_t) * (size_t)B * nt);  // part_a
+    if (dtype == DSPARK_BF16) bytes += align256((size_t)B * r * 2);   // E
     return bytes;
 }
 
@@ -305,6 +320,8 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     w.part_m = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
     w.part_s = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
     w.part_a = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (size_t)B * nt);
+    w.E = nullptr;
+    if (dtype == DSPARK_BF16) { w.E = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)B * r * 2); }
     w.nTiles = (int)nt;
     return w;
 }
@@ -320,7 +337,8 @@ static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos
     kern<<<a.B, kFinThreads, smem, st>>>(static_cast<const T *>(a.L), static_cast<const T *>(a.U),
                                          static_cast<const T *>(a.Wt), a.x0, a.temp, a.u_draft, a.B, a.G, a.V,
                                          a.r, pos, w.nTiles, draft_tile_cols(a.dtype), w.part_m, w.part_s,
-                                         w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out, w.hdr);
+                                         w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out,
+                                         reinterpret_cast<__nv_bfloat16 *>(w.E), w.hdr);
     return cudaGetLastError();
 }
 

@@ -59,11 +59,16 @@ struct TcLayout {
     uint32_t a_off, b_off, l_off, bar_off, total;
 };
 
+// Every epilogue warp group owns one logit slot (segment sg of each tile goes
+// to slot sg), so a group only ever waits on phases of its own slot; the B
+// ring takes what shared memory is left (3 stages for r <= 256, 1 for r = 512).
 __host__ __device__ inline TcLayout tc_layout(int r) {
     TcLayout t;
     t.nkb = (r + kKB - 1) / kKB;
-    t.sB = t.nkb <= 4 ? 3 : 2;       // B ring depth
-    t.sL = t.nkb <= 4 ? 4 : 2;       // logit segment ring depth
+    t.sL = kSegs;
+    const int fixed = t.nkb * kABlockBytes + t.sL * kSegBytes + 256 + 1024;
+    int sB = (227 * 1024 - fixed) / kStageBytes;
+    t.sB = sB > 3 ? 3 : (sB < 1 ? 1 : sB);   // B ring depth
     t.a_off = 0;
     t.b_off = t.a_off + t.nkb * kABlockBytes;
     t.l_off = t.b_off + t.sB * kStageBytes;
@@ -78,6 +83,7 @@ enum { kEpiDraft = 0, kEpiResidual = 1 };
 struct TcEpi {
     const float *temp;
     int B, G, V, pos, nParts;
+    int a_tma;                // 1: the A rows come from the staged E by TMA (drafting, positions >= 2)
     WsHeader *hdr;
     const __nv_bfloat16 *U;   // [V, r]: A-operand rows are U[previous token]
     const int32_t *x0;        // [B] last committed tokens
@@ -97,7 +103,8 @@ struct TcEpi {
 
 template <int MODE>
 __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_constant__ CUtensorMap mapW,
-                                                              const __grid_constant__ CUtensorMap mapL, int r,
+                                                              const __grid_constant__ CUtensorMap mapL,
+                                                              const __grid_constant__ CUtensorMap mapE, int r,
                                                               int nTilesN, const TcEpi ep)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -109,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     unsigned char *sL = base + lay.l_off;
     const int SB = lay.sB, SL = lay.sL, nkb = lay.nkb;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar_off);
-    uint64_t *a_full = bars;                 // 16 epilogue-warp arrivals: A is in shared memory
+    uint64_t *a_full = bars;                 // A is in shared memory (16 epilogue-warp arrivals, or the TMA bytes)
     uint64_t *b_full = a_full + 1;           // SB
     uint64_t *b_empty = b_full + SB;         // SB
     uint64_t *l_full = b_empty + SB;         // SL
@@ -133,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     if (m0 >= nrows) return;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(a_full, kEpiWarps);
+        tc::mbar_init(a_full, ep.a_tma ? 1 : kEpiWarps);
         for (int q = 0; q < SB; ++q) { tc::mbar_init(&b_full[q], 1); tc::mbar_init(&b_empty[q], 1); }
         for (int q = 0; q < SL; ++q) { tc::mbar_init(&l_full[q], 1); tc::mbar_init(&l_empty[q], 4); }
         for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], kEpiWarps); }
@@ -155,6 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         if (lane == 0) {
             tc::prefetch_tmap(&mapW);
             const uint64_t keep = tc::policy_evict_last();
+            if (ep.a_tma) {   // the staged A rows first: the MMA waits for them
+                const uint64_t once = tc::policy_evict_first();
+                tc::mbar_arrive_expect_tx(a_full, (uint32_t)nkb * kABlockBytes);
+                for (int kb = 0; kb < nkb; ++kb)
+                    tc::tma_load_2d(sA + kb * kABlockBytes, &mapE, a_full, kb * kKB, m0, once);
+            }
             int g = 0;
             bool ok = true;
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
@@ -178,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const int gg = g - 1 - q;
                     tc::mbar_wait_bounded(&b_full[gg % SB], (gg / SB) & 1, no_abort, kWaitBudget / 4);
                 }
+                if (ep.a_tma) tc::mbar_wait_bounded(a_full, 0, no_abort, kWaitBudget / 4);
                 flag_status(hdr, DSPARK_DEV_TIMEOUT);
             }
         }
@@ -260,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         // token, x0 at the first position, or for a queued rejection the token
         // before it).  This warp writes k-blocks kb = sg, sg + 4, ... of its
         // 32 rows in the 128-byte-swizzled K-major layout (zeros past r).
-        {
+        if (!ep.a_tma) {
             int prev = 0;
             if (MODE == kEpiDraft) {
                 const int b = m0 + row;
@@ -327,6 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
                     cur[u] = *reinterpret_cast<const uint4 *>(lsrc + ((u ^ (row & 7)) << 4));
+                // The segment is in registers: hand the slot back to the
+                // producer now, so the next tile's copy overlaps this one's math.
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&l_empty[q]);
                 const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
                 const int cbase = t * kBN + sg * kSeg;
                 const bool whole = cbase + kSeg <= V;   // no column of this segment lies past V
@@ -376,12 +395,8 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     m = mn;
                 }
                 tc::tc_fence_before();
-                tc::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    tc::mbar_arrive(&acc_empty[ab]);
-                    tc::mbar_arrive(&l_empty[q]);
-                }
+                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
                 const int p = t * kSegs + sg;
                 if (rowok && p < nParts) {
                     const size_t o = (size_t)b * nParts + p;
@@ -509,11 +524,31 @@ bool map_logits(CUtensorMap *m, const void *L, int B, int G, int V) {
     return res == CUDA_SUCCESS;
 }
 
+// Tensor map of the staged A rows E [B, r] (bf16): 64 x 128 boxes (one
+// k-block of one 128-row block), 128-byte swizzle, rows past B read as zero.
+bool map_stage(CUtensorMap *m, const void *E, int B, int r) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)B};
+    cuuint64_t strides[1] = {(cuuint64_t)r * 2};
+    cuuint32_t box[2] = {kKB, kM};
+    cuuint32_t es[2] = {1, 1};
+    CUresult res = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(E), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return res == CUDA_SUCCESS;
+}
+
 template <int MODE>
-cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, cudaStream_t st) {
-    CUtensorMap mW, mL;
+cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, const void *E, cudaStream_t st) {
+    CUtensorMap mW, mL, mE;
     if (!map_factor(&mW, Wt, ep.V, r)) return cudaErrorInvalidValue;
     if (!map_logits(&mL, ep.L, ep.B, ep.G, ep.V)) return cudaErrorInvalidValue;
+    if (ep.a_tma) {
+        if (!map_stage(&mE, E, ep.B, r)) return cudaErrorInvalidValue;
+    } else {
+        mE = mW;   // unused
+    }
     const TcLayout lay = tc_layout(r);
     cudaError_t e = cudaFuncSetAttribute(markov_tile_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)lay.total);
@@ -525,7 +560,7 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, cudaStream_
     const int nMB = (ep.B + kM - 1) / kM;
     int grid = std::min(sms, nMB * nTilesN);
     grid = std::max(grid, nMB);
-    markov_tile_tc<MODE><<<grid, kThreads, lay.total, st>>>(mW, mL, r, nTilesN, ep);
+    markov_tile_tc<MODE><<<grid, kThreads, lay.total, st>>>(mW, mL, mE, r, nTilesN, ep);
     return cudaGetLastError();
 }
 
@@ -537,7 +572,8 @@ cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, 
     ep.U = static_cast<const __nv_bfloat16 *>(a.U); ep.x0 = a.x0; ep.x = a.x_out;
     ep.L = static_cast<const __nv_bfloat16 *>(a.L);
     ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
-    return launch_markov_tc<kEpiDraft>(a.Wt, a.r, ep, st);
+    ep.a_tma = (pos > 0 && w.E != nullptr) ? 1 : 0;   // position 0 gathers U[x0] itself
+    return launch_markov_tc<kEpiDraft>(a.Wt, a.r, ep, w.E, st);
 }
 
 cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st) {
@@ -546,7 +582,8 @@ cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st) {
     ep.U = a.U; ep.x0 = a.x0; ep.x = a.x; ep.L = a.L;
     ep.nrows = a.nrows; ep.res_b = a.res_b; ep.res_k = a.res_k; ep.res_mt = a.res_mt; ep.res_zt = a.res_zt;
     ep.rowmax = a.rowmax; ep.rowsum = a.rowsum; ep.Tlog = a.Tlog; ep.rp = a.rp;
-    return launch_markov_tc<kEpiResidual>(a.Wt, a.r, ep, st);
+    ep.a_tma = 0;
+    return launch_markov_tc<kEpiResidual>(a.Wt, a.r, ep, nullptr, st);
 }
 
 }  // namespace dspark

@@ -25,6 +25,7 @@ struct DraftWs {
     WsHeader *hdr;
     float *part_m, *part_s;
     int32_t *part_a;
+    __nv_bfloat16 *E;   // bf16 only: [B, r] rows U[x_i] staged for the next position's MMA
     int nTiles;
 };
 

@@ -44,7 +44,8 @@ PROFILE = (np.array([0, 20, 60], np.int32), np.array([10.0, 11.0, 14.0]))
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("B,G,V,r,d", [(37, 5, 5000, 32, 96), (9, 3, 1288, 16, 40), (64, 8, 3072, 64, 256),
-                                       (130, 4, 9000, 256, 128), (200, 2, 2056, 80, 64)])
+                                       (130, 4, 9000, 256, 128), (200, 2, 2056, 80, 64),
+                                       (150, 3, 4104, 320, 64), (70, 3, 3000, 512, 64)])
 def test_round_parity_small(dtype, B, G, V, r, d):
     temps = np.tile(np.float32([1.0, 0.0, 0.6, 1.2]), B)[:B]
     inp, dr = _round(B, G, V, r, d, dtype, seed=B + V, knots_n=PROFILE[0], knots_t=PROFILE[1], temps=temps)

@@ -11,8 +11,9 @@
 // Launch sequence (fixed, graph-capturable; work counts live on the device):
 //   plan        1 CTA: row list of the admitted target rows, rows (b, k) for
 //               k = 0..ell_b (0-based), and their offsets per request.
-//   rows        persistent grid over (row, 8192-column chunk) work items:
-//               one streaming pass over each target row with 16-byte loads,
+//   rows        persistent grid over (row, 8192-column chunk) work items,
+//               one warp per item (bf16: 32-byte loads two steps ahead):
+//               one streaming pass over each target row,
 //               giving per chunk the max, lowest argmax and sum of
 //               exp((t - max) / T).
 //   decide      1 CTA per request: row max / Z from the chunk partials,
@@ -244,94 +245,107 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
     }
 }
 
-// bf16 rows: each chunk is one contiguous 16-byte-aligned run, so thread 0
-// streams the CTA's work items into a 3-stage shared-memory ring with bulk
-// async copies (evict-first), keeping up to three 16 KB chunks in flight per
-// CTA while the block reduces the oldest.  Waits are bounded.
-constexpr int kRowStages = 3;
+// bf16 rows: one warp per (row, 8192-column chunk) work item, no block
+// barriers.  The warp walks its chunk in eight 1024-column steps; lane l owns
+// columns [l * 32, l * 32 + 32) of a step, read with two 32-byte loads (four
+// 16-byte ones when rows are not 32-byte aligned) issued two steps ahead.
+// Each lane keeps an online (max, sum of exp((t - max) / T)) -- or, for a
+// greedy row, the lowest argmax -- and a warp merge writes the chunk partial.
+constexpr int kRowsWarpThreads = 256;
+constexpr int kStep = 1024;                 // columns per warp step
+constexpr int kSteps = kChunk / kStep;      // 8
 
-__global__ void __launch_bounds__(kRowThreads) verify_rows_bulk(const __nv_bfloat16 *__restrict__ Tlog,
-                                                                const float *__restrict__ temp, int G, int V,
-                                                                VerifyWs w) {
-    extern __shared__ __align__(128) unsigned char rows_smem[];
-    __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(rows_smem);   // [kRowStages][kChunk]
-    __shared__ __align__(8) uint64_t full[kRowStages];
-    __shared__ float rm[8], rs[8];
-    __shared__ int ra[8];
-    __shared__ int abort_s;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+// 32 bf16 of a row from column c (c a multiple of 32) into w; past n reads as
+// -inf (bf16 0xff80).
+__device__ __forceinline__ void ld_row32(const __nv_bfloat16 *row, int c, int n, bool a32, uint32_t (&w)[16]) {
+    const __nv_bfloat16 *p = row + c;
+    if (a32 && c + 32 <= n) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(w[h * 8 + 0]), "=r"(w[h * 8 + 1]), "=r"(w[h * 8 + 2]), "=r"(w[h * 8 + 3]),
+                           "=r"(w[h * 8 + 4]), "=r"(w[h * 8 + 5]), "=r"(w[h * 8 + 6]), "=r"(w[h * 8 + 7])
+                         : "l"(p + h * 16));
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (c + q * 8 + 8 <= n && ((reinterpret_cast<uintptr_t>(p + q * 8) & 15) == 0)) {
+                const uint4 v = ld_stream16(p + q * 8);
+                w[q * 4 + 0] = v.x; w[q * 4 + 1] = v.y; w[q * 4 + 2] = v.z; w[q * 4 + 3] = v.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int i0 = c + q * 8 + e * 2;
+                    const uint32_t lo = i0 < n ? (uint32_t)__bfloat16_as_ushort(p[q * 8 + e * 2]) : 0xff80u;
+                    const uint32_t hi = i0 + 1 < n ? (uint32_t)__bfloat16_as_ushort(p[q * 8 + e * 2 + 1]) : 0xff80u;
+                    w[q * 4 + e] = lo | (hi << 16);
+                }
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kRowsWarpThreads, 3) verify_rows_warp(const __nv_bfloat16 *__restrict__ Tlog,
+                                                                     const float *__restrict__ temp, int G, int V,
+                                                                     VerifyWs w) {
+    const int lane = threadIdx.x & 31;
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
     const int nwork = nrows * w.nChunks;
-    if ((int)blockIdx.x >= nwork) return;
-    const int my_items = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
-    auto issue = [&](int k) {  // k-th item of this CTA into stage k % kRowStages
-        const int item = blockIdx.x + k * gridDim.x;
+    const int nwarps = gridDim.x * (blockDim.x >> 5);
+    const bool a32 = (V & 15) == 0 && (reinterpret_cast<uintptr_t>(Tlog) & 31) == 0;
+    for (int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); item < nwork; item += nwarps) {
         const int j = item / w.nChunks, c = item - j * w.nChunks;
         const int rk = w.rows[j], b = rk >> 5, kk = rk & 31;
-        const int c0 = c * kChunk, n = min(V, c0 + kChunk) - c0;
-        const __nv_bfloat16 *src = Tlog + ((size_t)b * (G + 1) + kk) * V + c0;
-        uint64_t *bar = &full[k % kRowStages];
-        tc::mbar_arrive_expect_tx(bar, (uint32_t)n * 2);
-        asm volatile(
-            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-            " [%0], [%1], %2, [%3], %4;" ::"r"(tc::smem_u32(stage + (size_t)(k % kRowStages) * kChunk)),
-            "l"(src), "r"(n * 2), "r"(tc::smem_u32(bar)), "l"(tc::policy_evict_first())
-            : "memory");
-    };
-    if (tid == 0) {
-        for (int q = 0; q < kRowStages; ++q) tc::mbar_init(&full[q], 1);
-        tc::fence_barrier_init();
-        abort_s = 0;
-        for (int k = 0; k < kRowStages && k < my_items; ++k) issue(k);
-    }
-    __syncthreads();
-    for (int k = 0; k < my_items; ++k) {
-        const int item = blockIdx.x + k * gridDim.x;
-        const int j = item / w.nChunks, c = item - j * w.nChunks;
-        const int b = w.rows[j] >> 5;
+        const __nv_bfloat16 *row = Tlog + ((size_t)b * (G + 1) + kk) * V;
         float Tb = temp[b];
         Tb = Tb >= 0.f ? Tb : 0.f;
         const float cexp = Tb > 0.f ? kLog2e / Tb : 0.f;
-        const int c0 = c * kChunk, n = min(V, c0 + kChunk) - c0;
-        const bool ok = tc::mbar_wait_bounded(&full[k % kRowStages], (k / kRowStages) & 1, &abort_s,
-                                              2000000000LL);
-        if (!__syncthreads_and(ok)) {
-            if (tid == 0) flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
-            break;
-        }
-        const __nv_bfloat16 *st = stage + (size_t)(k % kRowStages) * kChunk;
-        float v[4][8];
+        const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
+        uint32_t buf[2][16];
+        ld_row32(row, c0 + lane * 32, c1, a32, buf[0]);
+        ld_row32(row, c0 + kStep + lane * 32, c1, a32, buf[1]);
+        float m = -INFINITY, s = 0.f;
+        int am = 0x7fffffff;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int i = (q * kRowThreads + tid) * 8;
-            if (i < n) {
-                const uint4 r4 = *reinterpret_cast<const uint4 *>(st + i);
-                v[q][0] = bf16lo(r4.x); v[q][1] = bf16hi(r4.x); v[q][2] = bf16lo(r4.y); v[q][3] = bf16hi(r4.y);
-                v[q][4] = bf16lo(r4.z); v[q][5] = bf16hi(r4.z); v[q][6] = bf16lo(r4.w); v[q][7] = bf16hi(r4.w);
-            } else {
+        for (int st = 0; st < kSteps; ++st) {
+            // The step's 32 values stay packed (two bf16 per word) and are
+            // widened where used, which keeps the lane under 80 registers.
+            uint32_t v[16];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) v[q][e] = -INFINITY;
+            for (int i = 0; i < 16; ++i) v[i] = buf[st & 1][i];
+            if (st + 2 < kSteps) ld_row32(row, c0 + (st + 2) * kStep + lane * 32, c1, a32, buf[st & 1]);
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                m4[(2 * i) & 3] = fmaxf(m4[(2 * i) & 3], bf16lo(v[i]));
+                m4[(2 * i + 1) & 3] = fmaxf(m4[(2 * i + 1) & 3], bf16hi(v[i]));
+            }
+            const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            const int base = c0 + st * kStep + lane * 32;
+            if (cexp == 0.f) {   // greedy row: the lowest index of the largest value (warp-uniform)
+                if (cm > m) {
+                    int ix = 0;
+#pragma unroll
+                    for (int i = 15; i >= 0; --i) {
+                        if (bf16hi(v[i]) == cm) ix = 2 * i + 1;
+                        if (bf16lo(v[i]) == cm) ix = 2 * i;
+                    }
+                    am = base + ix;
+                    m = cm;
+                }
+            } else if (cm > -INFINITY) {
+                const float mn = fmaxf(m, cm);
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    a4[(2 * i) & 3] += fast_exp2((bf16lo(v[i]) - mn) * cexp);
+                    a4[(2 * i + 1) & 3] += fast_exp2((bf16hi(v[i]) - mn) * cexp);
+                }
+                s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
+                m = mn;
             }
         }
-        float m = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) m = fmaxf(m, v[q][e]);
-        int am = 0x7fffffff;
-        float s = 0.f;
-        if (Tb == 0.f) {   // the item is one row: block-uniform branch
-#pragma unroll
-            for (int q = 3; q >= 0; --q)
-#pragma unroll
-                for (int e = 7; e >= 0; --e)
-                    if (v[q][e] == m) am = c0 + (q * kRowThreads + tid) * 8 + e;
-        } else if (m > -INFINITY) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) s += fast_exp2((v[q][e] - m) * cexp);
-        }
+        // Warp merge of (m, s, argmax) in lane order.
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             const float om = __shfl_xor_sync(0xffffffffu, m, o);
@@ -344,33 +358,11 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows_bulk(const __nv_bfloa
             if (om > m || (om == m && oa < am)) am = oa;
             m = nm;
         }
-        if (lane == 0) { rm[wid] = m; rs[wid] = s; ra[wid] = am; }
-        __syncthreads();   // also: every thread is done with this stage
-        if (tid == 0) {
-            float M = rm[0];
-            int A = ra[0];
-            for (int q = 1; q < 8; ++q)
-                if (rm[q] > M || (rm[q] == M && ra[q] < A)) { M = rm[q]; A = ra[q]; }
-            float S = 0.f;
-            if (cexp > 0.f)
-                for (int q = 0; q < 8; ++q)
-                    if (rm[q] > -INFINITY) S += rs[q] * fast_exp2((rm[q] - M) * cexp);
+        if (lane == 0) {
             const size_t o = (size_t)j * w.nChunks + c;
-            w.cm[o] = M;
-            w.cs[o] = S;
-            w.ca[o] = A;
-            if (k + kRowStages < my_items) {
-                tc::fence_proxy_async_smem();
-                issue(k + kRowStages);
-            }
-        }
-    }
-    // Copies still in flight after a timeout must land before the CTA exits.
-    if (tid == 0 && abort_s) {
-        int none = 0;
-        for (int k = 0; k < my_items && k < kRowStages; ++k) {
-            const int kk = my_items - 1 - k;
-            tc::mbar_wait_bounded(&full[kk % kRowStages], (kk / kRowStages) & 1, &none, 500000000LL);
+            w.cm[o] = m;
+            w.cs[o] = s;
+            w.ca[o] = am;
         }
     }
 }
@@ -743,13 +735,10 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int maxwork = a.B * (a.G + 1) * w.nChunks;
     if (a.dtype == DSPARK_BF16) {
-        const size_t smem = (size_t)kRowStages * kChunk * 2;
-        if ((e = cudaFuncSetAttribute(verify_rows_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
-            return e;
-        const int grid = max(1, min(maxwork, sms * 4));
-        verify_rows_bulk<<<grid, kRowThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp,
-                                                          a.G, a.V, w);
+        // Enough resident warps to keep ~100 KB per SM of row data in flight.
+        const int grid = max(1, min((maxwork + 7) / 8, sms * 3));
+        verify_rows_warp<<<grid, kRowsWarpThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp,
+                                                            a.G, a.V, w);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         const int grid = max(1, min(maxwork, sms * 8));

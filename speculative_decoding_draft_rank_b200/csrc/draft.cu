@@ -17,6 +17,7 @@
 //                 tile sums, recomputes that one tile's values and scans it to
 //                 the sampled token; writes x_i, p_d(x_i), max and Z.
 #include "common.cuh"
+#include "finalize.cuh"
 #include "kernels.cuh"
 
 namespace dspark {
@@ -137,162 +138,16 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
 }
 
 // ---------------------------------------------------------------------------
-// Finalize: one CTA of kFinThreads threads per request row.  Thread t owns the
-// contiguous partials [t K, t K + K) and loads them (with the previous token
-// and its U row) before any barrier, so the stage costs a few dependent
-// memory round trips: one block max, one block scan of the threads' scaled
-// partial sums, then the thread whose range holds u Z walks its partials to
-// the crossing one, whose columns the block recomputes and scans.
+// Finalize (fp32 rounds): one CTA of kFinThreads threads per request row, the
+// row work in finalize.cuh.
 constexpr int kFinThreads = 256;
-constexpr int kFinChunk = 8;   // partials per thread held in registers
 
 template <typename T>
-__global__ void __launch_bounds__(kFinThreads) draft_finalize(
-    const T *__restrict__ L, const T *__restrict__ U, const T *__restrict__ Wt,
-    const int32_t *__restrict__ x0, const float *__restrict__ temp,
-    const float *__restrict__ u_draft, int B, int G, int V, int r, int pos, int nTiles, int TN,
-    const float *__restrict__ part_m, const float *__restrict__ part_s,
-    const int32_t *__restrict__ part_a, int32_t *__restrict__ x_out, float *__restrict__ pd_out,
-    float *__restrict__ rowmax_out, float *__restrict__ rowsum_out, __nv_bfloat16 *__restrict__ E,
-    WsHeader *hdr)
-{
-    extern __shared__ float fin_smem[];
-    float *urow = fin_smem;                 // [r] U[x_{i-1}] row
-    __shared__ float s_max[32], s_loc[32], s_col[32];
-    __shared__ int s_own[32], s_own2[32], s_x[32], s_x2[32];
-    __shared__ int ts_s, xg_s;
-    __shared__ float rem_s;
-
-    const int b = blockIdx.x, tid = threadIdx.x, nthr = blockDim.x;
-    const size_t ro = (size_t)b * G + pos;
-    // bf16 rounds: the sampled token's U row is staged in E[b] for the next
-    // position's tensor-core pass (16-byte pieces; r is a multiple of 16).
-    auto stage_next = [&](int x) {
-        if (E != nullptr && pos + 1 < G)
-            for (int q = tid; q < r / 8; q += nthr)
-                reinterpret_cast<uint4 *>(E + (size_t)b * r)[q] = ld_nc16(U + (size_t)x * r + q * 8);
-    };
-    const float *pm = part_m + (size_t)b * nTiles;
-    const float *ps = part_s + (size_t)b * nTiles;
-    const int K = (nTiles + nthr - 1) / nthr;
-    const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
-
-    // Every load that depends on nothing else goes out first.
-    float cm[kFinChunk], cs[kFinChunk];
-#pragma unroll
-    for (int q = 0; q < kFinChunk; ++q) {
-        const bool in = t0 + q < t1;
-        cm[q] = in ? pm[t0 + q] : -INFINITY;
-        cs[q] = in ? ps[t0 + q] : 0.f;
-    }
-    const float Tb = sane_temp(temp[b], hdr);
-    const float u = u_draft[ro];
-    const int prev = (pos == 0) ? clamp_token(x0[b], V, hdr) : x_out[(size_t)b * G + pos - 1];
-    // The previous token's U row (r <= 512 = 2 x kFinThreads), kept in
-    // registers until after the first barrier.
-    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
-    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
-
-    float m = -INFINITY;
-#pragma unroll
-    for (int q = 0; q < kFinChunk; ++q) m = fmaxf(m, cm[q]);
-    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, pm[t]);   // very large vocabularies only
-    const float M = block_max1(m, s_max);
-
-    if (Tb == 0.f) {   // greedy row (block-uniform): lowest argmax over the partials
-        int first = 0x7fffffff;
-        for (int t = t1 - 1; t >= t0 + kFinChunk; --t)
-            if (pm[t] == M) first = t;
-#pragma unroll
-        for (int q = kFinChunk - 1; q >= 0; --q)
-            if (t0 + q < t1 && cm[q] == M) first = t0 + q;
-        first = block_min1(first, s_own);
-        if (tid == 0) {
-            if (first >= nTiles) first = 0;  // no partial matched (non-finite inputs)
-            int x = part_a[(size_t)b * nTiles + first];
-            if (x < 0 || x >= V) x = 0;
-            x_out[ro] = x;
-            pd_out[ro] = 1.f;
-            rowmax_out[ro] = M;
-            rowsum_out[ro] = 1.f;
-            xg_s = x;
-        }
-        if (E != nullptr && pos + 1 < G) {
-            __syncthreads();
-            stage_next(xg_s);
-        }
-        return;
-    }
-
-    const float cexp = kLog2e / Tb;
-    float loc = 0.f;
-#pragma unroll
-    for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
-    for (int t = t0 + kFinChunk; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
-    if (tid < r) urow[tid] = uv0;
-    if (tid + nthr < r) urow[tid + nthr] = uv1;
-    float Z;
-    const float incl = block_scan1(loc, s_loc, &Z);   // also publishes urow
-    const float target = u * Z;
-    // The first thread whose inclusive prefix passes u Z owns the crossing
-    // (the last thread with mass if rounding left u Z at the top).
-    int owner = block_min1((incl > target && loc > 0.f) ? tid : 0x7fffffff, s_own);
-    if (owner == 0x7fffffff) owner = max(0, block_max1_i(loc > 0.f ? tid : -1, s_own2));
-    if (tid == owner) {
-        float run = incl - loc, run_last = run;
-        int ts = -1, last = t1 - 1;
-#pragma unroll
-        for (int q = 0; q < kFinChunk; ++q) {
-            if (ts < 0 && t0 + q < t1) {
-                const float wt = cs[q] * fast_exp2((cm[q] - M) * cexp);
-                if (run + wt > target) {
-                    ts = t0 + q;
-                } else {
-                    if (wt > 0.f) { last = t0 + q; run_last = run; }
-                    run += wt;
-                }
-            }
-        }
-        for (int t = t0 + kFinChunk; t < t1 && ts < 0; ++t) {
-            const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
-            if (run + wt > target) {
-                ts = t;
-            } else {
-                if (wt > 0.f) { last = t; run_last = run; }
-                run += wt;
-            }
-        }
-        if (ts < 0) { ts = last; run = run_last; }
-        ts_s = max(ts, 0);
-        rem_s = target - run;
-    }
-    __syncthreads();
-    const int ts = ts_s;
-    const float rem = rem_s;
-    // Recompute the chosen partial's columns: tpc consecutive threads share one column.
-    const int c0 = ts * TN;
-    const int tpc = nthr / TN;
-    const int col = c0 + tid / tpc, part = tid % tpc;
-    const bool mine = part == 0 && col < V;
-    const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
-    float dl = 0.f;
-    if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
-    for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
-    const float e = mine ? fast_exp2(((lval - M) + dl) * cexp) : 0.f;
-    float ttot;
-    const float inc = block_scan1(e, s_col, &ttot);
-    int xs = block_min1((mine && inc > rem) ? col : 0x7fffffff, s_x);
-    if (xs == 0x7fffffff) {  // the recomputed mass fell short: last positive column
-        xs = block_max1_i((mine && e > 0.f) ? col : -1, s_x2);
-        if (xs < 0) xs = min(c0 + TN, V) - 1;
-    }
-    if (mine && col == xs) {
-        x_out[ro] = xs;
-        pd_out[ro] = e / Z;
-        rowmax_out[ro] = M;
-        rowsum_out[ro] = Z;
-    }
-    stage_next(xs);
+__global__ void __launch_bounds__(kFinThreads) draft_finalize(const FinArgs a, int pos) {
+    __shared__ FinScratch sc;
+    __shared__ float urow[512];
+    const Grp g{(int)threadIdx.x, (int)blockDim.x, (int)(threadIdx.x >> 5), (int)(blockDim.x >> 5), 0};
+    finalize_row<T>(g, &sc, urow, a, blockIdx.x, pos);
 }
 
 // ---------------------------------------------------------------------------
@@ -326,39 +181,29 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     return w;
 }
 
-template <typename T>
-static cudaError_t launch_finalize(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
-    size_t smem = sizeof(float) * (size_t)a.r;
-    auto kern = draft_finalize<T>;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    kern<<<a.B, kFinThreads, smem, st>>>(static_cast<const T *>(a.L), static_cast<const T *>(a.U),
-                                         static_cast<const T *>(a.Wt), a.x0, a.temp, a.u_draft, a.B, a.G, a.V,
-                                         a.r, pos, w.nTiles, draft_tile_cols(a.dtype), w.part_m, w.part_s,
-                                         w.part_a, a.x_out, a.pd_out, a.rowmax_out, a.rowsum_out,
-                                         reinterpret_cast<__nv_bfloat16 *>(w.E), w.hdr);
-    return cudaGetLastError();
+FinArgs fin_args(const DraftArgs &a, const DraftWs &w) {
+    FinArgs f{};
+    f.L = a.L; f.U = a.U; f.Wt = a.Wt; f.x0 = a.x0; f.temp = a.temp; f.u_draft = a.u_draft;
+    f.B = a.B; f.G = a.G; f.V = a.V; f.r = a.r; f.nTiles = w.nTiles; f.TN = draft_tile_cols(a.dtype);
+    f.part_m = w.part_m; f.part_s = w.part_s; f.part_a = w.part_a;
+    f.x_out = a.x_out; f.pd_out = a.pd_out; f.rowmax_out = a.rowmax_out; f.rowsum_out = a.rowsum_out;
+    f.E = w.E; f.hdr = w.hdr;
+    return f;
 }
 
 cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
     DraftWs w = carve_draft_ws(ws, a.B, a.V, a.r, a.dtype);
+    const FinArgs f = fin_args(a, w);
+    if (a.dtype == DSPARK_BF16) return launch_draft_tc(a, w, f, st);
     cudaError_t e;
     for (int pos = 0; pos < a.G; ++pos) {
-        if (a.dtype == DSPARK_F32) {
-            dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
-            draft_tile_simt<float><<<grid, 256, 0, st>>>(
-                static_cast<const float *>(a.L), static_cast<const float *>(a.U),
-                static_cast<const float *>(a.Wt), a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos,
-                w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            if ((e = launch_finalize<float>(a, w, pos, st)) != cudaSuccess) return e;
-        } else {
-            // bf16: tensor-core tile kernel (its A rows are U[previous token]).
-            if ((e = launch_draft_tile_tc(a, w, pos, st)) != cudaSuccess) return e;
-            if ((e = launch_finalize<__nv_bfloat16>(a, w, pos, st)) != cudaSuccess) return e;
-        }
+        dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
+        draft_tile_simt<float><<<grid, 256, 0, st>>>(
+            static_cast<const float *>(a.L), static_cast<const float *>(a.U), static_cast<const float *>(a.Wt),
+            a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos, w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        draft_finalize<float><<<a.B, kFinThreads, 0, st>>>(f, pos);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

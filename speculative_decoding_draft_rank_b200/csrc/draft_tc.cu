@@ -15,24 +15,31 @@
 //   warp 0      TMA producer of the B operand: the transition-factor tile
 //               Wt[n0:n0+256, :] one 64-deep k-block at a time through a ring
 //               (128-byte swizzle, evict-last: W is reused by every position
-//               and M-block).
+//               and M-block and stays in L2).
 //   warp 1      TMEM owner and MMA issuer: 128 x 256 x 16 bf16 MMAs, A and B
 //               from shared memory, into one of two 256-column fp32
 //               accumulators.
 //   warp 2      TMA producer of the logits L[:, i, :] in 128 x 64 segments
 //               (128-byte swizzle, evict-first; drafting only).
-//   warps 3-18  epilogue: first they write the A operand -- the 128 rows
-//               U[previous token] -- into shared memory in the swizzled
-//               K-major layout; then warp e owns TMEM lane quarter (warp % 4)
-//               and the 64-column segment (e / 4) of every tile: Delta from
-//               TMEM plus the logits from the segment give the 64-column
-//               partials (max, lowest argmax, sum of exp((y - max) / T)).
-// Delta never leaves the SM.  Every mbarrier wait is bounded by a clock
-// budget; on expiry the CTA raises a timeout bit in the status word, drains
-// its own copies and MMAs, frees TMEM and returns.
+//   warps 3-18  epilogue: warp e owns TMEM lane quarter (warp % 4) and the
+//               64-column segment (e / 4) of every tile: Delta from TMEM plus
+//               the logits give the 64-column partials (max, lowest argmax,
+//               sum of exp((y - max) / T)).
+// Drafting runs every position of the round in one cooperative launch: after
+// a position's tiles the CTAs meet at a grid barrier, the epilogue warps
+// finalize two rows per CTA (256 threads per row: the token draw, its
+// probability, and the token's U row staged for the next position), meet
+// again, and one thread loads the staged rows as the next position's A
+// operand with TMA.  The producers run straight across position boundaries.
+// At the first position (and for the residual rows) the epilogue warps gather
+// the A rows U[previous token] into shared memory themselves.
+// Delta never leaves the SM.  Every mbarrier and grid-barrier wait is bounded
+// by a clock budget; on expiry the CTA raises a timeout bit in the status
+// word, drains its own copies and MMAs, frees TMEM and returns.
 #include <algorithm>
 
 #include "common.cuh"
+#include "finalize.cuh"
 #include "kernels.cuh"
 #include "tc.cuh"
 
@@ -82,9 +89,10 @@ enum { kEpiDraft = 0, kEpiResidual = 1 };
 
 struct TcEpi {
     const float *temp;
-    int B, G, V, pos, nParts;
-    int a_tma;                // 1: the A rows come from the staged E by TMA (drafting, positions >= 2)
+    int B, G, V, nParts;
     WsHeader *hdr;
+    FinArgs fin;              // drafting: the per-row finalize of every position
+    uint32_t *grid_count;     // drafting: grid-barrier counter (zeroed before the launch)
     const __nv_bfloat16 *U;   // [V, r]: A-operand rows are U[previous token]
     const int32_t *x0;        // [B] last committed tokens
     const int32_t *x;         // [B, G] draft tokens (drafting: earlier positions of this call)
@@ -116,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     unsigned char *sL = base + lay.l_off;
     const int SB = lay.sB, SL = lay.sL, nkb = lay.nkb;
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + lay.bar_off);
-    uint64_t *a_full = bars;                 // A is in shared memory (16 epilogue-warp arrivals, or the TMA bytes)
+    uint64_t *a_full = bars;                 // A is in shared memory (one phase per position)
     uint64_t *b_full = a_full + 1;           // SB
     uint64_t *b_empty = b_full + SB;         // SB
     uint64_t *l_full = b_empty + SB;         // SL
@@ -127,8 +135,10 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
+    __shared__ int epi_flag;                 // epilogue-wide verdict of the last grid barrier
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = ep.B, V = ep.V, nParts = ep.nParts;
+    const int npos = (MODE == kEpiDraft) ? ep.G : 1;
     WsHeader *hdr = ep.hdr;
     const int nMB = (B + kM - 1) / kM;
     const int mb = blockIdx.x % nMB;
@@ -140,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     if (m0 >= nrows) return;
 
     if (threadIdx.x == 0) {
-        tc::mbar_init(a_full, ep.a_tma ? 1 : kEpiWarps);
+        tc::mbar_init(a_full, 1);
         for (int q = 0; q < SB; ++q) { tc::mbar_init(&b_full[q], 1); tc::mbar_init(&b_empty[q], 1); }
         for (int q = 0; q < SL; ++q) { tc::mbar_init(&l_full[q], 1); tc::mbar_init(&l_empty[q], 4); }
         for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], kEpiWarps); }
@@ -162,14 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         if (lane == 0) {
             tc::prefetch_tmap(&mapW);
             const uint64_t keep = tc::policy_evict_last();
-            if (ep.a_tma) {   // the staged A rows first: the MMA waits for them
-                const uint64_t once = tc::policy_evict_first();
-                tc::mbar_arrive_expect_tx(a_full, (uint32_t)nkb * kABlockBytes);
-                for (int kb = 0; kb < nkb; ++kb)
-                    tc::tma_load_2d(sA + kb * kABlockBytes, &mapE, a_full, kb * kKB, m0, once);
-            }
             int g = 0;
             bool ok = true;
+            for (int pos = 0; pos < npos && ok; ++pos)
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 const int n0 = t * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -191,7 +196,6 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const int gg = g - 1 - q;
                     tc::mbar_wait_bounded(&b_full[gg % SB], (gg / SB) & 1, no_abort, kWaitBudget / 4);
                 }
-                if (ep.a_tma) tc::mbar_wait_bounded(a_full, 0, no_abort, kWaitBudget / 4);
                 flag_status(hdr, DSPARK_DEV_TIMEOUT);
             }
         }
@@ -200,9 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         if (lane == 0) {
             const uint32_t idesc = tc::idesc_bf16_f32(kM, kBN);
             const uint32_t a_addr = tc::smem_u32(sA), b_addr = tc::smem_u32(sB);
-            bool ok = tc::mbar_wait_bounded(a_full, 0, abort_flag, kWaitBudget);
-            tc::tc_fence_after();
+            bool ok = true;
             int g = 0, j = 0;
+            for (int pos = 0; pos < npos && ok; ++pos) {
+            ok = tc::mbar_wait_bounded(a_full, pos & 1, abort_flag, kWaitBudget);
+            tc::tc_fence_after();
             for (int t = first_tile; t < nTilesN && ok; t += tile_step, ++j) {
                 const int ab = j & 1;
                 if (!tc::mbar_wait_bounded(&acc_empty[ab], ((j >> 1) & 1) ^ 1, abort_flag, kWaitBudget)) {
@@ -229,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 if (!ok) break;
                 tc::mma_commit(&acc_full[ab]);
             }
+            }
             // Drain: every MMA issued above has completed once this arrives.
             tc::mma_commit(drain);
             int dummy = 0;
@@ -242,6 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             const uint64_t stream = tc::policy_evict_first();
             int g = 0;
             bool ok = true;
+            for (int pos = 0; pos < npos && ok; ++pos)
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 for (int sg = 0; sg < kSegs; ++sg, ++g) {
                     const int q = g % SL;
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                         break;
                     }
                     tc::mbar_arrive_expect_tx(&l_full[q], kSegBytes);
-                    tc::tma_load_3d(sL + q * kSegBytes, &mapL, &l_full[q], t * kBN + sg * kSeg, ep.pos, m0, stream);
+                    tc::tma_load_3d(sL + q * kSegBytes, &mapL, &l_full[q], t * kBN + sg * kSeg, pos, m0, stream);
                 }
             }
             if (!ok) {
@@ -269,30 +277,15 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         const int sg = ew >> 2;                // 64-column segment of every tile (0..3)
         const int row = quarter * 32 + lane;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        // ---------------------------------------------- A operand into smem
-        // Row m0 + row is U[previous token] of that row (the previous draft
-        // token, x0 at the first position, or for a queued rejection the token
-        // before it).  This warp writes k-blocks kb = sg, sg + 4, ... of its
-        // 32 rows in the 128-byte-swizzled K-major layout (zeros past r).
-        if (!ep.a_tma) {
-            int prev = 0;
-            if (MODE == kEpiDraft) {
-                const int b = m0 + row;
-                if (b < B) {
-                    prev = (ep.pos == 0) ? ep.x0[b] : ep.x[(size_t)b * ep.G + ep.pos - 1];
-                    if (prev < 0 || prev >= V) {
-                        if (ep.pos == 0) flag_status(hdr, DSPARK_DEV_TOKEN_RANGE);
-                        prev = prev < 0 ? 0 : V - 1;
-                    }
-                }
-            } else {
-                const int sidx = m0 + row;
-                if (sidx < nrows) {
-                    const int b = ep.res_b[sidx], k = ep.res_k[sidx];
-                    prev = (k == 0) ? ep.x0[b] : ep.x[(size_t)b * ep.G + k - 1];
-                    prev = min(max(prev, 0), V - 1);
-                }
-            }
+        const bool leader = ew == 0 && lane == 0;
+        // Named barrier 1: the 16 epilogue warps only.
+        auto epi_sync = [&]() { asm volatile("bar.sync 1, %0;" ::"r"(kEpiWarps * 32) : "memory"); };
+        // A operand into shared memory: row `row` is U[prev] -- x0 at the
+        // first position, or for a queued rejection the token before it.
+        // This warp writes k-blocks kb = sg, sg + 4, ... of its 32 rows in the
+        // 128-byte-swizzled K-major layout (zeros past r); then one thread
+        // completes the A phase for the MMA warp.
+        auto gather_A = [&](int prev) {
             const __nv_bfloat16 *urow = ep.U + (size_t)prev * r;
             for (int kb = sg; kb < nkb; kb += kSegs) {
                 uint4 v[8];
@@ -306,9 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(dst + ((c ^ (row & 7)) << 4)) = v[c];
             }
             tc::fence_proxy_async_smem();   // generic writes -> tensor-core reads
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(a_full);
-        }
+            epi_sync();
+            if (leader) tc::mbar_arrive(a_full);
+        };
         if (MODE == kEpiDraft) {
             // ------------------------------------------ drafting epilogue
             // One online pass per 32-column chunk: y = L + Delta, chunk max,
@@ -325,87 +318,157 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             const float cexp = invT * kLog2e;      // exp((y - m) / T) = 2^((y - m) * cexp)
             const bool warp_greedy = __any_sync(0xffffffffu, rowok && invT == 0.f);
             const bool warp_soft = __any_sync(0xffffffffu, rowok && invT > 0.f);
-            int j = 0;
-            for (int t = first_tile; t < nTilesN; t += tile_step, ++j) {
-                const int ab = j & 1;
-                const int gl = j * kSegs + sg, q = gl % SL;
-                // Every lane waits; the vote keeps the warp converged for the
-                // warp-collective TMEM loads below even if the budget runs out.
-                bool ok = tc::mbar_wait_bounded(&l_full[q], (gl / SL) & 1, abort_flag, kWaitBudget);
-                ok = ok && tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
-                if (!__all_sync(0xffffffffu, ok)) break;
-                tc::tc_fence_after();
-                // This thread's 64 logits: one 128-byte row of the swizzled segment.
-                const unsigned char *lsrc = sL + q * kSegBytes + row * 128;
-                uint4 cur[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    cur[u] = *reinterpret_cast<const uint4 *>(lsrc + ((u ^ (row & 7)) << 4));
-                // The segment is in registers: hand the slot back to the
-                // producer now, so the next tile's copy overlaps this one's math.
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&l_empty[q]);
-                const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
-                const int cbase = t * kBN + sg * kSeg;
-                const bool whole = cbase + kSeg <= V;   // no column of this segment lies past V
-                float m = -INFINITY, s = 0.f;
-                int am = 0x7fffffff;
-#pragma unroll
-                for (int c = 0; c < kSeg / 32; ++c) {
-                    float y[32];
-                    tc::tmem_ld32(taddr + c * 32, y);
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const uint4 qv = cur[c * 4 + u];
-                        y[u * 8 + 0] += bf16lo(qv.x); y[u * 8 + 1] += bf16hi(qv.x);
-                        y[u * 8 + 2] += bf16lo(qv.y); y[u * 8 + 3] += bf16hi(qv.y);
-                        y[u * 8 + 4] += bf16lo(qv.z); y[u * 8 + 5] += bf16hi(qv.z);
-                        y[u * 8 + 6] += bf16lo(qv.w); y[u * 8 + 7] += bf16hi(qv.w);
+            // All CTAs' epilogue warps meet; false (uniform across the
+            // epilogue) when any role of this CTA aborted or the wait ran out.
+            auto grid_sync = [&](uint32_t target) -> bool {
+                epi_sync();
+                if (leader) {
+                    bool ok = *abort_flag == 0;
+                    if (ok) {
+                        __threadfence();
+                        atomicAdd(ep.grid_count, 1u);
+                        const long long t0 = clock64();
+                        while (tc::ld_acquire_gpu(ep.grid_count) < target) {
+                            if (*abort_flag || clock64() - t0 > kWaitBudget) { ok = false; break; }
+                            __nanosleep(32);
+                        }
                     }
-                    if (!whole) {
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (cbase + c * 32 + e >= V) y[e] = -INFINITY;
+                    if (!ok) {
+                        *abort_flag = 1;
+                        flag_status(hdr, DSPARK_DEV_TIMEOUT);
                     }
-                    // Tree max (short dependency chains).
-                    float t16[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) t16[e] = fmaxf(y[e], y[e + 16]);
-#pragma unroll
-                    for (int wdt = 8; wdt > 0; wdt >>= 1)
-#pragma unroll
-                        for (int e = 0; e < wdt; ++e) t16[e] = fmaxf(t16[e], t16[e + wdt]);
-                    const float cm = t16[0];
-                    if (warp_greedy && cm > m) {
-                        int ix = 0x7fffffff;
-#pragma unroll
-                        for (int e = 31; e >= 0; --e)
-                            if (y[e] == cm) ix = e;
-                        am = cbase + c * 32 + ix;
-                    }
-                    const float mn = fmaxf(m, cm);
-                    if (warp_soft) {
-                        float a4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sums
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2((y[e] - mn) * cexp);
-                        const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
-                        s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + acc;
-                    }
-                    m = mn;
+                    epi_flag = ok ? 0 : 1;
                 }
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
-                const int p = t * kSegs + sg;
-                if (rowok && p < nParts) {
-                    const size_t o = (size_t)b * nParts + p;
-                    ep.part_m[o] = m;
-                    ep.part_s[o] = s;
-                    ep.part_a[o] = am;
+                epi_sync();
+                return epi_flag == 0;
+            };
+            // Finalize: epilogue warps 0-7 and 8-15 are two 256-thread groups
+            // (named barriers 2 and 3), each with scratch in the A region,
+            // which no MMA reads between a position's last tile and the next
+            // position's A load.
+            const int grp = ew >> 3;
+            const Grp fg{(ew & 7) * 32 + lane, 256, ew & 7, 8, 2 + grp};
+            FinScratch *fsc = reinterpret_cast<FinScratch *>(sA + grp * 4096);
+            float *furow = reinterpret_cast<float *>(sA + 8192 + grp * 2048);
+            const uint32_t nblk = gridDim.x;
+            int j = 0;
+            for (int pos = 0; pos < ep.G; ++pos) {
+                if (pos == 0) {
+                    int prev = 0;
+                    if (rowok) {
+                        prev = ep.x0[b];
+                        if (prev < 0 || prev >= V) {
+                            flag_status(hdr, DSPARK_DEV_TOKEN_RANGE);
+                            prev = prev < 0 ? 0 : V - 1;
+                        }
+                    }
+                    gather_A(prev);
+                }
+                for (int t = first_tile; t < nTilesN; t += tile_step, ++j) {
+                    const int ab = j & 1;
+                    const int gl = j * kSegs + sg, q = gl % SL;
+                    // Every lane waits; the vote keeps the warp converged for the
+                    // warp-collective TMEM loads below even if the budget runs out.
+                    bool ok = tc::mbar_wait_bounded(&l_full[q], (gl / SL) & 1, abort_flag, kWaitBudget);
+                    ok = ok && tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
+                    if (!__all_sync(0xffffffffu, ok)) break;
+                    tc::tc_fence_after();
+                    // This thread's 64 logits: one 128-byte row of the swizzled segment.
+                    const unsigned char *lsrc = sL + q * kSegBytes + row * 128;
+                    uint4 cur[8];
+    #pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        cur[u] = *reinterpret_cast<const uint4 *>(lsrc + ((u ^ (row & 7)) << 4));
+                    // The segment is in registers: hand the slot back to the
+                    // producer now, so the next tile's copy overlaps this one's math.
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&l_empty[q]);
+                    const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
+                    const int cbase = t * kBN + sg * kSeg;
+                    const bool whole = cbase + kSeg <= V;   // no column of this segment lies past V
+                    float m = -INFINITY, s = 0.f;
+                    int am = 0x7fffffff;
+    #pragma unroll
+                    for (int c = 0; c < kSeg / 32; ++c) {
+                        float y[32];
+                        tc::tmem_ld32(taddr + c * 32, y);
+    #pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint4 qv = cur[c * 4 + u];
+                            y[u * 8 + 0] += bf16lo(qv.x); y[u * 8 + 1] += bf16hi(qv.x);
+                            y[u * 8 + 2] += bf16lo(qv.y); y[u * 8 + 3] += bf16hi(qv.y);
+                            y[u * 8 + 4] += bf16lo(qv.z); y[u * 8 + 5] += bf16hi(qv.z);
+                            y[u * 8 + 6] += bf16lo(qv.w); y[u * 8 + 7] += bf16hi(qv.w);
+                        }
+                        if (!whole) {
+    #pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (cbase + c * 32 + e >= V) y[e] = -INFINITY;
+                        }
+                        // Tree max (short dependency chains).
+                        float t16[16];
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e) t16[e] = fmaxf(y[e], y[e + 16]);
+    #pragma unroll
+                        for (int wdt = 8; wdt > 0; wdt >>= 1)
+    #pragma unroll
+                            for (int e = 0; e < wdt; ++e) t16[e] = fmaxf(t16[e], t16[e + wdt]);
+                        const float cm = t16[0];
+                        if (warp_greedy && cm > m) {
+                            int ix = 0x7fffffff;
+    #pragma unroll
+                            for (int e = 31; e >= 0; --e)
+                                if (y[e] == cm) ix = e;
+                            am = cbase + c * 32 + ix;
+                        }
+                        const float mn = fmaxf(m, cm);
+                        if (warp_soft) {
+                            float a4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sums
+    #pragma unroll
+                            for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2((y[e] - mn) * cexp);
+                            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                            s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + acc;
+                        }
+                        m = mn;
+                    }
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&acc_empty[ab]);
+                    const int p = t * kSegs + sg;
+                    if (rowok && p < nParts) {
+                        const size_t o = (size_t)b * nParts + p;
+                        ep.part_m[o] = m;
+                        ep.part_s[o] = s;
+                        ep.part_a[o] = am;
+                    }
+                }
+                // Every CTA's partials of this position are written.
+                if (!grid_sync(nblk * (2u * pos + 1u))) break;
+                for (int bb = (int)blockIdx.x * 2 + grp; bb < B; bb += 2 * (int)nblk)
+                    finalize_row<__nv_bfloat16>(fg, fsc, furow, ep.fin, bb, pos);
+                tc::fence_proxy_async_all();   // E rows and the scratch, before async-proxy use
+                // Every row's token (and staged U row) of this position is written.
+                if (!grid_sync(nblk * (2u * pos + 2u))) break;
+                if (pos + 1 < ep.G && leader) {
+                    tc::fence_proxy_async_all();
+                    tc::mbar_arrive_expect_tx(a_full, (uint32_t)nkb * kABlockBytes);
+                    const uint64_t once = tc::policy_evict_first();
+                    for (int kb = 0; kb < nkb; ++kb)
+                        tc::tma_load_2d(sA + kb * kABlockBytes, &mapE, a_full, kb * kKB, m0, once);
                 }
             }
         } else {
+            {
+                int prev = 0;
+                const int sidx = m0 + row;
+                if (sidx < nrows) {
+                    const int bq = ep.res_b[sidx], k = ep.res_k[sidx];
+                    prev = (k == 0) ? ep.x0[bq] : ep.x[(size_t)bq * ep.G + k - 1];
+                    prev = min(max(prev, 0), V - 1);
+                }
+                gather_A(prev);
+            }
             // ------------------------------------------ residual epilogue
             const int sidx = m0 + row;
             const bool rowok = sidx < nrows;
@@ -544,7 +607,7 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, const void 
     CUtensorMap mW, mL, mE;
     if (!map_factor(&mW, Wt, ep.V, r)) return cudaErrorInvalidValue;
     if (!map_logits(&mL, ep.L, ep.B, ep.G, ep.V)) return cudaErrorInvalidValue;
-    if (ep.a_tma) {
+    if (MODE == kEpiDraft && ep.G > 1) {
         if (!map_stage(&mE, E, ep.B, r)) return cudaErrorInvalidValue;
     } else {
         mE = mW;   // unused
@@ -560,29 +623,50 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, const void 
     const int nMB = (ep.B + kM - 1) / kM;
     int grid = std::min(sms, nMB * nTilesN);
     grid = std::max(grid, nMB);
-    markov_tile_tc<MODE><<<grid, kThreads, lay.total, st>>>(mW, mL, mE, r, nTilesN, ep);
-    return cudaGetLastError();
+    if (MODE == kEpiResidual) {
+        markov_tile_tc<MODE><<<grid, kThreads, lay.total, st>>>(mW, mL, mE, r, nTilesN, ep);
+        return cudaGetLastError();
+    }
+    // Drafting: every CTA must be resident for the grid barriers, which a
+    // cooperative launch guarantees (or refuses).
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, markov_tile_tc<MODE>, kThreads, lay.total)) !=
+        cudaSuccess)
+        return e;
+    if (per_sm < 1 || grid > per_sm * sms) return cudaErrorCooperativeLaunchTooLarge;
+    if ((e = cudaMemsetAsync(ep.grid_count, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = lay.total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, markov_tile_tc<MODE>, mW, mL, mE, r, nTilesN, ep);
 }
 
 }  // namespace
 
-cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st) {
+cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs &f, cudaStream_t st) {
     TcEpi ep{};
-    ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.pos = pos; ep.nParts = w.nTiles; ep.hdr = w.hdr;
+    ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.nParts = w.nTiles; ep.hdr = w.hdr;
     ep.U = static_cast<const __nv_bfloat16 *>(a.U); ep.x0 = a.x0; ep.x = a.x_out;
     ep.L = static_cast<const __nv_bfloat16 *>(a.L);
     ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
-    ep.a_tma = (pos > 0 && w.E != nullptr) ? 1 : 0;   // position 0 gathers U[x0] itself
+    ep.fin = f;
+    ep.grid_count = &w.hdr->pad[2];
     return launch_markov_tc<kEpiDraft>(a.Wt, a.r, ep, w.E, st);
 }
 
 cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st) {
     TcEpi ep{};
-    ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.pos = 0; ep.nParts = a.nParts; ep.hdr = a.hdr;
+    ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.nParts = a.nParts; ep.hdr = a.hdr;
     ep.U = a.U; ep.x0 = a.x0; ep.x = a.x; ep.L = a.L;
     ep.nrows = a.nrows; ep.res_b = a.res_b; ep.res_k = a.res_k; ep.res_mt = a.res_mt; ep.res_zt = a.res_zt;
     ep.rowmax = a.rowmax; ep.rowsum = a.rowsum; ep.Tlog = a.Tlog; ep.rp = a.rp;
-    ep.a_tma = 0;
     return launch_markov_tc<kEpiResidual>(a.Wt, a.r, ep, nullptr, st);
 }
 

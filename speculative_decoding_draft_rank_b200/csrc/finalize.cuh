@@ -1,0 +1,228 @@
+// finalize.cuh -- the per-row end of one drafting position, shared by the
+// standalone finalize kernel (fp32 rounds) and the persistent tensor-core
+// drafting kernel (bf16 rounds).
+//
+// Method (paperlayer.ai summary of DSpark, §3.1 Semi-autoregressive
+// generation: each position's token is drawn from the temperature softmax of
+// L[i] + Delta_i; the draw here is the inverse CDF at the round's uniform u):
+// the tile partials (max, sum of exp((y - max) / T), lowest argmax) of a row
+// are combined into the row's max M and normaliser Z; the partial where the
+// running mass passes u Z is found by a prefix over the partials, its columns
+// are recomputed (Delta from U[x_{i-1}] and W) and scanned to the token.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+// A group of whole warps working on one row: its thread index, size, warp
+// index and warp count, and the named barrier it synchronises on (0 with the
+// whole CTA as the group means __syncthreads).
+struct Grp {
+    int tid, n, wid, nw, bar;
+    __device__ __forceinline__ void sync() const {
+        if (bar == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(n) : "memory");
+    }
+};
+
+// One-barrier group reductions (every warp publishes into its own entry of
+// `slots`; each call site owns its slots, so no trailing barrier is needed).
+__device__ __forceinline__ float grp_max1(const Grp &g, float v, float *slots) {
+    v = warp_max(v);
+    if ((threadIdx.x & 31) == 0) slots[g.wid] = v;
+    g.sync();
+    float r = slots[0];
+    for (int w = 1; w < g.nw; ++w) r = fmaxf(r, slots[w]);
+    return r;
+}
+__device__ __forceinline__ int grp_min1(const Grp &g, int v, int *slots) {
+    v = warp_min_i(v);
+    if ((threadIdx.x & 31) == 0) slots[g.wid] = v;
+    g.sync();
+    int r = slots[0];
+    for (int w = 1; w < g.nw; ++w) r = min(r, slots[w]);
+    return r;
+}
+__device__ __forceinline__ int grp_max1_i(const Grp &g, int v, int *slots) { return -grp_min1(g, -v, slots); }
+__device__ __forceinline__ float grp_scan1(const Grp &g, float v, float *slots, float *total) {
+    const float s = warp_incl_scan(v);
+    if ((threadIdx.x & 31) == 31) slots[g.wid] = s;
+    g.sync();
+    float before = 0.f, tot = 0.f;
+    for (int w = 0; w < g.nw; ++w) {
+        if (w == g.wid) before = tot;
+        tot += slots[w];
+    }
+    *total = tot;
+    return before + s;
+}
+
+// Shared-memory scratch of one group (at most 8 warps).
+struct FinScratch {
+    float s_max[8], s_loc[8], s_col[8];
+    int s_own[8], s_own2[8], s_x[8], s_x2[8];
+    int ts, xg;
+    float rem;
+};
+
+constexpr int kFinChunk = 8;   // partials per thread held in registers
+
+struct FinArgs {
+    const void *L, *U, *Wt;
+    const int32_t *x0;
+    const float *temp, *u_draft;
+    int B, G, V, r, nTiles, TN;   // TN: columns per partial
+    const float *part_m, *part_s;
+    const int32_t *part_a;
+    int32_t *x_out;
+    float *pd_out, *rowmax_out, *rowsum_out;
+    __nv_bfloat16 *E;              // bf16 rounds: U[x_i] rows staged for position i + 1, else null
+    WsHeader *hdr;
+};
+
+// Row b at position pos.  Thread t of the group owns the contiguous partials
+// [t K, t K + K) and loads them (with the previous token and its U row) before
+// any barrier: one group max, one group scan of the threads' scaled partial
+// sums, then the thread whose range holds u Z walks its partials to the
+// crossing one, whose TN columns the group recomputes and scans.  urow holds
+// r floats.  Ends with a group barrier, so the scratch may be reused.
+template <typename T>
+__device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const FinArgs &a, int b, int pos) {
+    const T *L = static_cast<const T *>(a.L);
+    const T *U = static_cast<const T *>(a.U);
+    const T *Wt = static_cast<const T *>(a.Wt);
+    const int G = a.G, V = a.V, r = a.r, nTiles = a.nTiles, TN = a.TN;
+    const int tid = g.tid, nthr = g.n;
+    const size_t ro = (size_t)b * G + pos;
+    // bf16 rounds: the sampled token's U row is staged in E[b] for the next
+    // position's tensor-core pass (16-byte pieces; r is a multiple of 16).
+    auto stage_next = [&](int x) {
+        if (a.E != nullptr && pos + 1 < G)
+            for (int q = tid; q < r / 8; q += nthr)
+                reinterpret_cast<uint4 *>(a.E + (size_t)b * r)[q] = ld_nc16(U + (size_t)x * r + q * 8);
+    };
+    const float *pm = a.part_m + (size_t)b * nTiles;
+    const float *ps = a.part_s + (size_t)b * nTiles;
+    const int K = (nTiles + nthr - 1) / nthr;
+    const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
+
+    // Every load that depends on nothing else goes out first.
+    float cm[kFinChunk], cs[kFinChunk];
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) {
+        const bool in = t0 + q < t1;
+        cm[q] = in ? pm[t0 + q] : -INFINITY;
+        cs[q] = in ? ps[t0 + q] : 0.f;
+    }
+    const float Tb = sane_temp(a.temp[b], a.hdr);
+    const float u = a.u_draft[ro];
+    const int prev = (pos == 0) ? clamp_token(a.x0[b], V, a.hdr) : a.x_out[(size_t)b * G + pos - 1];
+    // The previous token's U row (r <= 512 = 2 x 256 threads), kept in
+    // registers until after the first barrier.
+    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
+    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+
+    float m = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) m = fmaxf(m, cm[q]);
+    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, pm[t]);   // very large vocabularies only
+    const float M = grp_max1(g, m, sc->s_max);
+
+    if (Tb == 0.f) {   // greedy row (group-uniform): lowest argmax over the partials
+        int first = 0x7fffffff;
+        for (int t = t1 - 1; t >= t0 + kFinChunk; --t)
+            if (pm[t] == M) first = t;
+#pragma unroll
+        for (int q = kFinChunk - 1; q >= 0; --q)
+            if (t0 + q < t1 && cm[q] == M) first = t0 + q;
+        first = grp_min1(g, first, sc->s_own);
+        if (tid == 0) {
+            if (first >= nTiles) first = 0;  // no partial matched (non-finite inputs)
+            int x = a.part_a[(size_t)b * nTiles + first];
+            if (x < 0 || x >= V) x = 0;
+            a.x_out[ro] = x;
+            a.pd_out[ro] = 1.f;
+            a.rowmax_out[ro] = M;
+            a.rowsum_out[ro] = 1.f;
+            sc->xg = x;
+        }
+        g.sync();
+        stage_next(sc->xg);
+        g.sync();
+        return;
+    }
+
+    const float cexp = kLog2e / Tb;
+    float loc = 0.f;
+#pragma unroll
+    for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
+    for (int t = t0 + kFinChunk; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
+    if (tid < r) urow[tid] = uv0;
+    if (tid + nthr < r) urow[tid + nthr] = uv1;
+    float Z;
+    const float incl = grp_scan1(g, loc, sc->s_loc, &Z);   // also publishes urow
+    const float target = u * Z;
+    // The first thread whose inclusive prefix passes u Z owns the crossing
+    // (the last thread with mass if rounding left u Z at the top).
+    int owner = grp_min1(g, (incl > target && loc > 0.f) ? tid : 0x7fffffff, sc->s_own);
+    if (owner == 0x7fffffff) owner = max(0, grp_max1_i(g, loc > 0.f ? tid : -1, sc->s_own2));
+    if (tid == owner) {
+        float run = incl - loc, run_last = run;
+        int ts = -1, last = t1 - 1;
+#pragma unroll
+        for (int q = 0; q < kFinChunk; ++q) {
+            if (ts < 0 && t0 + q < t1) {
+                const float wt = cs[q] * fast_exp2((cm[q] - M) * cexp);
+                if (run + wt > target) {
+                    ts = t0 + q;
+                } else {
+                    if (wt > 0.f) { last = t0 + q; run_last = run; }
+                    run += wt;
+                }
+            }
+        }
+        for (int t = t0 + kFinChunk; t < t1 && ts < 0; ++t) {
+            const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
+            if (run + wt > target) {
+                ts = t;
+            } else {
+                if (wt > 0.f) { last = t; run_last = run; }
+                run += wt;
+            }
+        }
+        if (ts < 0) { ts = last; run = run_last; }
+        sc->ts = max(ts, 0);
+        sc->rem = target - run;
+    }
+    g.sync();
+    const int ts = sc->ts;
+    const float rem = sc->rem;
+    // Recompute the chosen partial's columns: tpc consecutive threads share one column.
+    const int c0 = ts * TN;
+    const int tpc = nthr / TN;
+    const int col = c0 + tid / tpc, part = tid % tpc;
+    const bool mine = part == 0 && col < V;
+    const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
+    float dl = 0.f;
+    if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
+    for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);
+    const float e = mine ? fast_exp2(((lval - M) + dl) * cexp) : 0.f;
+    float ttot;
+    const float inc = grp_scan1(g, e, sc->s_col, &ttot);
+    int xs = grp_min1(g, (mine && inc > rem) ? col : 0x7fffffff, sc->s_x);
+    if (xs == 0x7fffffff) {  // the recomputed mass fell short: last positive column
+        xs = grp_max1_i(g, (mine && e > 0.f) ? col : -1, sc->s_x2);
+        if (xs < 0) xs = min(c0 + TN, V) - 1;
+    }
+    if (mine && col == xs) {
+        a.x_out[ro] = xs;
+        a.pd_out[ro] = e / Z;
+        a.rowmax_out[ro] = M;
+        a.rowsum_out[ro] = Z;
+    }
+    stage_next(xs);
+    g.sync();
+}
+
+}  // namespace dspark

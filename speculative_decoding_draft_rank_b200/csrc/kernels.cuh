@@ -34,7 +34,9 @@ size_t draft_tiles(int V, int dtype);
 size_t draft_ws_bytes(int B, int G, int V, int r, int dtype);
 DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype);
 cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st);
-cudaError_t launch_draft_tile_tc(const DraftArgs &a, const DraftWs &w, int pos, cudaStream_t st);
+struct FinArgs;
+// bf16 rounds: every position in one cooperative launch of the tensor-core kernel.
+cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs &f, cudaStream_t st);
 
 // --------------------------------------------------------------- confidence
 cudaError_t launch_confidence(const void *h, const void *w, float bias, const float *tau, int B,

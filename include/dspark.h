@@ -43,7 +43,9 @@
  *   concurrently.
  * - Limits checked on the host: 1 <= B <= 4096, 1 <= G <= 16,
  *   2 <= V <= 2^20, 1 <= r <= 512 (a multiple of 16 for bf16), 1 <= d <= 65536,
- *   B*G <= 16384 for the scheduler, 1 <= P <= 64 profile knots.
+ *   B*G <= 16384 for the scheduler, 1 <= P <= 64 profile knots.  For bf16
+ *   rounds V is a multiple of 8 and the bf16 arrays (L, U, Wt, Tlog) start on
+ *   16-byte boundaries (TMA and vector loads); otherwise DSPARK_ERR_INVALID_ARG.
  */
 #ifndef DSPARK_H
 #define DSPARK_H

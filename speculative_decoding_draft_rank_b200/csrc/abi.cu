@@ -12,6 +12,8 @@ namespace {
 
 bool dtype_ok(int dt) { return dt == DSPARK_F32 || dt == DSPARK_BF16; }
 bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
+// bf16 arrays are read by TMA and 16-byte vector loads.
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 dspark_status check_common(int B, int G, int V, int r, int dtype) {
     if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
@@ -60,6 +62,7 @@ dspark_status dspark_draft_markov(const void *L, const void *U, const void *Wt, 
     if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
     if (!L || !U || !Wt || !x0 || !temp || !u_draft || !x_out || !pd_x_out || !rowmax_out || !rowsum_out)
         return DSPARK_ERR_INVALID_ARG;
+    if (dtype == DSPARK_BF16 && !(aligned16(L) && aligned16(U) && aligned16(Wt))) return DSPARK_ERR_INVALID_ARG;
     if (dspark_status s = check_ws(ws, ws_bytes, draft_ws_bytes(B, G, V, r, dtype))) return s;
     DraftArgs a{L, U, Wt, x0, temp, u_draft, B, G, V, r, dtype, x_out, pd_x_out, rowmax_out, rowsum_out};
     return cuda_status(launch_draft(a, ws, static_cast<cudaStream_t>(stream)));
@@ -110,6 +113,8 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
     if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
     if (!Tlog || !L || !U || !Wt || !x0 || !x || !pd_x || !rowmax || !rowsum || !temp || !u_accept ||
         !u_final || !ell || !acc_out || !tokens_out || !nout_out)
+        return DSPARK_ERR_INVALID_ARG;
+    if (dtype == DSPARK_BF16 && !(aligned16(Tlog) && aligned16(L) && aligned16(U) && aligned16(Wt)))
         return DSPARK_ERR_INVALID_ARG;
     if (dspark_status s = check_ws(ws, ws_bytes, verify_ws_bytes(B, G, V, r, dtype))) return s;
     VerifyArgs a{Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell,

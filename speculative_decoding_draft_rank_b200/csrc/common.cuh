@@ -63,18 +63,32 @@ __device__ __forceinline__ float exp_e(float x) { return fast_exp2(x * kLog2e); 
 
 // Dot product of a shared-memory fp32 vector u[0..r) with a global row w
 // (fp32 or bf16) read in 16-byte pieces; piece q goes to the threads with
-// q % tpc == part.  The caller reduces the partial sums across the tpc threads.
+// q % tpc == part.  Eight pieces are loaded before any is used (one memory
+// round trip for r <= 64 * tpc bf16); the products are accumulated in piece
+// order.  The caller reduces the partial sums across the tpc threads.
 __device__ __forceinline__ float dot_part(const float *u, const __nv_bfloat16 *w, int r, int part, int tpc) {
     float acc = 0.f;
     const uint4 *wv = reinterpret_cast<const uint4 *>(w);
     if ((reinterpret_cast<uintptr_t>(w) & 15) == 0 && (r & 7) == 0) {
-        for (int q = part; q < r / 8; q += tpc) {
-            const uint4 v = __ldg(wv + q);
-            const float *uu = u + q * 8;
-            acc = fmaf(uu[0], bf16lo(v.x), acc); acc = fmaf(uu[1], bf16hi(v.x), acc);
-            acc = fmaf(uu[2], bf16lo(v.y), acc); acc = fmaf(uu[3], bf16hi(v.y), acc);
-            acc = fmaf(uu[4], bf16lo(v.z), acc); acc = fmaf(uu[5], bf16hi(v.z), acc);
-            acc = fmaf(uu[6], bf16lo(v.w), acc); acc = fmaf(uu[7], bf16hi(v.w), acc);
+        const int n = r / 8;
+        for (int q0 = part; q0 < n; q0 += 8 * tpc) {
+            uint4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * tpc;
+                v[i] = q < n ? __ldg(wv + q) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * tpc;
+                if (q < n) {
+                    const float *uu = u + q * 8;
+                    acc = fmaf(uu[0], bf16lo(v[i].x), acc); acc = fmaf(uu[1], bf16hi(v[i].x), acc);
+                    acc = fmaf(uu[2], bf16lo(v[i].y), acc); acc = fmaf(uu[3], bf16hi(v[i].y), acc);
+                    acc = fmaf(uu[4], bf16lo(v[i].z), acc); acc = fmaf(uu[5], bf16hi(v[i].z), acc);
+                    acc = fmaf(uu[6], bf16lo(v[i].w), acc); acc = fmaf(uu[7], bf16hi(v[i].w), acc);
+                }
+            }
         }
     } else {
         for (int k = part; k < r; k += tpc) acc = fmaf(u[k], __bfloat162float(w[k]), acc);
@@ -85,11 +99,23 @@ __device__ __forceinline__ float dot_part(const float *u, const float *w, int r,
     float acc = 0.f;
     if ((reinterpret_cast<uintptr_t>(w) & 15) == 0 && (r & 3) == 0) {
         const float4 *wv = reinterpret_cast<const float4 *>(w);
-        for (int q = part; q < r / 4; q += tpc) {
-            const float4 v = __ldg(wv + q);
-            const float *uu = u + q * 4;
-            acc = fmaf(uu[0], v.x, acc); acc = fmaf(uu[1], v.y, acc);
-            acc = fmaf(uu[2], v.z, acc); acc = fmaf(uu[3], v.w, acc);
+        const int n = r / 4;
+        for (int q0 = part; q0 < n; q0 += 8 * tpc) {
+            float4 v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * tpc;
+                v[i] = q < n ? __ldg(wv + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * tpc;
+                if (q < n) {
+                    const float *uu = u + q * 4;
+                    acc = fmaf(uu[0], v[i].x, acc); acc = fmaf(uu[1], v[i].y, acc);
+                    acc = fmaf(uu[2], v[i].z, acc); acc = fmaf(uu[3], v[i].w, acc);
+                }
+            }
         }
     } else {
         for (int k = part; k < r; k += tpc) acc = fmaf(u[k], w[k], acc);

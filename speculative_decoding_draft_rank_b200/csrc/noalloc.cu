@@ -57,6 +57,8 @@ dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const vo
     if (dtype == DSPARK_BF16 && ((r % 16) != 0 || (V % 8) != 0)) return DSPARK_ERR_INVALID_ARG;
     if (!L || !U || !Wt || !x0 || !temp || !u_draft || !x_out || !pd_x_out || !rowmax_out || !rowsum_out)
         return DSPARK_ERR_INVALID_ARG;
+    const auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+    if (dtype == DSPARK_BF16 && !(a16(L) && a16(U) && a16(Wt))) return DSPARK_ERR_INVALID_ARG;
     if (dspark::draft_ws_bytes(B, G, V, r, dtype) > kNoAllocScratchBytes) return DSPARK_ERR_WORKSPACE;
     void *ws = nullptr;
     if (dspark_status s = scratch_address(&ws)) return s;

@@ -76,6 +76,26 @@ def test_draft_argument_checks(lib):
     assert _draft(lib, ws_bytes=16) == 3                           # too small
 
 
+def test_bf16_arrays_must_be_16_byte_aligned(lib):
+    """bf16 rows are moved by TMA and 16-byte vector loads: a bf16 array that
+    does not start on a 16-byte boundary is refused on the host."""
+    odd = ctypes.c_void_p(0x200008)
+    for k in range(3):   # L, U, Wt
+        args = [FAKE] * 6
+        args[k] = odd
+        assert lib.dspark_draft_markov(*args, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE,
+                                       None) == 1
+        assert lib.dspark_draft_markov_noalloc(*args, 4, 5, 1024, 16, 1, FAKE, FAKE, FAKE, FAKE, None) == 1
+    f = lib.dspark_verify
+    for k in range(4):   # Tlog, L, U, Wt
+        args = [FAKE] * 13
+        args[k] = odd
+        assert f(*args, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 1
+    # fp32 arrays have no such rule (the CUDA-core paths check alignment themselves).
+    args = [odd] + [FAKE] * 5
+    assert lib.dspark_draft_markov(*args, 4, 5, 1024, 16, 0, FAKE_WS, 16, FAKE, FAKE, FAKE, FAKE, None) == 3
+
+
 def test_schedule_and_confidence_checks(lib):
     f = lib.dspark_schedule
     assert f(FAKE, 4, 5, FAKE, FAKE, 0, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1  # P = 0

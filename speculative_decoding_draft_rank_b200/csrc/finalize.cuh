@@ -66,6 +66,7 @@ struct FinScratch {
     float rem;
 };
 
+
 constexpr int kFinChunk = 8;   // partials per thread held in registers
 
 struct FinArgs {
@@ -107,13 +108,23 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     const int K = (nTiles + nthr - 1) / nthr;
     const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
 
-    // Every load that depends on nothing else goes out first.
+    // Every load that depends on nothing else goes out first (the partials
+    // as 16-byte pieces when the thread's eight are whole and aligned).
     float cm[kFinChunk], cs[kFinChunk];
+    if (t0 + kFinChunk <= t1 && ((reinterpret_cast<uintptr_t>(pm + t0) | reinterpret_cast<uintptr_t>(ps + t0)) & 15) == 0) {
+        const float4 m0 = __ldg(reinterpret_cast<const float4 *>(pm + t0));
+        const float4 m1 = __ldg(reinterpret_cast<const float4 *>(pm + t0 + 4));
+        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(ps + t0));
+        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(ps + t0 + 4));
+        cm[0] = m0.x; cm[1] = m0.y; cm[2] = m0.z; cm[3] = m0.w; cm[4] = m1.x; cm[5] = m1.y; cm[6] = m1.z; cm[7] = m1.w;
+        cs[0] = s0.x; cs[1] = s0.y; cs[2] = s0.z; cs[3] = s0.w; cs[4] = s1.x; cs[5] = s1.y; cs[6] = s1.z; cs[7] = s1.w;
+    } else {
 #pragma unroll
-    for (int q = 0; q < kFinChunk; ++q) {
-        const bool in = t0 + q < t1;
-        cm[q] = in ? pm[t0 + q] : -INFINITY;
-        cs[q] = in ? ps[t0 + q] : 0.f;
+        for (int q = 0; q < kFinChunk; ++q) {
+            const bool in = t0 + q < t1;
+            cm[q] = in ? pm[t0 + q] : -INFINITY;
+            cs[q] = in ? ps[t0 + q] : 0.f;
+        }
     }
     const float Tb = sane_temp(a.temp[b], a.hdr);
     const float u = a.u_draft[ro];

@@ -127,14 +127,17 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, 5 ms"}
 
 
+# The sources the drafting kernel is built from (kernel, its device helpers,
+# its host launcher): profile counters are valid only for the code they were
+# taken on.
+DRAFT_KERNEL_SOURCES = ("draft_tc.cu", "finalize.cuh", "tc.cuh", "common.cuh", "kernels.cuh", "draft.cu")
+
+
 def kernel_sources_digest():
-    """Digest of the CUDA sources: profile counters are valid only for the
-    kernels they were taken on."""
-    import glob
     import hashlib
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "speculative_decoding_draft_rank_b200", "csrc", "*.cu*"))):
-        h.update(open(p, "rb").read())
+    for name in DRAFT_KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "speculative_decoding_draft_rank_b200", "csrc", name), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -264,7 +267,7 @@ def main():
             f()
         stage_graphs.append(g)
 
-    launches_per_round = 1 + 2 * w.G + 1 + 1 + 5
+    launches_per_round = (1 if w.dtype == "bf16" else 2 * w.G) + 1 + 1 + 5
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -355,6 +358,14 @@ def main():
     stage_bytes = [parts["draft_logits"] + parts["transition_W"] + parts["U_rows"], parts["hidden"],
                    w.B * w.G * 8, parts["target_rows"]]
     ach = stage_bytes[dom] / (stage_means[dom] * 1e-3) / 1e9
+    # bf16 drafting is one persistent launch for every position (timed alone
+    # in its stage graph); fp32 rounds launch a tile and a finalize kernel per
+    # position.
+    bf16 = w.dtype == "bf16"
+    stage_kernels = ["markov_tile_tc (drafting, all positions in one launch)" if bf16 else "draft stage",
+                     "confidence_kernel", "schedule_kernel", "verify stage"]
+    stage_launches = [1 if bf16 else 2 * w.G, 1, 1, 5]
+    draft_flops = 2.0 * w.B * w.G * w.r * w.V
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -367,11 +378,15 @@ def main():
                   "algorithmic_bytes": round_bytes,
                   "hbm_roofline_frac": (round_bytes / (ms * 1e-3) / 1e9) / hbm_gbs,
                   "stage_ms": dict(zip(stage_names, stage_means))},
-        "roofline": {"kernel": f"{stage_names[dom]} stage", "bound": "hbm", "achieved": ach,
+        "roofline": {"kernel": stage_kernels[dom], "bound": "hbm", "achieved": ach,
                      "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
                      "traffic": profiled_traffic(w.name) if dom == 0 else None,
                      "algorithmic_bytes": stage_bytes[dom], "ms": stage_means[dom],
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"},
+                     "launches": stage_launches[dom],
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                     "tensor": ({"flops": draft_flops, "achieved_tflops": draft_flops / (stage_means[0] * 1e-3) / 1e12,
+                                 "peak_tflops": bf16_tf, "frac": draft_flops / (stage_means[0] * 1e-3) / 1e12 / bf16_tf}
+                                if dom == 0 else None)},
         "e2e": {"value": ell_tot / (e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e},
         "gpu_launches": launches_per_round * args.steps,

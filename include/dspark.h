@@ -70,7 +70,9 @@ typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
 
 typedef enum {
     DSPARK_SCHED_ALL = 0,               /* verify every drafted position */
-    DSPARK_SCHED_GREEDY_EARLY_STOP = 1  /* Algorithm 1 */
+    DSPARK_SCHED_GREEDY_EARLY_STOP = 1, /* Algorithm 1 */
+    DSPARK_SCHED_GLOBAL_ARGMAX = 2,     /* variant: offline search, no early stop */
+    DSPARK_SCHED_THRESHOLD = 3          /* variant: static survival threshold (dspark_schedule_threshold) */
 } dspark_sched_mode;
 
 /* Bits of the device status word. */
@@ -139,8 +141,14 @@ dspark_status dspark_confidence(const void *h, const void *w, float bias, const 
  *   t(n) is piecewise linear through the P knots (knots_n[j], knots_t[j]),
  *   knots_n[0] = 0 and strictly increasing, continued past the last knot
  *   with the last segment's slope (constant when P = 1); knots_t > 0.
+ *   mode DSPARK_SCHED_GLOBAL_ARGMAX (a scheduler variant, the offline global
+ *   search of [PL] Appendix A): the admitted count is the n in 0..budget
+ *   that maximises Theta_n (the lowest such n); it may look past a drop of
+ *   Theta, so with confidences that depend on drawn tokens it is not
+ *   lossless ([PL] Appendix A's counterexample).
  * Inputs:  S [B,G] f32, knots_n [P] int32, knots_t [P] f64 (device arrays),
- *          budget, mode (dspark_sched_mode).
+ *          budget, mode (DSPARK_SCHED_ALL, _GREEDY_EARLY_STOP or
+ *          _GLOBAL_ARGMAX; anything else is DSPARK_ERR_INVALID_ARG).
  * Outputs: ell_out [B] int32 admitted prefix length per request;
  *          n_adm_out [1] int32; theta_out [1] f64 = Theta at n_adm;
  *          order_out [B*G] int32 sorted candidate indices, or NULL. */
@@ -149,6 +157,21 @@ dspark_status dspark_schedule(const float *S, int B, int G, const int32_t *knots
                               const double *knots_t, int P, int budget, int mode, void *ws,
                               size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out,
                               double *theta_out, int32_t *order_out, void *stream);
+
+/* Scheduler variant: static-threshold pruning.  [KB] Key Contributions ranks
+ * candidates by cumulative survival; this variant admits, in the same stable
+ * order (S descending, ties by position-major index), every candidate with
+ * S >= threshold, at most `budget` (< 0: none).  No profile and no objective:
+ * the cut depends on the survival level alone, so a request's admitted
+ * positions are a prefix whenever its S is non-increasing (as the confidence
+ * stage's cumulative products are).
+ * Inputs:  S [B,G] f32, threshold, budget; same limits and workspace as
+ *          dspark_schedule.
+ * Outputs: ell_out [B] int32, n_adm_out [1] int32, order_out [B*G] int32 or
+ *          NULL. */
+dspark_status dspark_schedule_threshold(const float *S, int B, int G, float threshold, int budget, void *ws,
+                                        size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out,
+                                        int32_t *order_out, void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Stage 4: exact rejection-sampling verification.

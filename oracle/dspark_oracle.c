@@ -23,7 +23,7 @@
  * widened to double; all sums run sequentially in index order; exp() is the C
  * library's.  No blocking, fusion or reordering beyond the definitions.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - the Markov bias at position i is U[x_{i-1}] W with x_0 the last committed
  *     token, also at i = 1;
  *   - temperature T scales draft and target logits alike; T = 0 means greedy
@@ -326,6 +326,40 @@ int dspark_oracle_schedule(int B, int G, const double *S, int P, const int *knot
     *theta_out = theta;
     *margin_theta_out = mtheta;
     *margin_gap_out = (n > 0 && n < N) ? fabs(c[n - 1].s - c[n].s) : INFINITY;
+    free(c);
+    return ORACLE_OK;
+}
+
+/* Static-threshold pruning, a scheduler variant ([KB] Key Contributions:
+ * candidates ranked by cumulative survival; the threshold form prunes by a
+ * fixed survival level instead of the objective): in the same sorted order as
+ * above, admit the candidates with S >= threshold, at most `budget`
+ * (budget < 0: none).  Because the order is by S descending, the admitted
+ * candidates are exactly those with S >= threshold (up to the budget), and a
+ * request's admitted positions are a prefix whenever its S is non-increasing.
+ * Outputs ell [B], n_adm, order [B*G]. */
+int dspark_oracle_schedule_threshold(int B, int G, const double *S, double threshold, int budget, int *ell_out,
+                                     int *n_adm_out, int *order_out)
+{
+    if (B < 1 || G < 1) return ORACLE_ERR_ARG;
+    int N = B * G;
+    cand_t *c = malloc(sizeof(cand_t) * (size_t)N);
+    if (!c) return ORACLE_ERR_NOMEM;
+    for (int i = 0; i < G; ++i)
+        for (int b = 0; b < B; ++b) {
+            c[i * B + b].s = S[(size_t)b * G + i];
+            c[i * B + b].idx = i * B + b;
+        }
+    qsort(c, (size_t)N, sizeof(cand_t), cand_cmp);
+    if (order_out)
+        for (int n = 0; n < N; ++n) order_out[n] = c[n].idx;
+    int limit = N;
+    if (budget >= 0 && budget < limit) limit = budget;
+    int n = 0;
+    while (n < limit && c[n].s >= threshold) ++n;
+    for (int b = 0; b < B; ++b) ell_out[b] = 0;
+    for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;
+    *n_adm_out = n;
     free(c);
     return ORACLE_OK;
 }

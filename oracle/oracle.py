@@ -143,6 +143,19 @@ def schedule(S, knots_n, knots_t, budget=-1, mode=SCHED_GREEDY_EARLY_STOP, force
     return ScheduleResult(ell, n_adm.value, th.value, order, mth.value, mgap.value)
 
 
+def schedule_threshold(S, threshold, budget=-1):
+    """Static-threshold pruning over survivals S [B,G]: the sorted candidates
+    with S >= threshold, at most `budget`.  Returns (ell [B], n_adm, order)."""
+    S = _f64(S)
+    B, G = S.shape
+    ell = np.zeros(B, np.int32); order = np.zeros(B * G, np.int32)
+    n_adm = ctypes.c_int(0)
+    rc = _load().dspark_oracle_schedule_threshold(B, G, _p(S), ctypes.c_double(float(threshold)), int(budget),
+                                                  _p(ell), ctypes.byref(n_adm), _p(order))
+    _check(rc, "schedule_threshold")
+    return ell, n_adm.value, order
+
+
 @dataclass
 class VerifyResult:
     acc: np.ndarray          # [B] accepted count A

@@ -20,6 +20,8 @@ DSPARK_F32 = 0
 DSPARK_BF16 = 1
 SCHED_ALL = 0
 SCHED_GREEDY_EARLY_STOP = 1
+SCHED_GLOBAL_ARGMAX = 2
+SCHED_THRESHOLD = 3
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DTYPE", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
 DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
@@ -27,7 +29,7 @@ DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov", "dspark_confidence",
            "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
            "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
-           "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc")
+           "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold")
 
 
 class DsparkError(RuntimeError):
@@ -60,6 +62,8 @@ def load() -> ctypes.CDLL:
     lib.dspark_schedule_workspace_size.argtypes = [_i, _i]
     lib.dspark_schedule.restype = _i
     lib.dspark_schedule.argtypes = [_vp, _i, _i, _vp, _vp, _i, _i, _i, _vp, _sz, _vp, _vp, _vp, _vp, _vp]
+    lib.dspark_schedule_threshold.restype = _i
+    lib.dspark_schedule_threshold.argtypes = [_vp, _i, _i, _f, _i, _vp, _sz, _vp, _vp, _vp, _vp]
     lib.dspark_verify_workspace_size.restype = _sz
     lib.dspark_verify_workspace_size.argtypes = [_i] * 5
     lib.dspark_verify.restype = _i
@@ -155,6 +159,13 @@ def dspark_schedule(S, knots_n, knots_t, budget, mode, ws, ell_out, n_adm_out, t
     _call("dspark_schedule", _ptr(S), B, G, _ptr(knots_n), _ptr(knots_t), knots_n.numel(), int(budget),
           int(mode), _ptr(ws), ws.numel() * ws.element_size(), _ptr(ell_out), _ptr(n_adm_out),
           _ptr(theta_out), _ptr(order_out), _stream(stream))
+
+
+def dspark_schedule_threshold(S, threshold, budget, ws, ell_out, n_adm_out, order_out=None, stream=None):
+    """Static-threshold pruning: the sorted candidates with S >= threshold."""
+    B, G = S.shape
+    _call("dspark_schedule_threshold", _ptr(S), B, G, ctypes.c_float(threshold), int(budget), _ptr(ws),
+          ws.numel() * ws.element_size(), _ptr(ell_out), _ptr(n_adm_out), _ptr(order_out), _stream(stream))
 
 
 def dspark_verify(Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell, ws, acc_out,

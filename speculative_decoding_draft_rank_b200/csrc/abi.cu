@@ -90,11 +90,24 @@ dspark_status dspark_schedule(const float *S, int B, int G, const int32_t *knots
     if (dspark_status s = injected("dspark_schedule")) return s;
     if (B < 1 || B > 4096 || G < 1 || G > 16 || B * G > 16384 || P < 1 || P > 64)
         return DSPARK_ERR_INVALID_ARG;
-    if (mode != DSPARK_SCHED_ALL && mode != DSPARK_SCHED_GREEDY_EARLY_STOP) return DSPARK_ERR_INVALID_ARG;
+    if (mode != DSPARK_SCHED_ALL && mode != DSPARK_SCHED_GREEDY_EARLY_STOP && mode != DSPARK_SCHED_GLOBAL_ARGMAX)
+        return DSPARK_ERR_INVALID_ARG;
     if (!S || !knots_n || !knots_t || !ell_out || !n_adm_out || !theta_out) return DSPARK_ERR_INVALID_ARG;
     if (dspark_status s = check_ws(ws, ws_bytes, schedule_ws_bytes(B, G))) return s;
-    return cuda_status(launch_schedule(S, B, G, knots_n, knots_t, P, budget, mode, ws, ell_out, n_adm_out,
+    return cuda_status(launch_schedule(S, B, G, knots_n, knots_t, P, budget, mode, 0.f, ws, ell_out, n_adm_out,
                                        theta_out, order_out, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_schedule_threshold(const float *S, int B, int G, float threshold, int budget, void *ws,
+                                        size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out,
+                                        int32_t *order_out, void *stream) {
+    if (dspark_status s = injected("dspark_schedule_threshold")) return s;
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || B * G > 16384 || !(threshold == threshold))
+        return DSPARK_ERR_INVALID_ARG;
+    if (!S || !ell_out || !n_adm_out) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, schedule_ws_bytes(B, G))) return s;
+    return cuda_status(launch_schedule(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_THRESHOLD, threshold, ws,
+                                       ell_out, n_adm_out, nullptr, order_out, static_cast<cudaStream_t>(stream)));
 }
 
 size_t dspark_verify_workspace_size(int B, int G, int V, int r, int dtype) {

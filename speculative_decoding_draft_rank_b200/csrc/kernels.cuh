@@ -45,7 +45,7 @@ cudaError_t launch_confidence(const void *h, const void *w, float bias, const fl
 // ---------------------------------------------------------------- scheduler
 size_t schedule_ws_bytes(int B, int G);
 cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
-                            const double *knots_t, int P, int budget, int mode, void *ws,
+                            const double *knots_t, int P, int budget, int mode, float threshold, void *ws,
                             int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
                             int32_t *order_out, cudaStream_t st);
 

@@ -19,6 +19,12 @@
 //      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index
 //      (or the budget) is the admitted count;
 //   4. admitted candidates are counted per request in shared memory -> ell.
+// Variants (menfem.com KB entry, "Key Contributions"; paperlayer.ai summary,
+// Appendix A): the offline global search admits the count that maximises
+// Theta(n) = V_n / t(n) over every n up to the budget (lowest n on ties) --
+// no early stop, so not lossless when confidence depends on drawn tokens --
+// and static-threshold pruning admits the sorted candidates with
+// S >= threshold, up to the budget.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -59,8 +65,9 @@ __device__ __forceinline__ void bitonic_warp_step(unsigned long long &v0, unsign
 
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
-    const double *__restrict__ knots_t, int P, int budget, int mode, int32_t *__restrict__ ell_out,
-    int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out, int32_t *__restrict__ order_out)
+    const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
+    int32_t *__restrict__ ell_out, int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
+    int32_t *__restrict__ order_out)
 {
     extern __shared__ __align__(16) unsigned char sched_smem[];
     const int N = B * G;
@@ -157,8 +164,43 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     __syncthreads();
     const double Vbase = (double)B + (wsum - run) + (wid > 0 ? red_d[wid - 1] : 0.0);
     const int limit = (budget >= 0 && budget < N) ? budget : N;
-    int first_stop = 0x7fffffff;
-    {
+    int nadm;
+    if (mode == DSPARK_SCHED_GLOBAL_ARGMAX) {
+        // Theta at every count: n = 0 (thread 0) and n + 1 for the thread's
+        // ranks n; the block argmax keeps the lowest count among equal values.
+        double best = -INFINITY;
+        int bestn = 0x7fffffff;
+        if (tid == 0) { best = (double)B / profile_at(kn_s, kt_s, P, 0.0); bestn = 0; }
+        double Vn = Vbase;
+        for (int n = c0; n < c1 && n < limit; ++n) {
+            Vn += surv(n);
+            const double th = Vn / profile_at(kn_s, kt_s, P, (double)(n + 1));
+            if (th > best) { best = th; bestn = n + 1; }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+            const int on = __shfl_xor_sync(0xffffffffu, bestn, o);
+            if (ob > best || (ob == best && on < bestn)) { best = ob; bestn = on; }
+        }
+        __shared__ double arg_v[32];
+        __shared__ int arg_n[32];
+        if (lane == 0) { arg_v[wid] = best; arg_n[wid] = bestn; }
+        __syncthreads();
+        best = arg_v[0];
+        bestn = arg_n[0];
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            if (arg_v[w] > best || (arg_v[w] == best && arg_n[w] < bestn)) { best = arg_v[w]; bestn = arg_n[w]; }
+        nadm = bestn;
+    } else if (mode == DSPARK_SCHED_THRESHOLD) {
+        // The sorted survivals fall below the threshold at one index.
+        int first_below = 0x7fffffff;
+        for (int n = c0; n < c1; ++n)
+            if (surv(n) < (double)threshold) { first_below = n; break; }
+        nadm = block_min_i(first_below, red_i);
+        if (nadm > limit) nadm = limit;
+    } else {
+        int first_stop = 0x7fffffff;
         double Vn = Vbase;
         for (int n = c0; n < c1 && n < limit; ++n) {
             const double sn = surv(n);
@@ -167,9 +209,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
             if ((Vn + sn) * t0 < Vn * t1) { first_stop = n; break; }
             Vn += sn;
         }
+        nadm = block_min_i(first_stop, red_i);
+        if (nadm > limit) nadm = limit;
     }
-    int nadm = block_min_i(first_stop, red_i);
-    if (nadm > limit) nadm = limit;
 
     // Objective at the admitted count: V_nadm from the chunk that holds
     // index nadm (or the last chunk when nadm == N).
@@ -190,22 +232,22 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     for (int b = tid; b < B; b += blockDim.x) ell_out[b] = ell_s[b];
     if (tid == 0) {
         *n_adm_out = nadm;
-        *theta_out = Vadm_s / profile_at(kn_s, kt_s, P, (double)nadm);
+        if (theta_out != nullptr) *theta_out = Vadm_s / profile_at(kn_s, kt_s, P, (double)nadm);
     }
 }
 
 size_t schedule_ws_bytes(int, int) { return sizeof(WsHeader); }
 
 cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
-                            const double *knots_t, int P, int budget, int mode, void *,
+                            const double *knots_t, int P, int budget, int mode, float threshold, void *,
                             int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
                             int32_t *order_out, cudaStream_t st) {
     const size_t smem = sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096;
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, ell_out,
-                                                    n_adm_out, theta_out, order_out);
+    schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, threshold,
+                                                    ell_out, n_adm_out, theta_out, order_out);
     return cudaGetLastError();
 }
 

@@ -103,6 +103,14 @@ def test_schedule_and_confidence_checks(lib):
     assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 9, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1  # mode
     assert f(FAKE, 4096, 8, FAKE, FAKE, 2, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1
     assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 1, None, 1 << 20, FAKE, FAKE, FAKE, None, None) == 3
+    assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 3, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1  # threshold mode
+    assert f(FAKE, 4, 5, FAKE, FAKE, 2, -1, 4, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None, None) == 1
+    h = lib.dspark_schedule_threshold
+    assert h(FAKE, 0, 5, ctypes.c_float(0.5), -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 1    # B = 0
+    assert h(FAKE, 4096, 8, ctypes.c_float(0.5), -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 1  # B*G
+    assert h(FAKE, 4, 5, ctypes.c_float(float("nan")), -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 1
+    assert h(None, 4, 5, ctypes.c_float(0.5), -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 1
+    assert h(FAKE, 4, 5, ctypes.c_float(0.5), -1, None, 1 << 20, FAKE, FAKE, None, None) == 3
     g = lib.dspark_confidence
     assert g(FAKE, FAKE, ctypes.c_float(0), None, 4, 5, 0, 0, FAKE, FAKE, None) == 1   # d = 0
     assert g(FAKE, FAKE, ctypes.c_float(0), None, 4, 5, 8, 3, FAKE, FAKE, None) == 2   # dtype

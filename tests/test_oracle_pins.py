@@ -294,6 +294,54 @@ def test_scheduler_non_anticipation():
         assert (res.ell[b] > k) == (res2.ell[b] > k)
 
 
+def test_scheduler_global_search_maximises_theta():
+    """The offline-search variant admits the count that maximises Theta over
+    every n (the lowest such n), whatever the profile's shape (brute force over
+    prefix-closed sets; non-convex step profiles included)."""
+    rng = _rng(11)
+    for trial in range(60):
+        B, G = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+        S = _monotone_S(rng, B, G)
+        if trial % 2:
+            kn, kt = _convex_profile(rng)
+        else:   # a step-shaped, non-convex profile
+            kn = np.array([0, 1, 2, 3], np.int32)
+            kt = np.array([1.0, 1.0 + rng.uniform(0, 2), 3.2, 3.3])
+        best = {}
+        for ells in _prefix_sets(B, G):
+            n = sum(ells)
+            best[n] = max(best.get(n, -1), sum(S[b, :ells[b]].sum() for b in range(B)))
+        theta = [(B + best[n]) / _t_of(kn, kt, n) for n in range(B * G + 1)]
+        res = oracle.schedule(S, kn, kt, -1, oracle.SCHED_GLOBAL_ARGMAX)
+        assert res.n_adm == int(np.argmax(theta))
+        assert res.theta == pytest.approx(max(theta), rel=1e-12)
+
+
+def test_scheduler_threshold_is_the_survival_cut():
+    """Static-threshold pruning admits exactly the candidates with S >= the
+    threshold (all of them, or the first `budget` in the stable order), which
+    for monotone survivals are prefixes of every request."""
+    rng = _rng(12)
+    for trial in range(80):
+        B, G = int(rng.integers(1, 6)), int(rng.integers(1, 6))
+        c = rng.choice([1.0, 0.9, 0.5, 0.25], size=(B, G))
+        S = np.cumprod(c, axis=1)
+        th = float(rng.choice(S.ravel())) if trial % 3 else float(rng.uniform(0, 1))
+        budget = -1 if trial % 4 else int(rng.integers(0, B * G + 1))
+        ell, n_adm, order = oracle.schedule_threshold(S, th, budget)
+        # The stable order by S descending over the position-major list.
+        ids = sorted(range(B * G), key=lambda i: (-S[i % B, i // B], i))
+        assert list(order) == ids
+        above = [i for i in ids if S[i % B, i // B] >= th]
+        take = above if budget < 0 else above[:budget]
+        assert n_adm == len(take)
+        for b in range(B):
+            assert ell[b] == sum(1 for i in take if i % B == b)
+            assert all(S[b, k] >= th for k in range(ell[b]))   # a prefix of the request
+            if budget < 0:
+                assert all(S[b, k] < th for k in range(ell[b], G))
+
+
 # --------------------------------------------------------------------------
 # Verification
 # --------------------------------------------------------------------------

@@ -200,6 +200,78 @@ def run_reference(args):
     return 0
 
 
+def run_sharded(args):
+    """The request-sharded round: each rank drafts, scores and verifies its
+    own headline-sized batch; the survivals are all-gathered (NCCL) and every
+    rank runs the same admission over the whole batch (profile knots scaled
+    by the rank count).  Eager launches per round (the collective sits
+    between library calls); device time per round is the max over ranks."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_draft_rank_b200.round import DeviceRound
+    from speculative_decoding_draft_rank_b200.sharded import ShardedRound
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if dist.is_available() and not dist.is_initialized():
+        if "MASTER_ADDR" not in os.environ:
+            os.environ["MASTER_ADDR"] = "127.0.0.1"
+            os.environ["MASTER_PORT"] = "29511"
+        dist.init_process_group("nccl", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = _workload(args.workload)
+    w.seed = rank
+    inp = w.inputs()
+    kn = np.asarray(w.knots_n, np.int64) * world
+    dr = DeviceRound(inp, w.knots_n, w.knots_t, w.budget, w.mode, device=dev)
+    sh = ShardedRound(dr, kn.astype(np.int32), w.knots_t, w.budget * world if w.budget >= 0 else -1, w.mode)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            sh.run(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    times = []
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            flush.zero_()
+            e0.record(stream)
+            sh.run(stream)
+            e1.record(stream)
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    dist.barrier()
+    ms = statistics.mean(times)
+    ell_sum = int(dr.o["ell"].sum().item())
+    tt = torch.tensor([ms, float(ell_sum)], device=dev, dtype=torch.float64)
+    gathered = [torch.zeros_like(tt) for _ in range(world)]
+    dist.all_gather(gathered, tt)
+    ms = max(float(g[0]) for g in gathered)
+    ell_tot = sum(float(g[1]) for g in gathered)
+    if dr.device_status() != 0:
+        raise RuntimeError("device status word set")
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": ell_tot / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, one batch per rank)",
+            "config": {"workload": w.name, "B_per_rank": w.B, "G": w.G, "V": w.V, "r": w.r, "d": w.d,
+                       "l2_flush": "256 MiB write before every timed round", "graph_replay": False,
+                       "parallelism": f"{world} ranks, request-sharded, survivals all-gathered (NCCL)"},
+            "round": {"admitted_draft_tokens": ell_tot, "n_adm_global": int(sh.n_adm.item())}}))
+    dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -212,9 +284,14 @@ def main():
     ap.add_argument("--reference-requests", type=int, default=8,
                     help="requests per step of the reference arm (the oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+                    help="replicas: every rank an independent engine (default); sharded: one engine over all "
+                         "ranks' requests, survivals all-gathered for one global admission")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.mode == "sharded":
+        return run_sharded(args)
 
     import torch
     import torch.distributed as dist

@@ -402,28 +402,31 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     for (int c = 0; c < kSeg / 32; ++c) {
                         float y[32];
                         tc::tmem_ld32(taddr + c * 32, y);
+                        // y = L + Delta, two columns per instruction.
     #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             const uint4 qv = cur[c * 4 + u];
-                            y[u * 8 + 0] += bf16lo(qv.x); y[u * 8 + 1] += bf16hi(qv.x);
-                            y[u * 8 + 2] += bf16lo(qv.y); y[u * 8 + 3] += bf16hi(qv.y);
-                            y[u * 8 + 4] += bf16lo(qv.z); y[u * 8 + 5] += bf16hi(qv.z);
-                            y[u * 8 + 6] += bf16lo(qv.w); y[u * 8 + 7] += bf16hi(qv.w);
+                            const uint32_t wq[4] = {qv.x, qv.y, qv.z, qv.w};
+    #pragma unroll
+                            for (int h = 0; h < 4; ++h) {
+                                const float2 yy = add2(make_float2(y[u * 8 + 2 * h], y[u * 8 + 2 * h + 1]),
+                                                       make_float2(bf16lo(wq[h]), bf16hi(wq[h])));
+                                y[u * 8 + 2 * h] = yy.x;
+                                y[u * 8 + 2 * h + 1] = yy.y;
+                            }
                         }
                         if (!whole) {
     #pragma unroll
                             for (int e = 0; e < 32; ++e)
                                 if (cbase + c * 32 + e >= V) y[e] = -INFINITY;
                         }
-                        // Tree max (short dependency chains).
-                        float t16[16];
+                        // Chunk max: a tree of three-input maxima.
+                        float t11[11];
     #pragma unroll
-                        for (int e = 0; e < 16; ++e) t16[e] = fmaxf(y[e], y[e + 16]);
-    #pragma unroll
-                        for (int wdt = 8; wdt > 0; wdt >>= 1)
-    #pragma unroll
-                            for (int e = 0; e < wdt; ++e) t16[e] = fmaxf(t16[e], t16[e + wdt]);
-                        const float cm = t16[0];
+                        for (int e = 0; e < 10; ++e) t11[e] = max3(y[3 * e], y[3 * e + 1], y[3 * e + 2]);
+                        t11[10] = fmaxf(y[30], y[31]);
+                        const float cm = max3(max3(t11[0], t11[1], t11[2]), max3(t11[3], t11[4], t11[5]),
+                                              max3(max3(t11[6], t11[7], t11[8]), t11[9], t11[10]));
                         if (warp_greedy && cm > m) {
                             int ix = 0x7fffffff;
     #pragma unroll
@@ -433,10 +436,21 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                         }
                         const float mn = fmaxf(m, cm);
                         if (warp_soft) {
-                            float a4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent sums
+                            // exp((y - mn) / T) = 2^(y * cexp - mn * cexp): one fused
+                            // multiply-add per two columns, then the two ex2.
+                            const float2 c2 = make_float2(cexp, cexp);
+                            const float nmc = -mn * cexp;
+                            const float2 n2 = make_float2(nmc, nmc);
+                            float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                            make_float2(0.f, 0.f)};   // four independent pairs of sums
     #pragma unroll
-                            for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2((y[e] - mn) * cexp);
-                            const float acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                            for (int e = 0; e < 16; ++e) {
+                                const float2 arg = fma2(make_float2(y[2 * e], y[2 * e + 1]), c2, n2);
+                                s2[e & 3] = add2(s2[e & 3], make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
+                            }
+                            const float2 p01 = add2(s2[0], s2[1]), p23 = add2(s2[2], s2[3]);
+                            const float2 pall = add2(p01, p23);
+                            const float acc = pall.x + pall.y;
                             s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + acc;
                         }
                         m = mn;

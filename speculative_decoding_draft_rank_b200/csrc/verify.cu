@@ -314,12 +314,10 @@ __global__ void __launch_bounds__(kRowsWarpThreads, 3) verify_rows_warp(const __
 #pragma unroll
             for (int i = 0; i < 16; ++i) v[i] = buf[st & 1][i];
             if (st + 2 < kSteps) ld_row32(row, c0 + (st + 2) * kStep + lane * 32, c1, a32, buf[st & 1]);
+            // Step maximum: four running three-input maxima over the value pairs.
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                m4[(2 * i) & 3] = fmaxf(m4[(2 * i) & 3], bf16lo(v[i]));
-                m4[(2 * i + 1) & 3] = fmaxf(m4[(2 * i + 1) & 3], bf16hi(v[i]));
-            }
+            for (int i = 0; i < 16; ++i) m4[i & 3] = max3(m4[i & 3], bf16lo(v[i]), bf16hi(v[i]));
             const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             const int base = c0 + st * kStep + lane * 32;
             if (cexp == 0.f) {   // greedy row: the lowest index of the largest value (warp-uniform)
@@ -334,12 +332,15 @@ __global__ void __launch_bounds__(kRowsWarpThreads, 3) verify_rows_warp(const __
                     m = cm;
                 }
             } else if (cm > -INFINITY) {
+                // exp((t - mn) / T) = 2^(t * cexp - mn * cexp): one fused
+                // multiply-add per column.
                 const float mn = fmaxf(m, cm);
+                const float nmc = -mn * cexp;
                 float a4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    a4[(2 * i) & 3] += fast_exp2((bf16lo(v[i]) - mn) * cexp);
-                    a4[(2 * i + 1) & 3] += fast_exp2((bf16hi(v[i]) - mn) * cexp);
+                    a4[(2 * i) & 3] += fast_exp2(fmaf(bf16lo(v[i]), cexp, nmc));
+                    a4[(2 * i + 1) & 3] += fast_exp2(fmaf(bf16hi(v[i]), cexp, nmc));
                 }
                 s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
                 m = mn;

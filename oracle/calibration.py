@@ -80,7 +80,10 @@ def ece_vec(s, y, M):
     b = np.minimum(M - 1, np.floor(s * M).astype(np.int64))
     acc = np.zeros(M)
     np.add.at(acc, b, np.asarray(y, dtype=np.float64) - s)
-    return float(np.sum(np.abs(acc))) / s.shape[0]
+    tot = 0.0
+    for m in range(M):
+        tot += abs(float(acc[m]))
+    return tot / s.shape[0]
 
 
 def survival(z, tau):
@@ -103,7 +106,9 @@ def sts_fit(z, acc, tau_grid, M, vectorised=True):
     For i = 1..G in turn, with tau_1..tau_{i-1} already fixed, every grid
     temperature t gives the candidate survivals S_{i-1} * sigmoid(z_i / t);
     tau_i is the first grid entry whose candidate has the least ECE against
-    the labels y_i (A >= i).  The ordering of the survivals along a request's
+    the labels y_i (A >= i).  A grid entry that is not a positive finite
+    number is no temperature: its ECE counts as +inf (chosen only when no
+    entry is valid, and then the first).  The ordering of the survivals along a request's
     prefix is kept by construction: every factor lies in (0, 1), so S_i never
     exceeds S_{i-1}.
 
@@ -123,16 +128,17 @@ def sts_fit(z, acc, tau_grid, M, vectorised=True):
     ece_all = np.empty((G, K))
     prev = np.ones(N)
     for i in range(G):
-        best_k, best_e, best_s = -1, np.inf, None
         for k in range(K):
-            s = prev * sigmoid(z[:, i] / float(grid[k]))
-            ek = e(s, y[:, i], M)
-            ece_all[i, k] = ek
-            if ek < best_e:
-                best_k, best_e, best_s = k, ek, s
-        tau[i] = grid[best_k]
-        ece_fit[i] = best_e
-        prev = best_s
+            t = float(grid[k])
+            if not (np.isfinite(t) and t > 0.0):
+                ece_all[i, k] = np.inf      # not a temperature: never preferred
+                continue
+            ece_all[i, k] = e(prev * sigmoid(z[:, i] / t), y[:, i], M)
+        least = np.min(ece_all[i])
+        kstar = int(np.flatnonzero(ece_all[i] == least)[0])   # first of the least
+        tau[i] = grid[kstar]
+        ece_fit[i] = ece_all[i, kstar]
+        prev = prev * sigmoid(z[:, i] / float(grid[kstar]))
     return tau, ece_raw, ece_fit, ece_all
 
 

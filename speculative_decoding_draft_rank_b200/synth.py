@@ -142,3 +142,54 @@ def select_requests(inp: RoundInputs, idx) -> RoundInputs:
     return RoundInputs(len(idx), inp.G, inp.V, inp.r, inp.d, inp.dtype, inp.L[idx], inp.Tlog[idx],
                        inp.U, inp.W, inp.h[idx], inp.w, inp.bias, inp.x0[idx], inp.temp[idx],
                        inp.u_draft[idx], inp.u_accept[idx], inp.u_final[idx], bits)
+
+
+@dataclass
+class CalibrationSet:
+    """Labelled confidence-head outputs of N verified draft blocks.
+
+    z [N, G] fp32: the head's logits (w . h + bias) per position;
+    acc [N] int32: the accepted count A of each block, verified at full
+    length G (positions 1..A accepted, A + 1 rejected when A < G);
+    k [G] fp32: the over-confidence factor the logits were scaled by;
+    t [N, G] fp32: the latent logits whose logistic law drew acceptance."""
+    N: int
+    G: int
+    z: np.ndarray
+    acc: np.ndarray
+    k: np.ndarray
+    t: np.ndarray
+
+
+def calibration_set(N: int, G: int, k=2.0, seed: int = 0, mu0: float = 2.5, dmu: float = 0.5,
+                    sigma: float = 1.5) -> CalibrationSet:
+    """Draw a calibration set with a known miscalibration.
+
+    Recipe (one PCG64 child stream per tensor from ``SeedSequence(seed)``):
+    latent logits t[n, i] ~ N(mu0 - dmu * i, sigma^2) for i = 0..G-1, so the
+    per-position acceptance falls along the block; independent logistic
+    noise e[n, i] ~ Logistic(0, 1); position i passes when e < t (an event of
+    probability 1 / (1 + exp(-t)), drawn without evaluating it); A is the
+    number of leading passes.  The head reports z = k_i * t: k > 1 is an
+    over-confident head (the pages report raw ECE of 3-8 %), k < 1 an
+    under-confident one.  ``k`` is a scalar or a length-G sequence."""
+    ss = np.random.SeedSequence(seed)
+    s_t, s_e = ss.spawn(2)
+    gen = lambda s: np.random.Generator(np.random.PCG64(s))
+    mu = (np.float32(mu0) - np.float32(dmu) * np.arange(G, dtype=np.float32)).astype(np.float32)
+    t = gen(s_t).standard_normal((N, G), dtype=np.float32) * np.float32(sigma) + mu[None, :]
+    e = gen(s_e).logistic(0.0, 1.0, size=(N, G)).astype(np.float32)
+    passed = e < t
+    acc = np.where(passed.all(axis=1), G, np.argmin(passed, axis=1)).astype(np.int32)
+    kk = np.broadcast_to(np.asarray(k, dtype=np.float32), (G,)).astype(np.float32)
+    z = (t * kk[None, :]).astype(np.float32)
+    return CalibrationSet(N, G, np.ascontiguousarray(z), acc, kk, t)
+
+
+def tau_grid(K: int = 65, lo: float = 0.25, hi: float = 4.0) -> np.ndarray:
+    """K log-spaced candidate temperatures from lo to hi (fp32); with the
+    defaults the middle entry is exactly 1."""
+    g = np.exp(np.linspace(np.log(lo), np.log(hi), K)).astype(np.float32)
+    if K % 2 == 1 and abs(np.log(lo) + np.log(hi)) < 1e-12:
+        g[K // 2] = np.float32(1.0)
+    return g

@@ -272,6 +272,218 @@ def run_sharded(args):
     return 0
 
 
+# The sources of the calibration kernels: their fp64 counters are valid only
+# for the code they were taken on.
+STS_KERNEL_SOURCES = ("calibration.cu", "calibration.cuh", "common.cuh")
+
+
+def sts_sources_digest():
+    import hashlib
+    h = hashlib.sha256()
+    for name in STS_KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, "speculative_decoding_draft_rank_b200", "csrc", name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_sts_fp64(workload_name):
+    """fp64 FLOPs of one fit (all positions) and DRAM bytes from the committed
+    ncu summary, or None when the kernels changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", f"sts_position_fp64_{workload_name}.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    return d if d.get("sources_digest") == sts_sources_digest() else None
+
+
+# fp64 peak: 64 fp64 lanes per SM (one fused multiply-add each per clock, the
+# half rate of the 128 fp32 lanes), 148 SMs.
+FP64_LANES_PER_SM = 64
+SMS = 148
+
+
+def run_sts(args):
+    """Sequential temperature scaling fit of the confidence head (one step =
+    one fit over N labelled blocks: every grid temperature at every position,
+    left to right) and the survivals' ROC-AUC, on one GPU per rank (replicas:
+    every rank fits its own seeded set; time = max over ranks)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_draft_rank_b200 import _lib, workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    w = wl.calibration_headline()
+    metric = f"STS fit candidate evaluations/s, N={w.N} γ={w.G} K={w.K} M={w.M}"
+    unit = "candidate evaluations/s"
+    evals = w.N * (w.K + 1) * w.G          # every grid entry plus the raw chain, every position
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        from oracle import calibration as C
+        cs = w.inputs()
+        grid = w.grid()
+        times = []
+        for _ in range(max(1, args.warmup)):
+            C.sts_fit(cs.z, cs.acc, grid, w.M)
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            C.sts_fit(cs.z, cs.acc, grid, w.M)
+            times.append(time.perf_counter() - t0)
+        ms = 1e3 * statistics.mean(times)
+        v = evals / (ms * 1e-3)
+        print(json.dumps({"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": 1,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": {"workload": w.name, "N": w.N, "G": w.G, "K": w.K, "M": w.M},
+                          "cpu_baseline": {"value": v, "unit": unit, "cores": 1, "kind": "oracle",
+                                           "sample": "the whole fit, every step"},
+                          "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return 0
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w.seed = rank
+    cs = w.inputs()
+    grid = w.grid()
+    f32, f64 = dict(dtype=torch.float32, device=dev), dict(dtype=torch.float64, device=dev)
+    z = torch.from_numpy(cs.z).to(dev)
+    acc = torch.from_numpy(cs.acc).to(dev)
+    g = torch.from_numpy(grid).to(dev)
+    z_h = torch.from_numpy(cs.z).pin_memory()
+    acc_h = torch.from_numpy(cs.acc).pin_memory()
+    ws = torch.zeros(_lib.dspark_sts_workspace_size(w.N, w.G, w.K, w.M), dtype=torch.uint8, device=dev)
+    tau = torch.zeros(w.G, **f32)
+    tau_h = torch.zeros(w.G, dtype=torch.float32).pin_memory()
+    e_raw, e_fit = torch.zeros(w.G, **f64), torch.zeros(w.G, **f64)
+    S = torch.zeros((w.N, w.G), **f32)
+    twice = torch.zeros(w.G, dtype=torch.int64, device=dev)
+    pairs = torch.zeros(w.G, dtype=torch.int64, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def fit():
+        _lib.dspark_sts_fit(z, acc, g, w.M, ws, tau, e_raw, e_fit, None, S)
+
+    def auc():
+        _lib.dspark_survival_auc(S, acc, twice, pairs)
+
+    with torch.cuda.stream(stream):
+        fit()
+        auc()
+    torch.cuda.synchronize()
+    g_fit, g_auc = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_fit, stream=stream):
+        fit()
+    with torch.cuda.graph(g_auc, stream=stream):
+        auc()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            g_fit.replay()
+            g_auc.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    fit_ms, auc_ms = [], []
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                flush.zero_()
+                e0.record(stream)
+                g_fit.replay()
+                e1.record(stream)
+                e1.synchronize()
+                fit_ms.append(e0.elapsed_time(e1))
+        torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.steps // 4)):
+            flush.zero_()
+            e0.record(stream)
+            g_auc.replay()
+            e1.record(stream)
+            e1.synchronize()
+            auc_ms.append(e0.elapsed_time(e1))
+        # End to end: the labelled set from pinned host memory, the fit, the
+        # temperatures back to pinned host memory.
+        e2e_ms = []
+        for i in range(max(2, args.steps // 4) + 1):
+            e0.record(stream)
+            z.copy_(z_h, non_blocking=True)
+            acc.copy_(acc_h, non_blocking=True)
+            fit()
+            tau_h.copy_(tau, non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i > 0:
+                e2e_ms.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    status = _lib.dspark_get_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x}")
+    ms, a_ms, e2e = statistics.mean(fit_ms), statistics.mean(auc_ms), statistics.mean(e2e_ms)
+    if world > 1:
+        tt = torch.tensor([ms, a_ms, e2e], device=dev, dtype=torch.float64)
+        gathered = [torch.zeros_like(tt) for _ in range(world)]
+        dist.all_gather(gathered, tt)
+        ms, a_ms, e2e = (max(float(x[j]) for x in gathered) for j in range(3))
+    tw, pr = twice.cpu().numpy(), pairs.cpu().numpy()
+    clocks = clk.summary()
+    mhz = clocks["sm_mhz"] or 1965.0
+    peak_tflops = SMS * FP64_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    prof = profiled_sts_fp64(w.name)
+    roof = {"kernel": f"sts_position ({w.G} launches per fit)", "bound": "alu", "unit": "TFLOP/s",
+            "peak": peak_tflops, "peak_source": f"derived: {SMS} SMs x {FP64_LANES_PER_SM} fp64 lanes x 2 x "
+                                                f"{mhz:.0f} MHz (median SM clock of the timed region)",
+            "achieved": None, "frac": None, "traffic": None, "ms": ms, "launches": w.G}
+    if prof is not None:
+        ach = prof["fp64_flops_per_fit"] / (ms * 1e-3) / 1e12
+        roof.update(achieved=ach, frac=ach / peak_tflops, traffic=prof["dram_bytes_per_fit"],
+                    fp64_flops_per_fit=prof["fp64_flops_per_fit"])
+    line = {
+        "metric": metric, "value": world * evals / (ms * 1e-3), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded calibration sets, one per rank)",
+        "config": {"workload": w.name, "N": w.N, "G": w.G, "K": w.K, "M": w.M,
+                   "l2_flush": "256 MiB write before every timed fit", "graph_replay": True,
+                   "parallelism": f"{world} independent fits"},
+        "fit": {"tau": [float(x) for x in tau.cpu()], "ece_raw": [float(x) for x in e_raw.cpu()],
+                "ece_fit": [float(x) for x in e_fit.cpu()]},
+        "auc": {"ms": a_ms, "pairs_per_s": float(pr.sum()) / (a_ms * 1e-3),
+                "auc_fit": [float(tw[i]) / (2.0 * float(pr[i])) if pr[i] else None for i in range(w.G)]},
+        "roofline": roof,
+        "e2e": {"value": world * evals / (e2e * 1e-3), "unit": unit,
+                "h2d_bytes_per_step": z_h.numel() * 4 + acc_h.numel() * 4, "d2h_bytes_per_step": w.G * 4,
+                "ms_per_step": e2e},
+        "gpu_launches": (w.G + 1) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import calibration as C
+        n, t0 = 0, time.perf_counter()
+        while n == 0 or time.perf_counter() - t0 < 10.0:
+            C.sts_fit(cs.z, cs.acc, grid, w.M)
+            n += 1
+        secs = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n * evals / secs, "unit": unit, "cores": 1, "kind": "oracle",
+                                "sample": f"{n} whole fits, {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line))
+    g_fit.reset()
+    g_auc.reset()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -284,10 +496,13 @@ def main():
     ap.add_argument("--reference-requests", type=int, default=8,
                     help="requests per step of the reference arm (the oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded", "sts"],
                     help="replicas: every rank an independent engine (default); sharded: one engine over all "
-                         "ranks' requests, survivals all-gathered for one global admission")
+                         "ranks' requests, survivals all-gathered for one global admission; sts: the "
+                         "confidence head's sequential temperature scaling fit")
     args = ap.parse_args()
+    if args.mode == "sts":
+        return run_sts(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.mode == "sharded":

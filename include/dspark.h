@@ -80,6 +80,7 @@ typedef enum {
 #define DSPARK_DEV_ELL_RANGE 0x2u    /* an admitted length outside [0, G] was clamped */
 #define DSPARK_DEV_BAD_TEMP 0x4u     /* a temperature < 0 or NaN was treated as 0 */
 #define DSPARK_DEV_TIMEOUT 0x8u      /* a bounded device wait ran out */
+#define DSPARK_DEV_BAD_VALUE 0x10u   /* calibration: a non-finite logit, or a grid entry that is no temperature */
 
 /* Library version and the build's target (a string such as "sm_100a"). */
 const char *dspark_version(void);
@@ -237,6 +238,48 @@ dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const vo
                                           float *rowmax_out, float *rowsum_out, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* ------------------------------------------------------------------------ */
+/* Confidence calibration: sequential temperature scaling (STS).
+ * [PL] §3.2: STS calibrates the cumulative prefix-survival probabilities left
+ * to right, minimising the expected calibration error (ECE) of the running
+ * products of the per-position scores while keeping their ordering.  [KB]
+ * Key Contributions (post-hoc, left to right) and Results (ECE 3-8 % raw,
+ * about 1 % after STS).  The fitted tau is what dspark_confidence takes.
+ *   Labels: y[n,i] = 1 if acc[n] >= i (i = 1..G): the first i draft tokens of
+ *   block n were accepted (acc = the accepted counts of blocks verified at
+ *   full length, e.g. dspark_verify's acc_out under DSPARK_SCHED_ALL).
+ *   Scores: S[n,i] = S[n,i-1] * sigmoid(z[n,i] / tau_i), S[n,0] = 1.
+ *   ECE(s, y) = sum over M equal-width bins of |sum_{n in bin} (y_n - s_n)| / N,
+ *   bin(s) = min(M - 1, floor(s * M)).
+ *   Fit: for i = 1..G in turn (earlier tau fixed), tau_i = the first entry of
+ *   tau_grid with the least ECE(S[:,i], y[:,i]).  A grid entry that is not a
+ *   positive finite number has ECE +inf (and sets DSPARK_DEV_BAD_VALUE).
+ *   All arithmetic in fp64 (scores, bins, sums); the per-bin sums run in a
+ *   fixed order, so the result is deterministic.
+ * Inputs:  z [N,G] f32 head logits (w . h + bias, before any temperature),
+ *          acc [N] int32 in [0, G] (others: DSPARK_DEV_ELL_RANGE, labels as
+ *          defined), tau_grid [K] f32, n_bins M.
+ * Outputs: tau_out [G] f32; ece_raw_out [G] f64 (tau = 1), ece_fit_out [G]
+ *          f64, ece_all_out [G,K] f64 (every candidate), S_out [N,G] f32 (the
+ *          fitted survivals rounded to fp32); the last four may be NULL.
+ * Limits:  1 <= N <= 2^24, 1 <= G <= 16, 1 <= K <= 4096, 1 <= M <= 32.
+ * Enqueues a 4-byte memset and G kernel launches. */
+size_t dspark_sts_workspace_size(int N, int G, int K, int n_bins);
+dspark_status dspark_sts_fit(const float *z, const int32_t *acc, const float *tau_grid, int N, int G, int K,
+                             int n_bins, void *ws, size_t ws_bytes, float *tau_out, double *ece_raw_out,
+                             double *ece_fit_out, double *ece_all_out, float *S_out, void *stream);
+
+/* ROC-AUC of the prefix survivals against the same labels ([KB] Results
+ * reports the raw confidence's ROC-AUC): for each position i, over every pair
+ * of a positive (acc[p] >= i) and a negative sample, 2 when the positive's
+ * S is larger, 1 on a tie, 0 otherwise (NaN scores compare false).
+ * Inputs:  S [N,G] f32, acc [N] int32.
+ * Outputs: twice_out [G] uint64 = the pair total; pairs_out [G] uint64 =
+ *          positives * negatives; AUC_i = twice_out[i] / (2 * pairs_out[i]).
+ *          Exact integers.  Needs no workspace; limits as dspark_sts_fit. */
+dspark_status dspark_survival_auc(const float *S, const int32_t *acc, int N, int G, uint64_t *twice_out,
+                                  uint64_t *pairs_out, void *stream);
+
 /* Device status word of a workspace: dspark_get_device_status synchronises
  * `stream`, then copies the word to *status_out (0 = no data error since the
  * last clear).  dspark_clear_device_status enqueues a reset of the word. */

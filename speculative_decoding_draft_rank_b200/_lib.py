@@ -24,12 +24,13 @@ SCHED_GLOBAL_ARGMAX = 2
 SCHED_THRESHOLD = 3
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DTYPE", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
-DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT, DEV_BAD_VALUE = 0x1, 0x2, 0x4, 0x8, 0x10
 
 EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov", "dspark_confidence",
            "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
            "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
-           "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold")
+           "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold",
+           "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc")
 
 
 class DsparkError(RuntimeError):
@@ -76,6 +77,12 @@ def load() -> ctypes.CDLL:
     lib.dspark_draft_noalloc_max_scratch.argtypes = []
     lib.dspark_draft_markov_noalloc.restype = _i
     lib.dspark_draft_markov_noalloc.argtypes = [_vp] * 6 + [_i] * 5 + [_vp] * 5
+    lib.dspark_sts_workspace_size.restype = _sz
+    lib.dspark_sts_workspace_size.argtypes = [_i] * 4
+    lib.dspark_sts_fit.restype = _i
+    lib.dspark_sts_fit.argtypes = [_vp] * 3 + [_i] * 4 + [_vp, _sz] + [_vp] * 6
+    lib.dspark_survival_auc.restype = _i
+    lib.dspark_survival_auc.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp]
     _lib = lib
     return lib
 
@@ -176,6 +183,29 @@ def dspark_verify(Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u
           _ptr(rowmax), _ptr(rowsum), _ptr(temp), _ptr(u_accept), _ptr(u_final), _ptr(ell), B, G1 - 1, V, r,
           _dtype(Tlog), _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out), _ptr(tokens_out),
           _ptr(nout_out), _ptr(pt_x_out), _stream(stream))
+
+
+def dspark_sts_workspace_size(N, G, K, n_bins) -> int:
+    return int(load().dspark_sts_workspace_size(N, G, K, n_bins))
+
+
+def dspark_sts_fit(z, acc, tau_grid, n_bins, ws, tau_out, ece_raw_out=None, ece_fit_out=None, ece_all_out=None,
+                   S_out=None, stream=None):
+    """Sequential temperature scaling: z [N, G] f32 logits, acc [N] int32,
+    tau_grid [K] f32 candidates -> tau_out [G] f32 (and the optional ECEs,
+    fp64, and fitted survivals S_out [N, G] f32)."""
+    N, G = z.shape
+    K = tau_grid.shape[0]
+    _call("dspark_sts_fit", _ptr(z), _ptr(acc), _ptr(tau_grid), N, G, K, int(n_bins), _ptr(ws),
+          ws.numel() * ws.element_size(), _ptr(tau_out), _ptr(ece_raw_out), _ptr(ece_fit_out), _ptr(ece_all_out),
+          _ptr(S_out), _stream(stream))
+
+
+def dspark_survival_auc(S, acc, twice_out, pairs_out, stream=None):
+    """ROC-AUC pair counts per position: twice_out, pairs_out [G] int64
+    tensors (uint64 bit patterns); AUC = twice / (2 * pairs)."""
+    N, G = S.shape
+    _call("dspark_survival_auc", _ptr(S), _ptr(acc), N, G, _ptr(twice_out), _ptr(pairs_out), _stream(stream))
 
 
 def dspark_get_device_status(ws, stream=None) -> int:

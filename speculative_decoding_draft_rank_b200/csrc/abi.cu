@@ -3,6 +3,7 @@
 // allocates memory or synchronises, except dspark_get_device_status.
 #include <cstring>
 
+#include "calibration.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -41,6 +42,10 @@ dspark_status injected(const char *name) {
 }
 
 dspark_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+bool sts_sizes_ok(int N, int G, int K, int M) {
+    return N >= 1 && N <= (1 << 24) && G >= 1 && G <= 16 && K >= 1 && K <= 4096 && M >= 1 && M <= kStsMaxBins;
+}
 
 }  // namespace
 
@@ -108,6 +113,31 @@ dspark_status dspark_schedule_threshold(const float *S, int B, int G, float thre
     if (dspark_status s = check_ws(ws, ws_bytes, schedule_ws_bytes(B, G))) return s;
     return cuda_status(launch_schedule(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_THRESHOLD, threshold, ws,
                                        ell_out, n_adm_out, nullptr, order_out, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dspark_sts_workspace_size(int N, int G, int K, int n_bins) {
+    if (!sts_sizes_ok(N, G, K, n_bins)) return 0;
+    return sts_ws_bytes(N, K, n_bins);
+}
+
+dspark_status dspark_sts_fit(const float *z, const int32_t *acc, const float *tau_grid, int N, int G, int K,
+                             int n_bins, void *ws, size_t ws_bytes, float *tau_out, double *ece_raw_out,
+                             double *ece_fit_out, double *ece_all_out, float *S_out, void *stream) {
+    if (dspark_status s = injected("dspark_sts_fit")) return s;
+    if (!sts_sizes_ok(N, G, K, n_bins) || !z || !acc || !tau_grid || !tau_out) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, sts_ws_bytes(N, K, n_bins))) return s;
+    StsArgs a{z, acc, tau_grid, N, G, K, n_bins, tau_out, ece_raw_out, ece_fit_out, ece_all_out, S_out};
+    return cuda_status(launch_sts_fit(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_survival_auc(const float *S, const int32_t *acc, int N, int G, uint64_t *twice_out,
+                                  uint64_t *pairs_out, void *stream) {
+    if (dspark_status s = injected("dspark_survival_auc")) return s;
+    if (N < 1 || N > (1 << 24) || G < 1 || G > 16 || !S || !acc || !twice_out || !pairs_out)
+        return DSPARK_ERR_INVALID_ARG;
+    return cuda_status(launch_survival_auc(S, acc, N, G, reinterpret_cast<unsigned long long *>(twice_out),
+                                           reinterpret_cast<unsigned long long *>(pairs_out),
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 size_t dspark_verify_workspace_size(int B, int G, int V, int r, int dtype) {

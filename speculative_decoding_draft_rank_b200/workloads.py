@@ -91,3 +91,30 @@ def long_block(G: int) -> Workload:
 
 def all_workloads():
     return [tiny(), qwen_vocab(), headline(), saturated()] + [long_block(g) for g in (4, 8, 12, 16)]
+
+
+@dataclass
+class CalibrationWorkload:
+    """A sequential-temperature-scaling fit: N verified blocks of G positions,
+    K candidate temperatures, M ECE bins; the head's logits are k times the
+    latent ones (an over-confident head when k > 1)."""
+    name: str
+    N: int
+    G: int
+    K: int
+    M: int
+    k: float = 2.0
+    seed: int = 0
+
+    def inputs(self) -> synth.CalibrationSet:
+        return synth.calibration_set(self.N, self.G, k=self.k, seed=self.seed)
+
+    def grid(self) -> np.ndarray:
+        return synth.tau_grid(self.K)
+
+
+def calibration_headline() -> CalibrationWorkload:
+    """64 rounds of the headline batch (256 requests) verified at full length
+    G = 5: N = 16384 labelled blocks; 65 log-spaced temperatures in [1/4, 4];
+    15 bins."""
+    return CalibrationWorkload("sts_n16384_g5_k65_m15", 16384, 5, 65, 15)

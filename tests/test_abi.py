@@ -139,3 +139,30 @@ def test_injected_failure(lib, monkeypatch):
         _lib._call("dspark_schedule", FAKE, 4, 5, FAKE, FAKE, 2, -1, 1, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE,
                    None, None)
     assert ei.value.status == 5
+
+
+def test_calibration_argument_checks(lib):
+    assert lib.dspark_sts_workspace_size(16384, 5, 65, 15) > 0
+    assert lib.dspark_sts_workspace_size(0, 5, 65, 15) == 0
+    assert lib.dspark_sts_workspace_size(16, 17, 65, 15) == 0
+    assert lib.dspark_sts_workspace_size(16, 5, 4097, 15) == 0
+    assert lib.dspark_sts_workspace_size(16, 5, 65, 33) == 0
+    assert lib.dspark_sts_workspace_size(16, 5, 65, 0) == 0
+
+    def fit(N=64, G=5, K=9, M=15, ws=FAKE_WS, ws_bytes=1 << 20, null=None):
+        args = [FAKE, FAKE, FAKE]
+        if null is not None and null < 3:
+            args[null] = None
+        return lib.dspark_sts_fit(*args, N, G, K, M, ws, ws_bytes, FAKE if null != 3 else None, None, None, None,
+                                  None, None)
+
+    assert fit(N=0) == 1 and fit(G=0) == 1 and fit(G=17) == 1 and fit(K=0) == 1 and fit(M=33) == 1
+    for k in range(4):
+        assert fit(null=k) == 1
+    assert fit(ws=None) == 3
+    assert fit(ws=ctypes.c_void_p(0x200010)) == 3
+    assert fit(ws_bytes=256) == 3
+    assert lib.dspark_survival_auc(FAKE, FAKE, 0, 5, FAKE, FAKE, None) == 1
+    assert lib.dspark_survival_auc(FAKE, FAKE, 16, 17, FAKE, FAKE, None) == 1
+    assert lib.dspark_survival_auc(None, FAKE, 16, 5, FAKE, FAKE, None) == 1
+    assert lib.dspark_survival_auc(FAKE, FAKE, 16, 5, None, FAKE, None) == 1

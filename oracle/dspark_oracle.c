@@ -364,6 +364,40 @@ int dspark_oracle_schedule_threshold(int B, int G, const double *S, double thres
     return ORACLE_OK;
 }
 
+/* Dynamic top-K admission, the production scheduler's selection step ([PL]
+ * §5.2 Production Scheduler: asynchronous; the capacity limit comes from
+ * historical predictions, the current candidates are ranked by their latest
+ * cumulative confidence, and a dynamic top-K selection keeps the confidence
+ * ordering).  In the same sorted order as above, admit the first K candidates,
+ * K = capacity clamped to [0, B*G], at most `budget` (budget < 0: none).  The
+ * capacity itself is an input: the production form computes it from an
+ * earlier round (the global search over the profile on that round's
+ * survivals), so the count does not look at the current round at all.
+ * Outputs ell [B], n_adm, order [B*G]. */
+int dspark_oracle_schedule_topk(int B, int G, const double *S, int capacity, int budget, int *ell_out,
+                                int *n_adm_out, int *order_out)
+{
+    if (B < 1 || G < 1) return ORACLE_ERR_ARG;
+    int N = B * G;
+    cand_t *c = malloc(sizeof(cand_t) * (size_t)N);
+    if (!c) return ORACLE_ERR_NOMEM;
+    for (int i = 0; i < G; ++i)
+        for (int b = 0; b < B; ++b) {
+            c[i * B + b].s = S[(size_t)b * G + i];
+            c[i * B + b].idx = i * B + b;
+        }
+    qsort(c, (size_t)N, sizeof(cand_t), cand_cmp);
+    if (order_out)
+        for (int n = 0; n < N; ++n) order_out[n] = c[n].idx;
+    int n = capacity < 0 ? 0 : (capacity > N ? N : capacity);
+    if (budget >= 0 && budget < n) n = budget;
+    for (int b = 0; b < B; ++b) ell_out[b] = 0;
+    for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;
+    *n_adm_out = n;
+    free(c);
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Stage 4, exact rejection-sampling verification: [KB] Methodology (x_k is
  * accepted with probability min(1, p_t(x_k)/p_d(x_k)); the first rejection

@@ -156,6 +156,30 @@ def schedule_threshold(S, threshold, budget=-1):
     return ell, n_adm.value, order
 
 
+def schedule_topk(S, capacity, budget=-1):
+    """Dynamic top-K admission over survivals S [B,G]: the first `capacity`
+    candidates of the stable order (clamped to [0, B*G]), at most `budget`.
+    Returns (ell [B], n_adm, order)."""
+    S = _f64(S)
+    B, G = S.shape
+    ell = np.zeros(B, np.int32); order = np.zeros(B * G, np.int32)
+    n_adm = ctypes.c_int(0)
+    rc = _load().dspark_oracle_schedule_topk(B, G, _p(S), int(capacity), int(budget), _p(ell),
+                                             ctypes.byref(n_adm), _p(order))
+    _check(rc, "schedule_topk")
+    return ell, n_adm.value, order
+
+
+def production_schedule(S_prev, S_cur, knots_n, knots_t, budget=-1):
+    """The production scheduler's two steps for one round: the capacity from
+    the previous round's survivals (the global search of Theta over the
+    profile, which copes with non-smooth capacity curves), then the top-K of
+    the current round's candidates.  Returns (capacity, ell, n_adm, order)."""
+    cap = schedule(S_prev, knots_n, knots_t, budget, SCHED_GLOBAL_ARGMAX).n_adm
+    ell, n_adm, order = schedule_topk(S_cur, cap, budget)
+    return cap, ell, n_adm, order
+
+
 @dataclass
 class VerifyResult:
     acc: np.ndarray          # [B] accepted count A

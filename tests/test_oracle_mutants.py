@@ -70,3 +70,39 @@ def test_mutant_is_caught(tmp_path, name, old, new):
         assert _preservation_probe() > 1e-6
     finally:
         oracle.use_library(oracle.build())
+
+
+# Planted mistakes in the scheduler variants, caught by the scheduler pins.
+SCHED_MUTANTS = [
+    ("topk_counts_from_one", "int n = capacity < 0 ? 0 : (capacity > N ? N : capacity);",
+     "int n = capacity < 1 ? 0 : (capacity > N ? N : capacity - 1);"),
+    ("topk_ignores_budget", "    if (budget >= 0 && budget < n) n = budget;\n    for (int b = 0; b < B; ++b) ell_out[b] = 0;\n"
+     "    for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;\n    *n_adm_out = n;\n    free(c);\n"
+     "    return ORACLE_OK;\n}\n\n/* ----",
+     "    for (int b = 0; b < B; ++b) ell_out[b] = 0;\n"
+     "    for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;\n    *n_adm_out = n;\n    free(c);\n"
+     "    return ORACLE_OK;\n}\n\n/* ----"),
+    ("topk_request_index", "for (int k = 0; k < n; ++k) ell_out[c[k].idx % B] += 1;\n    *n_adm_out = n;\n    free(c);\n"
+     "    return ORACLE_OK;\n}\n\n/* ----",
+     "for (int k = 0; k < n; ++k) ell_out[c[k].idx / G % B] += 1;\n    *n_adm_out = n;\n    free(c);\n"
+     "    return ORACLE_OK;\n}\n\n/* ----"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", SCHED_MUTANTS, ids=[m[0] for m in SCHED_MUTANTS])
+def test_scheduler_mutant_is_caught(tmp_path, name, old, new):
+    import test_oracle_pins as pins
+    so = _build_mutant(tmp_path, name, old, new)
+    caught = False
+    try:
+        oracle.use_library(so)
+        for pin in (pins.test_scheduler_topk_is_the_first_k_of_the_stable_order,
+                    pins.test_scheduler_topk_with_the_greedy_count_is_the_greedy_schedule):
+            try:
+                pin()
+            except AssertionError:
+                caught = True
+    finally:
+        oracle.use_library(oracle.build())
+    assert caught, f"no scheduler pin catches {name}"
+

@@ -342,6 +342,61 @@ def test_scheduler_threshold_is_the_survival_cut():
                 assert all(S[b, k] < th for k in range(ell[b], G))
 
 
+def test_scheduler_topk_is_the_first_k_of_the_stable_order():
+    """Dynamic top-K admits the first K candidates of the stable order by S
+    descending (Python's sort as the reference), clamped to [0, B*G] and to the
+    budget; with monotone survivals every request's admitted set is a prefix."""
+    rng = _rng(13)
+    for trial in range(80):
+        B, G = int(rng.integers(1, 6)), int(rng.integers(1, 6))
+        c = rng.choice([1.0, 0.9, 0.5, 0.25], size=(B, G))
+        S = np.cumprod(c, axis=1)
+        cap = int(rng.integers(-2, B * G + 3))
+        budget = -1 if trial % 4 else int(rng.integers(0, B * G + 1))
+        ell, n_adm, order = oracle.schedule_topk(S, cap, budget)
+        ids = sorted(range(B * G), key=lambda i: (-S[i % B, i // B], i))
+        assert list(order) == ids
+        k = min(max(cap, 0), B * G)
+        if budget >= 0:
+            k = min(k, budget)
+        take = ids[:k]
+        assert n_adm == k
+        for b in range(B):
+            assert ell[b] == sum(1 for i in take if i % B == b)
+            admitted = {i // B for i in take if i % B == b}
+            assert admitted == set(range(ell[b]))              # a prefix of the request
+
+
+def test_scheduler_topk_with_the_greedy_count_is_the_greedy_schedule():
+    """With K equal to Algorithm 1's admitted count on the same survivals, the
+    top-K selection admits exactly Algorithm 1's set (both are prefixes of the
+    same stable order), and with the global search's count, that search's set."""
+    rng = _rng(14)
+    for trial in range(40):
+        B, G = int(rng.integers(1, 9)), int(rng.integers(1, 6))
+        S = _monotone_S(rng, B, G)
+        kn, kt = _convex_profile(rng)
+        for mode in (oracle.SCHED_GREEDY_EARLY_STOP, oracle.SCHED_GLOBAL_ARGMAX):
+            res = oracle.schedule(S, kn, kt, -1, mode)
+            ell, n_adm, order = oracle.schedule_topk(S, res.n_adm)
+            assert n_adm == res.n_adm and np.array_equal(ell, res.ell) and np.array_equal(order, res.order)
+
+
+def test_production_schedule_takes_its_capacity_from_the_previous_round():
+    """The production form's admitted count depends on the previous round
+    only: changing the current round's survivals changes which candidates are
+    admitted, never how many."""
+    rng = _rng(15)
+    kn, kt = np.array([0, 4, 8], np.int32), np.array([10.0, 10.5, 30.0])   # a step in capacity
+    for trial in range(30):
+        B, G = int(rng.integers(2, 7)), int(rng.integers(1, 5))
+        S_prev = _monotone_S(rng, B, G)
+        cap, _, n1, _ = oracle.production_schedule(S_prev, _monotone_S(rng, B, G), kn, kt)
+        _, _, n2, _ = oracle.production_schedule(S_prev, _monotone_S(rng, B, G), kn, kt)
+        assert n1 == n2 == min(cap, B * G)
+        assert cap == oracle.schedule(S_prev, kn, kt, -1, oracle.SCHED_GLOBAL_ARGMAX).n_adm
+
+
 # --------------------------------------------------------------------------
 # Verification
 # --------------------------------------------------------------------------

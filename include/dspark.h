@@ -72,7 +72,8 @@ typedef enum {
     DSPARK_SCHED_ALL = 0,               /* verify every drafted position */
     DSPARK_SCHED_GREEDY_EARLY_STOP = 1, /* Algorithm 1 */
     DSPARK_SCHED_GLOBAL_ARGMAX = 2,     /* variant: offline search, no early stop */
-    DSPARK_SCHED_THRESHOLD = 3          /* variant: static survival threshold (dspark_schedule_threshold) */
+    DSPARK_SCHED_THRESHOLD = 3,         /* variant: static survival threshold (dspark_schedule_threshold) */
+    DSPARK_SCHED_TOPK = 4               /* variant: dynamic top-K of the production scheduler (dspark_schedule_topk) */
 } dspark_sched_mode;
 
 /* Bits of the device status word. */
@@ -173,6 +174,28 @@ dspark_status dspark_schedule(const float *S, int B, int G, const int32_t *knots
 dspark_status dspark_schedule_threshold(const float *S, int B, int G, float threshold, int budget, void *ws,
                                         size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out,
                                         int32_t *order_out, void *stream);
+
+/* Scheduler variant: the production scheduler's dynamic top-K.  [PL] §5.2
+ * Production Scheduler: the scheduler runs asynchronously; the capacity limit
+ * comes from historical predictions and the current candidates are ranked by
+ * their latest cumulative confidence; the top-K selection keeps the
+ * confidence ordering and hides the scheduling latency, and the capacity's
+ * global search copes with irregular hardware-capacity curves.  This call is
+ * the selection: it admits the first K candidates of the same stable order as
+ * dspark_schedule, K = *capacity clamped to [0, B*G], at most `budget` (< 0:
+ * none).  `capacity` is a DEVICE int32, typically the n_adm_out of a
+ * dspark_schedule call in mode DSPARK_SCHED_GLOBAL_ARGMAX on the previous
+ * round's survivals, enqueued on another stream while this round drafts; the
+ * count is read when the kernel runs, so one captured graph serves every
+ * capacity.  A negative capacity admits none and sets DSPARK_DEV_ELL_RANGE in
+ * the workspace's status word.
+ * Inputs:  S [B,G] f32, capacity [1] int32 (device), budget; limits and
+ *          workspace as dspark_schedule.
+ * Outputs: ell_out [B] int32, n_adm_out [1] int32, order_out [B*G] int32 or
+ *          NULL. */
+dspark_status dspark_schedule_topk(const float *S, int B, int G, const int32_t *capacity, int budget, void *ws,
+                                   size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out, int32_t *order_out,
+                                   void *stream);
 
 /* ------------------------------------------------------------------------ */
 /* Stage 4: exact rejection-sampling verification.

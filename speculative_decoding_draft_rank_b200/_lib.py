@@ -22,6 +22,7 @@ SCHED_ALL = 0
 SCHED_GREEDY_EARLY_STOP = 1
 SCHED_GLOBAL_ARGMAX = 2
 SCHED_THRESHOLD = 3
+SCHED_TOPK = 4
 
 STATUS = {0: "OK", 1: "INVALID_ARG", 2: "UNSUPPORTED_DTYPE", 3: "WORKSPACE", 4: "CUDA", 5: "TIMEOUT"}
 DEV_TOKEN_RANGE, DEV_ELL_RANGE, DEV_BAD_TEMP, DEV_TIMEOUT, DEV_BAD_VALUE = 0x1, 0x2, 0x4, 0x8, 0x10
@@ -30,7 +31,7 @@ EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov
            "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
            "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
            "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold",
-           "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc")
+           "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc", "dspark_schedule_topk")
 
 
 class DsparkError(RuntimeError):
@@ -77,6 +78,8 @@ def load() -> ctypes.CDLL:
     lib.dspark_draft_noalloc_max_scratch.argtypes = []
     lib.dspark_draft_markov_noalloc.restype = _i
     lib.dspark_draft_markov_noalloc.argtypes = [_vp] * 6 + [_i] * 5 + [_vp] * 5
+    lib.dspark_schedule_topk.restype = _i
+    lib.dspark_schedule_topk.argtypes = [_vp, _i, _i, _vp, _i, _vp, _sz, _vp, _vp, _vp, _vp]
     lib.dspark_sts_workspace_size.restype = _sz
     lib.dspark_sts_workspace_size.argtypes = [_i] * 4
     lib.dspark_sts_fit.restype = _i
@@ -172,6 +175,14 @@ def dspark_schedule_threshold(S, threshold, budget, ws, ell_out, n_adm_out, orde
     """Static-threshold pruning: the sorted candidates with S >= threshold."""
     B, G = S.shape
     _call("dspark_schedule_threshold", _ptr(S), B, G, ctypes.c_float(threshold), int(budget), _ptr(ws),
+          ws.numel() * ws.element_size(), _ptr(ell_out), _ptr(n_adm_out), _ptr(order_out), _stream(stream))
+
+
+def dspark_schedule_topk(S, capacity, budget, ws, ell_out, n_adm_out, order_out=None, stream=None):
+    """Dynamic top-K: the first *capacity (a device int32) candidates of the
+    stable order by S."""
+    B, G = S.shape
+    _call("dspark_schedule_topk", _ptr(S), B, G, _ptr(capacity), int(budget), _ptr(ws),
           ws.numel() * ws.element_size(), _ptr(ell_out), _ptr(n_adm_out), _ptr(order_out), _stream(stream))
 
 

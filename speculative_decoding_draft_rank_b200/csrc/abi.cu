@@ -6,6 +6,7 @@
 #include "calibration.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
+#include "schedule_variants.cuh"
 
 using namespace dspark;
 
@@ -138,6 +139,17 @@ dspark_status dspark_survival_auc(const float *S, const int32_t *acc, int N, int
     return cuda_status(launch_survival_auc(S, acc, N, G, reinterpret_cast<unsigned long long *>(twice_out),
                                            reinterpret_cast<unsigned long long *>(pairs_out),
                                            static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_schedule_topk(const float *S, int B, int G, const int32_t *capacity, int budget, void *ws,
+                                   size_t ws_bytes, int32_t *ell_out, int32_t *n_adm_out, int32_t *order_out,
+                                   void *stream) {
+    if (dspark_status s = injected("dspark_schedule_topk")) return s;
+    if (B < 1 || B > 4096 || G < 1 || G > 16 || B * G > 16384) return DSPARK_ERR_INVALID_ARG;
+    if (!S || !capacity || !ell_out || !n_adm_out) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, schedule_ws_bytes(B, G))) return s;
+    return cuda_status(launch_schedule_topk(S, B, G, capacity, budget, ws, ell_out, n_adm_out, order_out,
+                                            static_cast<cudaStream_t>(stream)));
 }
 
 size_t dspark_verify_workspace_size(int B, int G, int V, int r, int dtype) {

@@ -24,9 +24,16 @@
 // Theta(n) = V_n / t(n) over every n up to the budget (lowest n on ties) --
 // no early stop, so not lossless when confidence depends on drawn tokens --
 // and static-threshold pruning admits the sorted candidates with
-// S >= threshold, up to the budget.
+// S >= threshold, up to the budget.  The production scheduler's dynamic
+// top-K (paperlayer.ai summary, §5.2 Production Scheduler: the capacity limit
+// comes from historical predictions, the current candidates are ranked by
+// their latest cumulative confidence) admits the first K of the sorted
+// candidates, K read from device memory -- written there by an earlier
+// schedule call on an earlier round -- so one captured graph serves every
+// capacity.
 #include "common.cuh"
 #include "kernels.cuh"
+#include "schedule_variants.cuh"
 
 namespace dspark {
 
@@ -66,6 +73,7 @@ __device__ __forceinline__ void bitonic_warp_step(unsigned long long &v0, unsign
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
     const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
+    const int32_t *__restrict__ capacity, WsHeader *hdr,
     int32_t *__restrict__ ell_out, int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
     int32_t *__restrict__ order_out)
 {
@@ -192,6 +200,15 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
         for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
             if (arg_v[w] > best || (arg_v[w] == best && arg_n[w] < bestn)) { best = arg_v[w]; bestn = arg_n[w]; }
         nadm = bestn;
+    } else if (mode == DSPARK_SCHED_TOPK) {
+        // The first K of the stable order; a negative capacity admits none
+        // and is recorded.
+        int kcap = *capacity;
+        if (kcap < 0) {
+            if (tid == 0) flag_status(hdr, DSPARK_DEV_ELL_RANGE);
+            kcap = 0;
+        }
+        nadm = kcap < limit ? kcap : limit;
     } else if (mode == DSPARK_SCHED_THRESHOLD) {
         // The sorted survivals fall below the threshold at one index.
         int first_below = 0x7fffffff;
@@ -247,7 +264,19 @@ cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n
                                          (int)smem);
     if (e != cudaSuccess) return e;
     schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, threshold,
-                                                    ell_out, n_adm_out, theta_out, order_out);
+                                                    nullptr, nullptr, ell_out, n_adm_out, theta_out, order_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_schedule_topk(const float *S, int B, int G, const int32_t *capacity, int budget, void *ws,
+                                 int32_t *ell_out, int32_t *n_adm_out, int32_t *order_out, cudaStream_t st) {
+    const size_t smem = sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096;
+    cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_TOPK, 0.f,
+                                                    capacity, static_cast<WsHeader *>(ws), ell_out, n_adm_out,
+                                                    nullptr, order_out);
     return cudaGetLastError();
 }
 

@@ -166,3 +166,16 @@ def test_calibration_argument_checks(lib):
     assert lib.dspark_survival_auc(FAKE, FAKE, 16, 17, FAKE, FAKE, None) == 1
     assert lib.dspark_survival_auc(None, FAKE, 16, 5, FAKE, FAKE, None) == 1
     assert lib.dspark_survival_auc(FAKE, FAKE, 16, 5, None, FAKE, None) == 1
+
+
+def test_schedule_topk_argument_checks(lib):
+    def topk(B=8, G=5, cap=FAKE, ws=FAKE_WS, ws_bytes=1 << 20, S=FAKE, ell=FAKE, nadm=FAKE):
+        return lib.dspark_schedule_topk(S, B, G, cap, -1, ws, ws_bytes, ell, nadm, None, None)
+
+    assert topk(B=0) == 1 and topk(G=17) == 1 and topk(B=4096, G=8) == 1
+    assert topk(cap=None) == 1 and topk(S=None) == 1 and topk(ell=None) == 1 and topk(nadm=None) == 1
+    assert topk(ws=None) == 3 and topk(ws=ctypes.c_void_p(0x200010)) == 3 and topk(ws_bytes=8) == 3
+    # mode 4 needs its capacity: the plain scheduler entry rejects it.
+    assert lib.dspark_schedule(FAKE, 8, 5, FAKE, FAKE, 2, -1, 4, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None,
+                               None) == 1
+

@@ -60,6 +60,48 @@ static void markov_bias_row(const float *U, const float *W, int V, int r, int a,
     }
 }
 
+/* Bias of draft position k (1-based) of one request, given its prefix
+ * x_0 (last committed token) and xs[0..k-2] = x_1..x_{k-1}: [PL] §3.1 (the
+ * sequential stage conditions each position on the tokens sampled before it;
+ * a Markov head uses a low-rank transition matrix, an RNN head keeps a
+ * recurrent state that summarises the whole prefix); [KB] Key Contributions
+ * (Markov head: first-order dependency by a low-rank factorization; RNN head:
+ * full within-block history).
+ *   A == NULL (Markov head): Delta = U[x_{k-1}] W.
+ *   A != NULL (RNN head, A stored [r][r]): the state h_0 = 0 and
+ *     h_j[c] = tanh(sum_q h_{j-1}[q] A[q][c] + U[x_{j-1}][c]), j = 1..k;
+ *     Delta = h_k W.  The pages give no equations for this head; this is
+ *     the plainest recurrence over the same factors (a state of size r fed
+ *     by the token's U row, read out through W).
+ * h and hn are scratch rows of r doubles.  The state is recomputed from the
+ * start of the block at every call (slow, and the same arithmetic wherever
+ * the bias is needed). */
+static void draft_bias(const float *U, const float *A, const float *W, int V, int r, int x0,
+                       const int *xs, int k, double *h, double *hn, double *delta)
+{
+    if (A == NULL) {
+        markov_bias_row(U, W, V, r, k == 1 ? x0 : xs[k - 2], delta);
+        return;
+    }
+    for (int c = 0; c < r; ++c) h[c] = 0.0;
+    for (int j = 1; j <= k; ++j) {
+        int tok = (j == 1) ? x0 : xs[j - 2];
+        for (int c = 0; c < r; ++c) {
+            double a = 0.0;
+            for (int q = 0; q < r; ++q) a += h[q] * (double)A[(size_t)q * r + c];
+            a += (double)U[(size_t)tok * r + c];
+            hn[c] = tanh(a);
+        }
+        for (int c = 0; c < r; ++c) h[c] = hn[c];
+    }
+    for (int v = 0; v < V; ++v) delta[v] = 0.0;
+    for (int c = 0; c < r; ++c) {
+        double hc = h[c];
+        const float *wc = W + (size_t)c * V;
+        for (int v = 0; v < V; ++v) delta[v] += hc * (double)wc[v];
+    }
+}
+
 /* Index of the largest entry (lowest index on ties) and the gap to the
  * largest entry at any other index (the decision margin of an argmax). */
 static int argmax_with_gap(const double *z, int V, double *gap)
@@ -121,7 +163,8 @@ static double softmax_row(const double *row, int V, double T, double *e, double 
  * conditioning each position on the previously sampled token); [WK]
  * draft-generation figure (L[i] + Delta[i], then sample the draft token).
  *
- * L [B][G][V], U [V][r], W [r][V]; x0 [B] last committed token per request;
+ * L [B][G][V], U [V][r], W [r][V], A [r][r] or NULL (see draft_bias: NULL is
+ * the Markov head, else the RNN head); x0 [B] last committed token per request;
  * temp [B]; u_draft [B][G] uniforms in [0,1).  force_x (nullable, [B][G]):
  * entries >= 0 replace the sampled token (used to follow another
  * implementation's decision after a reported near-tie).
@@ -129,24 +172,24 @@ static double softmax_row(const double *row, int V, double T, double *e, double 
  * rowmax = max_v y_v (logit units, before the temperature), rowsum =
  * sum_v exp(z_v - max z), margin = decision margin.  For T = 0: x = argmax y,
  * pd = 1, rowmax = max y, rowsum = 1, margin = top-two gap. */
-int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float *U,
-                        const float *W, const int *x0, const float *temp,
-                        const double *u_draft, const int *force_x, int *x_out,
-                        double *pd_out, double *rowmax_out, double *rowsum_out,
-                        double *margin_out)
+int dspark_oracle_draft_head(int B, int G, int V, int r, const float *L, const float *U,
+                             const float *A, const float *W, const int *x0, const float *temp,
+                             const double *u_draft, const int *force_x, int *x_out,
+                             double *pd_out, double *rowmax_out, double *rowsum_out,
+                             double *margin_out)
 {
     if (B < 0 || G < 1 || V < 2 || r < 1) return ORACLE_ERR_ARG;
     double *delta = malloc(sizeof(double) * (size_t)V);
     double *y = malloc(sizeof(double) * (size_t)V);
     double *e = malloc(sizeof(double) * (size_t)V);
-    if (!delta || !y || !e) { free(delta); free(y); free(e); return ORACLE_ERR_NOMEM; }
+    double *h = malloc(sizeof(double) * (size_t)r * 2);
+    if (!delta || !y || !e || !h) { free(delta); free(y); free(e); free(h); return ORACLE_ERR_NOMEM; }
     for (int b = 0; b < B; ++b) {
-        int prev = x0[b];
-        if (prev < 0 || prev >= V) { free(delta); free(y); free(e); return ORACLE_ERR_ARG; }
+        if (x0[b] < 0 || x0[b] >= V) { free(delta); free(y); free(e); free(h); return ORACLE_ERR_ARG; }
         double T = (double)temp[b];
         for (int i = 0; i < G; ++i) {
             size_t o = (size_t)b * G + i;
-            markov_bias_row(U, W, V, r, prev, delta);
+            draft_bias(U, A, W, V, r, x0[b], x_out + (size_t)b * G, i + 1, h, h + r, delta);
             const float *Lrow = L + o * (size_t)V;
             for (int v = 0; v < V; ++v) y[v] = (double)Lrow[v] + delta[v];
             int x;
@@ -171,11 +214,21 @@ int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float 
                 pd_out[o] = e[x] / Z;
             }
             x_out[o] = x;
-            prev = x;
         }
     }
-    free(delta); free(y); free(e);
+    free(delta); free(y); free(e); free(h);
     return ORACLE_OK;
+}
+
+/* The Markov-head drafting of [PL] §3.1 (the head of the headline path). */
+int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float *U,
+                        const float *W, const int *x0, const float *temp,
+                        const double *u_draft, const int *force_x, int *x_out,
+                        double *pd_out, double *rowmax_out, double *rowsum_out,
+                        double *margin_out)
+{
+    return dspark_oracle_draft_head(B, G, V, r, L, U, NULL, W, x0, temp, u_draft, force_x, x_out, pd_out,
+                                    rowmax_out, rowsum_out, margin_out);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -420,16 +473,18 @@ int dspark_oracle_schedule_topk(int B, int G, const double *S, int capacity, int
  * margin_acc [B][G] (|u - ratio|, or the top-two gap for T = 0; +inf beyond
  * ell), margin_fin [B], final_kind [B]: 0 residual, 1 bonus/fresh token,
  * 2 greedy, 3 residual that was all zero (drawn from p_t). */
-int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const float *L,
-                         const float *U, const float *W, const int *x0, const int *x,
-                         const float *temp, const double *u_accept,
-                         const double *u_final, const int *ell,
-                         const int *force_accept, int *acc_out, int *tokens_out,
-                         int *nout_out, double *pt_x_out, double *pd_x_out,
-                         double *margin_acc_out, double *margin_fin_out,
-                         int *final_kind_out)
+int dspark_oracle_verify_head(int B, int G, int V, int r, const float *Tlog, const float *L,
+                              const float *U, const float *Arec, const float *W, const int *x0, const int *x,
+                              const float *temp, const double *u_accept,
+                              const double *u_final, const int *ell,
+                              const int *force_accept, int *acc_out, int *tokens_out,
+                              int *nout_out, double *pt_x_out, double *pd_x_out,
+                              double *margin_acc_out, double *margin_fin_out,
+                              int *final_kind_out)
 {
     if (B < 0 || G < 1 || V < 2 || r < 1) return ORACLE_ERR_ARG;
+    double *hs = malloc(sizeof(double) * (size_t)r * 2);
+    if (!hs) return ORACLE_ERR_NOMEM;
     double *delta = malloc(sizeof(double) * (size_t)V);
     double *yd = malloc(sizeof(double) * (size_t)V);
     double *yt = malloc(sizeof(double) * (size_t)V);
@@ -437,7 +492,7 @@ int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const fl
     double *et = malloc(sizeof(double) * (size_t)V);
     double *q = malloc(sizeof(double) * (size_t)V);
     if (!delta || !yd || !yt || !ed || !et || !q) {
-        free(delta); free(yd); free(yt); free(ed); free(et); free(q);
+        free(delta); free(yd); free(yt); free(ed); free(et); free(q); free(hs);
         return ORACLE_ERR_NOMEM;
     }
     int rc = ORACLE_OK;
@@ -456,7 +511,6 @@ int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const fl
         for (int k = 1; k <= lb; ++k) {
             size_t o = (size_t)b * G + (k - 1);
             int xk = x[o];
-            int prev = (k == 1) ? x0[b] : x[o - 1];
             const float *Trow = Tlog + ((size_t)b * (G + 1) + (k - 1)) * (size_t)V;
             for (int v = 0; v < V; ++v) yt[v] = (double)Trow[v];
             int accept;
@@ -474,7 +528,7 @@ int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const fl
                 pd_x_out[o] = 1.0;
             } else {
                 double mt, Zt = softmax_row(yt, V, T, et, &mt);
-                markov_bias_row(U, W, V, r, prev, delta);
+                draft_bias(U, Arec, W, V, r, x0[b], x + (size_t)b * G, k, hs, hs + r, delta);
                 const float *Lrow = L + o * (size_t)V;
                 for (int v = 0; v < V; ++v) yd[v] = (double)Lrow[v] + delta[v];
                 double md, Zd = softmax_row(yd, V, T, ed, &md);
@@ -504,8 +558,7 @@ int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const fl
             double mt, Zt = softmax_row(yt, V, T, et, &mt);
             if (A < lb) {
                 size_t o = (size_t)b * G + (ks - 1);
-                int prev = (ks == 1) ? x0[b] : x[o - 1];
-                markov_bias_row(U, W, V, r, prev, delta);
+                draft_bias(U, Arec, W, V, r, x0[b], x + (size_t)b * G, ks, hs, hs + r, delta);
                 const float *Lrow = L + o * (size_t)V;
                 for (int v = 0; v < V; ++v) yd[v] = (double)Lrow[v] + delta[v];
                 double md, Zd = softmax_row(yd, V, T, ed, &md);
@@ -536,6 +589,21 @@ int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const fl
         margin_fin_out[b] = mfin;
         final_kind_out[b] = kind;
     }
-    free(delta); free(yd); free(yt); free(ed); free(et); free(q);
+    free(delta); free(yd); free(yt); free(ed); free(et); free(q); free(hs);
     return rc;
+}
+
+/* Verification of Markov-head drafts (the headline path). */
+int dspark_oracle_verify(int B, int G, int V, int r, const float *Tlog, const float *L,
+                         const float *U, const float *W, const int *x0, const int *x,
+                         const float *temp, const double *u_accept,
+                         const double *u_final, const int *ell,
+                         const int *force_accept, int *acc_out, int *tokens_out,
+                         int *nout_out, double *pt_x_out, double *pd_x_out,
+                         double *margin_acc_out, double *margin_fin_out,
+                         int *final_kind_out)
+{
+    return dspark_oracle_verify_head(B, G, V, r, Tlog, L, U, NULL, W, x0, x, temp, u_accept, u_final, ell,
+                                     force_accept, acc_out, tokens_out, nout_out, pt_x_out, pd_x_out,
+                                     margin_acc_out, margin_fin_out, final_kind_out);
 }

@@ -51,8 +51,8 @@ def use_library(path: str) -> None:
     broken copies this way to show that the pins catch them)."""
     global _lib
     lib = ctypes.CDLL(path)
-    for name in ("dspark_oracle_draft", "dspark_oracle_confidence",
-                 "dspark_oracle_schedule", "dspark_oracle_verify"):
+    for name in ("dspark_oracle_draft", "dspark_oracle_draft_head", "dspark_oracle_confidence",
+                 "dspark_oracle_schedule", "dspark_oracle_verify", "dspark_oracle_verify_head"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
 
@@ -91,18 +91,22 @@ class DraftResult:
     margin: np.ndarray   # [B, G] decision margin
 
 
-def draft(L, U, W, x0, temp, u_draft, force_x=None) -> DraftResult:
-    """Markov-head drafting.  L [B,G,V], U [V,r], W [r,V], x0 [B], temp [B], u_draft [B,G]."""
+def draft(L, U, W, x0, temp, u_draft, force_x=None, A=None) -> DraftResult:
+    """Semi-autoregressive drafting.  L [B,G,V], U [V,r], W [r,V], x0 [B],
+    temp [B], u_draft [B,G]; A [r,r] selects the RNN head (state
+    h_k = tanh(h_{k-1} A + U[x_{k-1}]), bias h_k W), None the Markov head."""
     L = _f32(L); U = _f32(U); W = _f32(W)
     B, G, V = L.shape
     r = U.shape[1]
     assert U.shape == (V, r) and W.shape == (r, V)
+    Ar = _f32(A) if A is not None else None
+    assert Ar is None or Ar.shape == (r, r)
     x0 = _i32(x0); temp = _f32(temp); u = _f64(u_draft)
     fx = _i32(force_x) if force_x is not None else None
     x = np.zeros((B, G), np.int32)
     pd = np.zeros((B, G)); rm = np.zeros((B, G)); rs = np.zeros((B, G)); mg = np.zeros((B, G))
-    rc = _load().dspark_oracle_draft(B, G, V, r, _p(L), _p(U), _p(W), _p(x0), _p(temp), _p(u),
-                                     _p(fx), _p(x), _p(pd), _p(rm), _p(rs), _p(mg))
+    rc = _load().dspark_oracle_draft_head(B, G, V, r, _p(L), _p(U), _p(Ar), _p(W), _p(x0), _p(temp), _p(u),
+                                          _p(fx), _p(x), _p(pd), _p(rm), _p(rs), _p(mg))
     _check(rc, "draft")
     return DraftResult(x, pd, rm, rs, mg)
 
@@ -192,9 +196,11 @@ class VerifyResult:
     final_kind: np.ndarray   # [B] 0 residual, 1 bonus, 2 greedy, 3 empty residual
 
 
-def verify(Tlog, L, U, W, x0, x, temp, u_accept, u_final, ell, force_accept=None) -> VerifyResult:
-    """Rejection-sampling verification over the admitted prefixes."""
+def verify(Tlog, L, U, W, x0, x, temp, u_accept, u_final, ell, force_accept=None, A=None) -> VerifyResult:
+    """Rejection-sampling verification over the admitted prefixes (A: the
+    RNN head's recurrent matrix, as for draft; None for the Markov head)."""
     Tlog = _f32(Tlog); L = _f32(L); U = _f32(U); W = _f32(W)
+    Ar = _f32(A) if A is not None else None
     B, G1, V = Tlog.shape
     G = G1 - 1
     r = U.shape[1]
@@ -205,8 +211,8 @@ def verify(Tlog, L, U, W, x0, x, temp, u_accept, u_final, ell, force_accept=None
     acc = np.zeros(B, np.int32); tok = np.zeros((B, G + 1), np.int32); nout = np.zeros(B, np.int32)
     ptx = np.zeros((B, G)); pdx = np.zeros((B, G)); ma = np.zeros((B, G)); mf = np.zeros(B)
     kind = np.zeros(B, np.int32)
-    rc = _load().dspark_oracle_verify(B, G, V, r, _p(Tlog), _p(L), _p(U), _p(W), _p(x0), _p(x),
-                                      _p(temp), _p(ua), _p(uf), _p(ell), _p(fa), _p(acc), _p(tok),
-                                      _p(nout), _p(ptx), _p(pdx), _p(ma), _p(mf), _p(kind))
+    rc = _load().dspark_oracle_verify_head(B, G, V, r, _p(Tlog), _p(L), _p(U), _p(Ar), _p(W), _p(x0), _p(x),
+                                           _p(temp), _p(ua), _p(uf), _p(ell), _p(fa), _p(acc), _p(tok),
+                                           _p(nout), _p(ptx), _p(pdx), _p(ma), _p(mf), _p(kind))
     _check(rc, "verify")
     return VerifyResult(acc, tok, nout, ptx, pdx, ma, mf, kind)

@@ -193,3 +193,10 @@ def tau_grid(K: int = 65, lo: float = 0.25, hi: float = 4.0) -> np.ndarray:
     if K % 2 == 1 and abs(np.log(lo) + np.log(hi)) < 1e-12:
         g[K // 2] = np.float32(1.0)
     return g
+
+
+def rnn_matrix(r: int, seed: int = 0, gain: float = 0.8) -> np.ndarray:
+    """A recurrent matrix [r, r] ~ N(0, gain^2 / r) (fp32) for the RNN head:
+    with gain < 1 the state update is contractive on average."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, 0x52])))
+    return (g.standard_normal((r, r), dtype=np.float32) * np.float32(gain / np.sqrt(r))).astype(np.float32)

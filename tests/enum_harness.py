@@ -52,7 +52,7 @@ class Scenario:
     state at position k equal to Htab[k-1, x_{k-1}], and the scheduler setup."""
 
     def __init__(self, Lrows, U, W, x0, T, target, hconf=None, knots_n=None, knots_t=None,
-                 budget=-1, mode=oracle.SCHED_ALL, others_S=None, ell_fixed=None):
+                 budget=-1, mode=oracle.SCHED_ALL, others_S=None, ell_fixed=None, A=None):
         self.Lrows = np.asarray(Lrows, np.float32)
         self.G, self.V = self.Lrows.shape
         self.U = np.asarray(U, np.float32)
@@ -67,13 +67,14 @@ class Scenario:
         self.mode = mode
         self.others_S = others_S  # [B_other, G] fixed survivals of other requests
         self.ell_fixed = ell_fixed
+        self.A = None if A is None else np.asarray(A, np.float32)   # RNN head (None: Markov head)
 
     # -- drafting -------------------------------------------------------
     def _draft(self, u_rows, force=None):
         n = u_rows.shape[0]
         L = np.broadcast_to(self.Lrows, (n, self.G, self.V))
         return oracle.draft(L, self.U, self.W, np.full(n, self.x0, np.int32),
-                            np.full(n, self.T, np.float32), u_rows, force_x=force)
+                            np.full(n, self.T, np.float32), u_rows, force_x=force, A=self.A)
 
     def draft_paths(self):
         """All draft paths with probabilities and uniforms realising them."""
@@ -132,7 +133,7 @@ class Scenario:
 
         def run(idx, ua, uf):
             return oracle.verify(Tl[idx], L[idx], self.U, self.W, x0[idx], X[idx], temp[idx],
-                                 ua, uf, ell[idx])
+                                 ua, uf, ell[idx], A=self.A)
 
         # Accept thresholds per (path, k): probability that x_k is accepted
         # given x_1..x_{k-1} were.

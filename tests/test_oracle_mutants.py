@@ -16,10 +16,10 @@ MUTANTS = [
     ("residual_sign", "double d = et[v] / Zt - ed[v] / Zd;", "double d = ed[v] / Zd - et[v] / Zt;"),
     ("ratio_inverted", "double ratio = pt / pd;", "double ratio = pd / pt;"),
     ("verify_conditions_on_current_token",
-     "int prev = (k == 1) ? x0[b] : x[o - 1];\n            const float *Trow",
-     "int prev = x[o];\n            const float *Trow"),
-    ("draft_ignores_previous_token", "            x_out[o] = x;\n            prev = x;",
-     "            x_out[o] = x;"),
+     "draft_bias(U, Arec, W, V, r, x0[b], x + (size_t)b * G, k, hs, hs + r, delta);",
+     "draft_bias(U, Arec, W, V, r, x0[b], x + (size_t)b * G, k + 1, hs, hs + r, delta);"),
+    ("draft_ignores_previous_token", "draft_bias(U, A, W, V, r, x0[b], x_out + (size_t)b * G, i + 1, h, h + r, delta);",
+     "draft_bias(U, A, W, V, r, x0[b], x_out + (size_t)b * G, 1, h, h + r, delta);"),
     ("bonus_from_last_admitted_row", "int ks = A + 1;", "int ks = (A == lb && A > 0) ? A : A + 1;"),
     ("residual_without_clamp", "q[v] = d > 0.0 ? d : 0.0;", "q[v] = d > 0.0 ? d : -d;"),
     ("target_row_shifted", "const float *Trow = Tlog + ((size_t)b * (G + 1) + (k - 1)) * (size_t)V;",
@@ -106,3 +106,31 @@ def test_scheduler_mutant_is_caught(tmp_path, name, old, new):
         oracle.use_library(oracle.build())
     assert caught, f"no scheduler pin catches {name}"
 
+
+
+# Planted mistakes in the RNN head, caught by the RNN pins.
+RNN_MUTANTS = [
+    ("rnn_state_not_carried", "        for (int c = 0; c < r; ++c) h[c] = hn[c];\n", "\n"),
+    ("rnn_without_tanh", "            hn[c] = tanh(a);", "            hn[c] = a;"),
+    ("rnn_state_from_current_token", "int tok = (j == 1) ? x0 : xs[j - 2];", "int tok = (j == 1) ? x0 : xs[j - 1];"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", RNN_MUTANTS, ids=[m[0] for m in RNN_MUTANTS])
+def test_rnn_mutant_is_caught(tmp_path, name, old, new):
+    import test_oracle_rnn as pins
+    so = _build_mutant(tmp_path, name, old, new)
+    caught = []
+    try:
+        oracle.use_library(so)
+        for pin, args in ((pins.test_zero_recurrence_is_the_markov_head_with_tanh_factor, (1.0,)),
+                          (pins.test_bias_depends_on_the_whole_prefix, ()),
+                          (pins.test_rnn_head_keeps_the_target_law, (0, 3, 3, 2, 1.0)),
+                          (pins.test_rnn_and_markov_drafts_differ_when_the_state_carries, ())):
+            try:
+                pin(*args)
+            except (AssertionError, ValueError):
+                caught.append(pin.__name__)
+    finally:
+        oracle.use_library(oracle.build())
+    assert caught, f"no RNN pin catches {name}"

@@ -484,6 +484,113 @@ def run_sts(args):
     return 0
 
 
+def run_production(args):
+    """The headline round with the production scheduler: the capacity from the
+    previous round's survivals (global search, side stream, overlapping
+    drafting) and the dynamic top-K of the current survivals.  One graph per
+    round (the fork to the side stream and the join are in it), replayed with
+    L2 flushed before each; one GPU per rank (replicas)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_draft_rank_b200 import _lib
+    from speculative_decoding_draft_rank_b200.production import ProductionRound, ProductionScheduler
+    from speculative_decoding_draft_rank_b200.round import DeviceRound
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = _workload(args.workload)
+    w.seed = rank
+    inp = w.inputs()
+    dr = DeviceRound(inp, w.knots_n, w.knots_t, w.budget, w.mode, device=dev)
+    ps = ProductionScheduler(w.B, w.G, w.knots_n, w.knots_t, w.budget, device=dev)
+    pr = ProductionRound(dr, ps)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        pr.run(stream)          # round 0: Algorithm 1's own count, no history
+        pr.run(stream)          # round 1: capacity from round 0
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        pr.run(stream)
+    # The selection alone (the stage that replaces Algorithm 1 on the round's
+    # critical path) in its own graph.
+    o = dr.o
+    sel = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(sel, stream=stream):
+        _lib.dspark_schedule_topk(o["S"], ps.capacity, ps.budget, ps.ws_sel, o["ell"], o["n_adm"], o["order"],
+                                  stream)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            graph.replay()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    step_ms, sel_ms = [], []
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                flush.zero_()
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                e1.synchronize()
+                step_ms.append(e0.elapsed_time(e1))
+        torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.steps // 4)):
+            flush.zero_()
+            e0.record(stream)
+            sel.replay()
+            e1.record(stream)
+            e1.synchronize()
+            sel_ms.append(e0.elapsed_time(e1))
+    torch.cuda.synchronize()
+    status = dr.device_status() | ps.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x}")
+    ms = statistics.mean(step_ms)
+    ell_sum = int(o["ell"].sum().item())
+    if world > 1:
+        tt = torch.tensor([ms, float(ell_sum)], device=dev, dtype=torch.float64)
+        gathered = [torch.zeros_like(tt) for _ in range(world)]
+        dist.all_gather(gathered, tt)
+        ms = max(float(g[0]) for g in gathered)
+        ell_tot = sum(float(g[1]) for g in gathered)
+    else:
+        ell_tot = float(ell_sum)
+    line = {
+        "metric": METRIC, "value": ell_tot / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, one batch per rank)",
+        "config": {"workload": w.name, "B": w.B, "G": w.G, "V": w.V, "r": w.r, "d": w.d,
+                   "scheduler": "production: capacity from the previous round (global search, side stream), "
+                                "dynamic top-K of the current survivals",
+                   "l2_flush": "256 MiB write before every timed round", "graph_replay": True,
+                   "parallelism": f"{world} independent engines"},
+        "round": {"admitted_draft_tokens": ell_sum, "capacity": int(ps.capacity.item()),
+                  "selection_ms": statistics.mean(sel_ms)},
+        "gpu_launches": (1 + 1 + 1 + 1 + 5) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    graph.reset()
+    sel.reset()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,13 +603,16 @@ def main():
     ap.add_argument("--reference-requests", type=int, default=8,
                     help="requests per step of the reference arm (the oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded", "sts"],
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded", "sts", "production"],
                     help="replicas: every rank an independent engine (default); sharded: one engine over all "
                          "ranks' requests, survivals all-gathered for one global admission; sts: the "
-                         "confidence head's sequential temperature scaling fit")
+                         "confidence head's sequential temperature scaling fit; production: the round with "
+                         "the production scheduler (capacity from the previous round, dynamic top-K)")
     args = ap.parse_args()
     if args.mode == "sts":
         return run_sts(args)
+    if args.mode == "production" and args.impl == "native":
+        return run_production(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.mode == "sharded":

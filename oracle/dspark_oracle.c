@@ -231,6 +231,36 @@ int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float 
                                     rowmax_out, rowsum_out, margin_out);
 }
 
+/* The RNN head's states along drafted blocks (see draft_bias): for every
+ * request b and position k = 1..G, h_k from x_0 and x_1..x_{k-1} of x [B][G].
+ * Output h_out [B][G][r] (fp64). */
+int dspark_oracle_rnn_states(int B, int G, int r, const float *U, const float *Arec, const int *x0,
+                             const int *x, double *h_out)
+{
+    if (B < 0 || G < 1 || r < 1 || !Arec) return ORACLE_ERR_ARG;
+    double *h = malloc(sizeof(double) * (size_t)r);
+    double *hn = malloc(sizeof(double) * (size_t)r);
+    if (!h || !hn) { free(h); free(hn); return ORACLE_ERR_NOMEM; }
+    for (int b = 0; b < B; ++b) {
+        for (int c = 0; c < r; ++c) h[c] = 0.0;
+        for (int k = 1; k <= G; ++k) {
+            int tok = (k == 1) ? x0[b] : x[(size_t)b * G + k - 2];
+            for (int c = 0; c < r; ++c) {
+                double a = 0.0;
+                for (int q = 0; q < r; ++q) a += h[q] * (double)Arec[(size_t)q * r + c];
+                a += (double)U[(size_t)tok * r + c];
+                hn[c] = tanh(a);
+            }
+            for (int c = 0; c < r; ++c) {
+                h[c] = hn[c];
+                h_out[((size_t)b * G + (k - 1)) * r + c] = hn[c];
+            }
+        }
+    }
+    free(h); free(hn);
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Stage 2, confidence and prefix survival: [KB] Key Contributions (a
  * lightweight linear confidence head gives a per-position survival

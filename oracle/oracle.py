@@ -111,6 +111,18 @@ def draft(L, U, W, x0, temp, u_draft, force_x=None, A=None) -> DraftResult:
     return DraftResult(x, pd, rm, rs, mg)
 
 
+def rnn_states(U, A, x0, x):
+    """The RNN head's states h_1..h_G [B, G, r] (fp64) along the drafted
+    tokens x [B, G] from x0 [B]: h_k = tanh(h_{k-1} A + U[x_{k-1}])."""
+    U = _f32(U); A = _f32(A); x0 = _i32(x0); x = _i32(x)
+    B, G = x.shape
+    r = U.shape[1]
+    h = np.zeros((B, G, r))
+    rc = _load().dspark_oracle_rnn_states(B, G, r, _p(U), _p(A), _p(x0), _p(x), _p(h))
+    _check(rc, "rnn_states")
+    return h
+
+
 def confidence(h, w, bias=0.0, tau=None):
     """Linear confidence head and prefix survival.  h [B,G,d], w [d] -> (c, S) fp64 [B,G]."""
     h = _f32(h); w = _f32(w)

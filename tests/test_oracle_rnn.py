@@ -102,3 +102,29 @@ def test_rnn_and_markov_drafts_differ_when_the_state_carries():
     b = oracle.draft(L, U, W, x0, temp, u, A=A, force_x=a.x)
     assert np.array_equal(a.rowmax[:, 0], b.rowmax[:, 0]) and np.array_equal(a.rowsum[:, 0], b.rowsum[:, 0])
     assert np.all(np.abs(a.rowmax[:, 1:] - b.rowmax[:, 1:]) > 0)
+
+
+def test_states_with_zero_recurrence_are_tanh_of_the_factor_rows():
+    # A = 0: h_k = tanh(U[x_{k-1}]) exactly as numpy's tanh gives it.
+    rng, L, U, W, x0, u = _tiny(5, 4, 3, 20, 6)
+    x = rng.integers(0, 20, (4, 3)).astype(np.int32)
+    h = oracle.rnn_states(U, np.zeros((6, 6), np.float32), x0, x)
+    prev = np.concatenate([x0[:, None], x[:, :-1]], axis=1)
+    np.testing.assert_allclose(h, np.tanh(U.astype(np.float64)[prev]), rtol=0, atol=1e-15)
+
+
+def test_states_match_the_drafting_bias():
+    # The state the drafting stage used is the one rnn_states reports: with
+    # W = identity (V = r) and L = 0, row max and log Z of a greedy row are
+    # max_c h_k[c] and 0.
+    rng = np.random.default_rng(6)
+    r = 5
+    U = rng.uniform(-1, 1, (r, r)).astype(np.float32)
+    W = np.eye(r, dtype=np.float32)
+    A = synth.rnn_matrix(r, seed=7)
+    L = np.zeros((3, 4, r), np.float32)
+    x0 = np.array([0, 2, 4], np.int32)
+    d = oracle.draft(L, U, W, x0, np.zeros(3, np.float32), rng.random((3, 4)), A=A)
+    h = oracle.rnn_states(U, A, x0, d.x)
+    np.testing.assert_allclose(d.rowmax, h.max(axis=2), rtol=0, atol=1e-15)
+    assert np.array_equal(d.x, h.argmax(axis=2))

@@ -111,7 +111,8 @@ def test_scheduler_mutant_is_caught(tmp_path, name, old, new):
 # Planted mistakes in the RNN head, caught by the RNN pins.
 RNN_MUTANTS = [
     ("rnn_state_not_carried", "        for (int c = 0; c < r; ++c) h[c] = hn[c];\n", "\n"),
-    ("rnn_without_tanh", "            hn[c] = tanh(a);", "            hn[c] = a;"),
+    ("rnn_without_tanh", "            hn[c] = tanh(a);\n        }\n        for (int c = 0; c < r; ++c) h[c] = hn[c];",
+     "            hn[c] = a;\n        }\n        for (int c = 0; c < r; ++c) h[c] = hn[c];"),
     ("rnn_state_from_current_token", "int tok = (j == 1) ? x0 : xs[j - 2];", "int tok = (j == 1) ? x0 : xs[j - 1];"),
 ]
 

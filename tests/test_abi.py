@@ -179,3 +179,15 @@ def test_schedule_topk_argument_checks(lib):
     assert lib.dspark_schedule(FAKE, 8, 5, FAKE, FAKE, 2, -1, 4, FAKE_WS, 1 << 20, FAKE, FAKE, FAKE, None,
                                None) == 1
 
+
+
+def test_injected_failure_on_variant_entries(lib, monkeypatch):
+    """The calibration and top-K entry points honour host-side injection too
+    (they fail before touching any pointer)."""
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_sts_fit=4")
+    assert lib.dspark_sts_fit(FAKE, FAKE, FAKE, 64, 5, 9, 15, FAKE_WS, 1 << 20, FAKE, None, None, None, None,
+                              None) == 4
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_survival_auc=5")
+    assert lib.dspark_survival_auc(FAKE, FAKE, 64, 5, FAKE, FAKE, None) == 5
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_schedule_topk=4")
+    assert lib.dspark_schedule_topk(FAKE, 8, 5, FAKE, -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 4

@@ -130,7 +130,8 @@ class ClockSampler:
 # The sources the drafting kernel is built from (kernel, its device helpers,
 # its host launcher): profile counters are valid only for the code they were
 # taken on.
-DRAFT_KERNEL_SOURCES = ("draft_tc.cu", "finalize.cuh", "tc.cuh", "common.cuh", "kernels.cuh", "draft.cu")
+DRAFT_KERNEL_SOURCES = ("draft_tc.cu", "draft_pair.cu", "finalize.cuh", "tc.cuh", "common.cuh", "kernels.cuh",
+                        "draft.cu")
 
 
 def kernel_sources_digest():
@@ -151,7 +152,7 @@ def profiled_traffic(workload_name):
     return d["dram_bytes_per_round"] if d.get("sources_digest") == kernel_sources_digest() else None
 
 
-def oracle_sample(w, inp, n_req, seed=0):
+def oracle_sample(w, inp, n_req, seed=0, A=None):
     """Time the fp64 oracle (as it stands, one thread) on a bounded sample of
     the round: confidence and scheduling for the whole batch, drafting and
     verification for n_req requests.  Returns (verified tokens in the sample,
@@ -166,9 +167,9 @@ def oracle_sample(w, inp, n_req, seed=0):
     c0 = time.process_time()
     _, S = oracle.confidence(inp.h, inp.w, inp.bias)
     sch = oracle.schedule(S, w.knots_n, w.knots_t, w.budget, w.mode)
-    dr = oracle.draft(sub.L, sub.U, sub.W, sub.x0, sub.temp, sub.u_draft.astype(np.float64))
+    dr = oracle.draft(sub.L, sub.U, sub.W, sub.x0, sub.temp, sub.u_draft.astype(np.float64), A=A)
     oracle.verify(sub.Tlog, sub.L, sub.U, sub.W, sub.x0, dr.x, sub.temp, sub.u_accept.astype(np.float64),
-                  sub.u_final.astype(np.float64), sch.ell[idx])
+                  sub.u_final.astype(np.float64), sch.ell[idx], A=A)
     dt = time.perf_counter() - t0
     oracle_sample.cpu_s = time.process_time() - c0   # CPU time of every thread in the region
     return int(sch.ell[idx].sum()), dt, len(idx)
@@ -612,6 +613,8 @@ def main():
     ap.add_argument("--reference-requests", type=int, default=8,
                     help="requests per step of the reference arm (the oracle)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--head", default="markov", choices=["markov", "rnn"],
+                    help="sequential draft head: the Markov head (the headline path) or the RNN head")
     ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded", "sts", "production"],
                     help="replicas: every rank an independent engine (default); sharded: one engine over all "
                          "ranks' requests, survivals all-gathered for one global admission; sts: the "
@@ -647,7 +650,11 @@ def main():
     w = _workload(args.workload)
     w.seed = rank  # every engine drafts its own batch
     inp = w.inputs()
-    dr = DeviceRound(inp, w.knots_n, w.knots_t, w.budget, w.mode, device=dev, pinned_host=True)
+    Arec = None
+    if args.head == "rnn":
+        from speculative_decoding_draft_rank_b200 import synth
+        Arec = synth.bf16_to_f32(synth.bf16_bits(synth.rnn_matrix(w.r, seed=rank))).reshape(w.r, w.r)
+    dr = DeviceRound(inp, w.knots_n, w.knots_t, w.budget, w.mode, device=dev, pinned_host=True, Arec=Arec)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
 
@@ -658,19 +665,15 @@ def main():
     from speculative_decoding_draft_rank_b200 import _lib
     t, o = dr.t, dr.o
     stages = [
-        lambda: _lib.dspark_draft_markov(t["L"], t["U"], t["Wt"], t["x0"], t["temp"], t["u_draft"], dr.ws,
-                                         o["x"], o["pd_x"], o["rowmax"], o["rowsum"]),
+        lambda: dr.draft(),
         lambda: _lib.dspark_confidence(t["h"], t["w"], float(inp.bias), t["tau"], o["c"], o["S"]),
         lambda: _lib.dspark_schedule(o["S"], t["knots_n"], t["knots_t"], dr.budget, dr.mode, dr.ws, o["ell"],
                                      o["n_adm"], o["theta"], o["order"]),
-        lambda: _lib.dspark_verify(t["Tlog"], t["L"], t["U"], t["Wt"], t["x0"], o["x"], o["pd_x"], o["rowmax"],
-                                   o["rowsum"], t["temp"], t["u_accept"], t["u_final"], o["ell"], dr.ws,
-                                   o["acc"], o["tokens"], o["nout"], o["pt_x"]),
+        lambda: dr.verify(),
     ]
     graph = torch.cuda.CUDAGraph()          # the whole round: the timed unit
     with torch.cuda.graph(graph, stream=stream):
-        for f in stages:
-            f()
+        dr.run(stream)                      # confidence forked to a side stream, joined before scheduling
     stage_graphs = []                       # one graph per stage: the breakdown
     for f in stages:
         g = torch.cuda.CUDAGraph()
@@ -773,8 +776,10 @@ def main():
     # in its stage graph); fp32 rounds launch a tile and a finalize kernel per
     # position.
     bf16 = w.dtype == "bf16"
-    stage_kernels = ["markov_tile_tc (drafting, all positions in one launch)" if bf16 else "draft stage",
-                     "confidence_kernel", "schedule_kernel", "verify stage"]
+    pair = bf16 and (w.B > 128 or args.head == "rnn")
+    draft_kernel = ("markov_pair_tc (drafting on CTA pairs, all positions in one launch)" if pair else
+                    "markov_tile_tc (drafting, all positions in one launch)") if bf16 else "draft stage"
+    stage_kernels = [draft_kernel, "confidence_kernel", "schedule_kernel", "verify stage"]
     stage_launches = [1 if bf16 else 2 * w.G, 1, 1, 5]
     draft_flops = 2.0 * w.B * w.G * w.r * w.V
     line = {
@@ -782,6 +787,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded generator, one batch per rank)",
         "config": {"workload": w.name, "B": w.B, "G": w.G, "V": w.V, "r": w.r, "d": w.d,
+                   "head": args.head,
                    "l2_flush": "256 MiB write before every timed round", "graph_replay": True,
                    "parallelism": f"{world} independent engines"},
         "round": {"admitted_draft_tokens": ell_sum, "emitted_tokens": nout_sum,
@@ -804,7 +810,7 @@ def main():
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
-        t, secs, n = oracle_sample(w, inp, args.oracle_requests)
+        t, secs, n = oracle_sample(w, inp, args.oracle_requests, A=Arec)
         cores = max(1, round(oracle_sample.cpu_s / secs))
         line["cpu_baseline"] = {"value": t / secs, "unit": UNIT, "cores": cores, "kind": "oracle",
                                 "sample": f"{n} of {w.B} requests drafted+verified, whole-batch "

@@ -228,6 +228,41 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
                             float *pt_x_out, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* The RNN sequential head.  [PL] §3.1: the sequential stage conditions each
+ * position on the tokens sampled before it; besides the Markov head's
+ * low-rank transition matrix it names an RNN head whose recurrent state
+ * summarises the whole in-block prefix.  [KB] Key Contributions: the two
+ * variants (first-order dependency by a low-rank factorisation; the full
+ * within-block history).  The pages give no equations; the reading here is
+ * the plainest recurrence over the Markov head's factors: a state of size r,
+ *   h_1 = tanh(U[x_0]),  h_k = tanh(h_{k-1} Arec + U[x_{k-1}]),
+ *   Delta_k = h_k W  (Delta_k[v] = sum_c h_k[c] * Wt[v,c]),
+ * with everything else as in dspark_draft_markov / dspark_verify.
+ *
+ * dspark_draft_rnn: as dspark_draft_markov, plus Arec [r,r] bf16 (row q,
+ *   column c: the weight from state q to state c) and the output
+ *   H_out [B,G,r] f32: H_out[b,k-1,:] = h_k, the state that biased position k
+ *   (verification rebuilds p_d from it).  bf16 only (DSPARK_ERR_UNSUPPORTED_DTYPE
+ *   otherwise), r <= 256, H_out 16-byte aligned; same workspace size.
+ *   The state is computed in fp32 and enters the tensor-core product as two
+ *   bf16 parts (high + low, about 2^-17 relative).
+ * dspark_verify_rnn: as dspark_verify with the states H [B,G,r] f32 from
+ *   dspark_draft_rnn in place of U and x0 (the residual at a rejection
+ *   rebuilds p_d from L + h_k W).  Same limits as dspark_draft_rnn. */
+dspark_status dspark_draft_rnn(const void *L, const void *U, const void *Arec, const void *Wt,
+                               const int32_t *x0, const float *temp, const float *u_draft, int B,
+                               int G, int V, int r, int dtype, void *ws, size_t ws_bytes,
+                               int32_t *x_out, float *pd_x_out, float *rowmax_out,
+                               float *rowsum_out, float *H_out, void *stream);
+dspark_status dspark_verify_rnn(const void *Tlog, const void *L, const float *H, const void *Wt,
+                                const int32_t *x, const float *pd_x, const float *rowmax,
+                                const float *rowsum, const float *temp, const float *u_accept,
+                                const float *u_final, const int32_t *ell, int B, int G, int V,
+                                int r, int dtype, void *ws, size_t ws_bytes, int32_t *acc_out,
+                                int32_t *tokens_out, int32_t *nout_out, float *pt_x_out,
+                                void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Drafting without a workspace, for callers that cannot allocate device
  * memory when they draft: e.g. a plugin of an inference engine that receives
  * only its inputs and outputs at enqueue time (the engine planned all memory
@@ -242,8 +277,8 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
  * this library holds until the process exits.  Rounds whose drafting
  * workspace (dspark_draft_workspace_size) would exceed that size are rejected
  * with DSPARK_ERR_WORKSPACE before any work is enqueued; the headline shape
- * B = 256, V = 129280, r = 256 needs about 6.3 MB.  No call allocates: no
- * cudaMalloc, cudaFree or allocating library routine.
+ * B = 256, G = 5, V = 129280, r = 256 needs 6,467,840 bytes.  No call
+ * allocates: no cudaMalloc, cudaFree or allocating library routine.
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream
@@ -251,9 +286,14 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
  * contents: the call clears the status word it needs to start at zero, and
  * the rest is written before it is read.  Calls that may overlap on the GPU
  * (other streams, other host threads) race on the array and must be
- * serialised by the caller.  Device-side data errors are clamped as in
- * dspark_draft_markov but are not reported back. */
+ * serialised by the caller.  Device-side data errors and a bounded wait
+ * that ran out are clamped or abandoned as in dspark_draft_markov and
+ * recorded in the array's status word, which the call clears first:
+ * dspark_draft_noalloc_device_status synchronises `stream` and copies that
+ * word (the DSPARK_DEV_* bits of the last call enqueued on `stream`) to
+ * *status_out.  After DSPARK_DEV_TIMEOUT the outputs are not valid. */
 size_t dspark_draft_noalloc_max_scratch(void);
+dspark_status dspark_draft_noalloc_device_status(void *stream, uint32_t *status_out);
 dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const void *Wt,
                                           const int32_t *x0, const float *temp,
                                           const float *u_draft, int B, int G, int V, int r,

@@ -233,11 +233,17 @@ int dspark_oracle_draft(int B, int G, int V, int r, const float *L, const float 
 
 /* The RNN head's states along drafted blocks (see draft_bias): for every
  * request b and position k = 1..G, h_k from x_0 and x_1..x_{k-1} of x [B][G].
+ * Tokens index U [V][r]: any token outside [0, V) is an argument error.
  * Output h_out [B][G][r] (fp64). */
-int dspark_oracle_rnn_states(int B, int G, int r, const float *U, const float *Arec, const int *x0,
+int dspark_oracle_rnn_states(int B, int G, int V, int r, const float *U, const float *Arec, const int *x0,
                              const int *x, double *h_out)
 {
-    if (B < 0 || G < 1 || r < 1 || !Arec) return ORACLE_ERR_ARG;
+    if (B < 1 || G < 1 || V < 2 || r < 1 || !Arec) return ORACLE_ERR_ARG;
+    for (int b = 0; b < B; ++b) {
+        if (x0[b] < 0 || x0[b] >= V) return ORACLE_ERR_ARG;
+        for (int k = 0; k + 1 < G; ++k)
+            if (x[(size_t)b * G + k] < 0 || x[(size_t)b * G + k] >= V) return ORACLE_ERR_ARG;
+    }
     double *h = malloc(sizeof(double) * (size_t)r);
     double *hn = malloc(sizeof(double) * (size_t)r);
     if (!h || !hn) { free(h); free(hn); return ORACLE_ERR_NOMEM; }
@@ -338,14 +344,20 @@ static int cand_cmp(const void *pa, const void *pb)
  * count maximises Theta over all n (no early stop).  force_n >= 0 replaces
  * the admitted count (used to follow another implementation after a
  * near-tie).  Outputs: ell [B], n_adm, theta (objective at the admitted
- * count), order [B*G] (sorted candidate indices), margin_theta (smallest
- * relative |Theta_{n+1} - Theta_n| / Theta_n over the comparisons made),
- * margin_gap (S gap across the cut, +inf if nothing is cut). */
+ * count), order [B*G] (sorted candidate indices), margin_theta (the
+ * decision margin of the early stop, taken at the stop point: the relative
+ * objective change |Theta_{n+1} - Theta_n| / Theta_n of the comparison that
+ * ended admission; +inf when admission ended at the budget or with every
+ * candidate admitted, or in the other modes), margin_gap (S gap across the
+ * cut, +inf if nothing is cut), and margins (nullable, [B*G]): the relative
+ * objective change of every comparison n the early stop made (n = 0..the
+ * stop), NaN for comparisons not made -- the margin at another
+ * implementation's stop point when it stopped earlier. */
 int dspark_oracle_schedule(int B, int G, const double *S, int P, const int *knots_n,
                            const double *knots_t, int budget, int mode, int force_n,
                            int *ell_out, int *n_adm_out, double *theta_out,
                            int *order_out, double *margin_theta_out,
-                           double *margin_gap_out)
+                           double *margin_gap_out, double *margins_out)
 {
     if (B < 1 || G < 1 || P < 1 || knots_n[0] != 0) return ORACLE_ERR_ARG;
     int N = B * G;
@@ -359,6 +371,8 @@ int dspark_oracle_schedule(int B, int G, const double *S, int P, const int *knot
     qsort(c, (size_t)N, sizeof(cand_t), cand_cmp);
     if (order_out)
         for (int n = 0; n < N; ++n) order_out[n] = c[n].idx;
+    if (margins_out)
+        for (int n = 0; n < N; ++n) margins_out[n] = NAN;
 
     int limit = N;
     if (budget >= 0 && budget < limit) limit = budget;
@@ -377,8 +391,11 @@ int dspark_oracle_schedule(int B, int G, const double *S, int P, const int *knot
             double Vn1 = Vn + c[n].s;
             double th1 = Vn1 / t1;
             double rel = fabs(th1 - theta) / theta;
-            if (rel < mtheta) mtheta = rel;
-            if (Vn1 * t0 < Vn * t1) break; /* Theta_{n+1} < Theta_n: stop */
+            if (margins_out) margins_out[n] = rel;
+            if (Vn1 * t0 < Vn * t1) { /* Theta_{n+1} < Theta_n: stop */
+                mtheta = rel;
+                break;
+            }
             Vn = Vn1;
             theta = th1;
             ++n;

@@ -116,9 +116,9 @@ def rnn_states(U, A, x0, x):
     tokens x [B, G] from x0 [B]: h_k = tanh(h_{k-1} A + U[x_{k-1}])."""
     U = _f32(U); A = _f32(A); x0 = _i32(x0); x = _i32(x)
     B, G = x.shape
-    r = U.shape[1]
+    V, r = U.shape
     h = np.zeros((B, G, r))
-    rc = _load().dspark_oracle_rnn_states(B, G, r, _p(U), _p(A), _p(x0), _p(x), _p(h))
+    rc = _load().dspark_oracle_rnn_states(B, G, V, r, _p(U), _p(A), _p(x0), _p(x), _p(h))
     _check(rc, "rnn_states")
     return h
 
@@ -141,8 +141,9 @@ class ScheduleResult:
     n_adm: int               # admitted candidates
     theta: float             # objective at the admitted count
     order: np.ndarray        # [B*G] sorted candidate indices (idx = i*B + b)
-    margin_theta: float      # smallest relative objective change compared
+    margin_theta: float      # relative objective change at the stop point (+inf: no stop comparison)
     margin_gap: float        # survival gap across the cut
+    margins: np.ndarray      # [B*G] relative objective change of every comparison made (NaN: not made)
 
 
 def schedule(S, knots_n, knots_t, budget=-1, mode=SCHED_GREEDY_EARLY_STOP, force_n=-1) -> ScheduleResult:
@@ -152,11 +153,12 @@ def schedule(S, knots_n, knots_t, budget=-1, mode=SCHED_GREEDY_EARLY_STOP, force
     kn = _i32(knots_n); kt = _f64(knots_t)
     ell = np.zeros(B, np.int32); order = np.zeros(B * G, np.int32)
     n_adm = ctypes.c_int(0); th = ctypes.c_double(0); mth = ctypes.c_double(0); mgap = ctypes.c_double(0)
+    margins = np.zeros(B * G)
     rc = _load().dspark_oracle_schedule(B, G, _p(S), len(kn), _p(kn), _p(kt), int(budget), int(mode),
                                         int(force_n), _p(ell), ctypes.byref(n_adm), ctypes.byref(th),
-                                        _p(order), ctypes.byref(mth), ctypes.byref(mgap))
+                                        _p(order), ctypes.byref(mth), ctypes.byref(mgap), _p(margins))
     _check(rc, "schedule")
-    return ScheduleResult(ell, n_adm.value, th.value, order, mth.value, mgap.value)
+    return ScheduleResult(ell, n_adm.value, th.value, order, mth.value, mgap.value, margins)
 
 
 def schedule_threshold(S, threshold, budget=-1):

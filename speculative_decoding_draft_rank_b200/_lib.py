@@ -31,7 +31,8 @@ EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov
            "dspark_schedule_workspace_size", "dspark_schedule", "dspark_verify_workspace_size",
            "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
            "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold",
-           "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc", "dspark_schedule_topk")
+           "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc", "dspark_schedule_topk",
+           "dspark_draft_noalloc_device_status", "dspark_draft_rnn", "dspark_verify_rnn")
 
 
 class DsparkError(RuntimeError):
@@ -78,6 +79,12 @@ def load() -> ctypes.CDLL:
     lib.dspark_draft_noalloc_max_scratch.argtypes = []
     lib.dspark_draft_markov_noalloc.restype = _i
     lib.dspark_draft_markov_noalloc.argtypes = [_vp] * 6 + [_i] * 5 + [_vp] * 5
+    lib.dspark_draft_rnn.restype = _i
+    lib.dspark_draft_rnn.argtypes = [_vp] * 7 + [_i] * 5 + [_vp, _sz] + [_vp] * 6
+    lib.dspark_verify_rnn.restype = _i
+    lib.dspark_verify_rnn.argtypes = [_vp] * 12 + [_i] * 5 + [_vp, _sz] + [_vp] * 5
+    lib.dspark_draft_noalloc_device_status.restype = _i
+    lib.dspark_draft_noalloc_device_status.argtypes = [_vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.dspark_schedule_topk.restype = _i
     lib.dspark_schedule_topk.argtypes = [_vp, _i, _i, _vp, _i, _vp, _sz, _vp, _vp, _vp, _vp]
     lib.dspark_sts_workspace_size.restype = _sz
@@ -144,6 +151,28 @@ def dspark_draft_markov(L, U, Wt, x0, temp, u_draft, ws, x_out, pd_x_out, rowmax
           _ptr(rowmax_out), _ptr(rowsum_out), _stream(stream))
 
 
+def dspark_draft_rnn(L, U, Arec, Wt, x0, temp, u_draft, ws, x_out, pd_x_out, rowmax_out, rowsum_out, H_out,
+                     stream=None):
+    """Drafting with the RNN head: Arec [r, r] bf16 recurrent matrix; H_out
+    [B, G, r] fp32 receives the state that biased every position."""
+    B, G, V = L.shape
+    r = U.shape[1]
+    _call("dspark_draft_rnn", _ptr(L), _ptr(U), _ptr(Arec), _ptr(Wt), _ptr(x0), _ptr(temp), _ptr(u_draft), B, G,
+          V, r, _dtype(L), _ptr(ws), ws.numel() * ws.element_size(), _ptr(x_out), _ptr(pd_x_out), _ptr(rowmax_out),
+          _ptr(rowsum_out), _ptr(H_out), _stream(stream))
+
+
+def dspark_verify_rnn(Tlog, L, H, Wt, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell, ws, acc_out,
+                      tokens_out, nout_out, pt_x_out=None, stream=None):
+    """Verification of RNN-head drafts (the states H from dspark_draft_rnn)."""
+    B, G1, V = Tlog.shape
+    r = H.shape[2]
+    _call("dspark_verify_rnn", _ptr(Tlog), _ptr(L), _ptr(H), _ptr(Wt), _ptr(x), _ptr(pd_x), _ptr(rowmax),
+          _ptr(rowsum), _ptr(temp), _ptr(u_accept), _ptr(u_final), _ptr(ell), B, G1 - 1, V, r, _dtype(Tlog),
+          _ptr(ws), ws.numel() * ws.element_size(), _ptr(acc_out), _ptr(tokens_out), _ptr(nout_out),
+          _ptr(pt_x_out), _stream(stream))
+
+
 def dspark_draft_noalloc_max_scratch() -> int:
     return int(load().dspark_draft_noalloc_max_scratch())
 
@@ -155,6 +184,14 @@ def dspark_draft_markov_noalloc(L, U, Wt, x0, temp, u_draft, x_out, pd_x_out, ro
     r = U.shape[1]
     _call("dspark_draft_markov_noalloc", _ptr(L), _ptr(U), _ptr(Wt), _ptr(x0), _ptr(temp), _ptr(u_draft), B,
           G, V, r, _dtype(L), _ptr(x_out), _ptr(pd_x_out), _ptr(rowmax_out), _ptr(rowsum_out), _stream(stream))
+
+
+def dspark_draft_noalloc_device_status(stream=None) -> int:
+    """Status word of the last allocation-free drafting call on `stream`
+    (synchronises the stream)."""
+    out = ctypes.c_uint32(0)
+    _call("dspark_draft_noalloc_device_status", _stream(stream), ctypes.byref(out))
+    return int(out.value)
 
 
 def dspark_confidence(h, w, bias, tau, c_out, S_out, stream=None):

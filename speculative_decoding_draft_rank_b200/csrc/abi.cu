@@ -3,6 +3,7 @@
 // allocates memory or synchronises, except dspark_get_device_status.
 #include <cstring>
 
+#include "abi_util.cuh"
 #include "calibration.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
@@ -11,36 +12,6 @@
 using namespace dspark;
 
 namespace {
-
-bool dtype_ok(int dt) { return dt == DSPARK_F32 || dt == DSPARK_BF16; }
-bool aligned256(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255) == 0; }
-// bf16 arrays are read by TMA and 16-byte vector loads.
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
-
-dspark_status check_common(int B, int G, int V, int r, int dtype) {
-    if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
-    if (B < 1 || B > 4096 || G < 1 || G > 16 || V < 2 || V > (1 << 20) || r < 1 || r > 512)
-        return DSPARK_ERR_INVALID_ARG;
-    // bf16 rows are moved by TMA: 16-byte row pitches for the logits and factors.
-    if (dtype == DSPARK_BF16 && ((r % 16) != 0 || (V % 8) != 0)) return DSPARK_ERR_INVALID_ARG;
-    return DSPARK_OK;
-}
-
-dspark_status check_ws(const void *ws, size_t have, size_t need) {
-    if (ws == nullptr || !aligned256(ws) || have < need) return DSPARK_ERR_WORKSPACE;
-    return DSPARK_OK;
-}
-
-// Host-side fault injection for failure-path tests: DSPARK_INJECT_ERROR=<entry
-// point name>=<status> makes that entry point return <status> without
-// enqueuing work.
-dspark_status injected(const char *name) {
-    const char *env = getenv("DSPARK_INJECT_ERROR");
-    if (env == nullptr) return DSPARK_OK;
-    const size_t n = strlen(name);
-    if (strncmp(env, name, n) == 0 && env[n] == '=') return (dspark_status)atoi(env + n + 1);
-    return DSPARK_OK;
-}
 
 dspark_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
 
@@ -172,7 +143,45 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
     if (dtype == DSPARK_BF16 && !(aligned16(Tlog) && aligned16(L) && aligned16(U) && aligned16(Wt)))
         return DSPARK_ERR_INVALID_ARG;
     if (dspark_status s = check_ws(ws, ws_bytes, verify_ws_bytes(B, G, V, r, dtype))) return s;
-    VerifyArgs a{Tlog, L, U, Wt, x0, x, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell,
+    VerifyArgs a{Tlog, L, U, Wt, x0, x, nullptr, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell,
+                 B, G, V, r, dtype, acc_out, tokens_out, nout_out, pt_x_out};
+    return cuda_status(launch_verify(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_draft_rnn(const void *L, const void *U, const void *Arec, const void *Wt, const int32_t *x0,
+                               const float *temp, const float *u_draft, int B, int G, int V, int r, int dtype,
+                               void *ws, size_t ws_bytes, int32_t *x_out, float *pd_x_out, float *rowmax_out,
+                               float *rowsum_out, float *H_out, void *stream) {
+    if (dspark_status s = injected("dspark_draft_rnn")) return s;
+    if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
+    if (dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED_DTYPE;
+    if (r > 256) return DSPARK_ERR_INVALID_ARG;
+    if (!L || !U || !Arec || !Wt || !x0 || !temp || !u_draft || !x_out || !pd_x_out || !rowmax_out ||
+        !rowsum_out || !H_out)
+        return DSPARK_ERR_INVALID_ARG;
+    if (!(aligned16(L) && aligned16(U) && aligned16(Wt) && aligned16(H_out))) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, draft_ws_bytes(B, G, V, r, dtype))) return s;
+    DraftArgs a{L, U, Wt, x0, temp, u_draft, B, G, V, r, dtype, x_out, pd_x_out, rowmax_out, rowsum_out};
+    a.Arec = Arec;
+    a.H_out = H_out;
+    return cuda_status(launch_draft(a, ws, static_cast<cudaStream_t>(stream)));
+}
+
+dspark_status dspark_verify_rnn(const void *Tlog, const void *L, const float *H, const void *Wt, const int32_t *x,
+                                const float *pd_x, const float *rowmax, const float *rowsum, const float *temp,
+                                const float *u_accept, const float *u_final, const int32_t *ell, int B, int G, int V,
+                                int r, int dtype, void *ws, size_t ws_bytes, int32_t *acc_out, int32_t *tokens_out,
+                                int32_t *nout_out, float *pt_x_out, void *stream) {
+    if (dspark_status s = injected("dspark_verify_rnn")) return s;
+    if (dspark_status s = check_common(B, G, V, r, dtype)) return s;
+    if (dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED_DTYPE;
+    if (r > 256) return DSPARK_ERR_INVALID_ARG;
+    if (!Tlog || !L || !H || !Wt || !x || !pd_x || !rowmax || !rowsum || !temp || !u_accept || !u_final || !ell ||
+        !acc_out || !tokens_out || !nout_out)
+        return DSPARK_ERR_INVALID_ARG;
+    if (!(aligned16(Tlog) && aligned16(L) && aligned16(H) && aligned16(Wt))) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = check_ws(ws, ws_bytes, verify_ws_bytes(B, G, V, r, dtype))) return s;
+    VerifyArgs a{Tlog, L, nullptr, Wt, nullptr, x, H, pd_x, rowmax, rowsum, temp, u_accept, u_final, ell,
                  B, G, V, r, dtype, acc_out, tokens_out, nout_out, pt_x_out};
     return cuda_status(launch_verify(a, ws, static_cast<cudaStream_t>(stream)));
 }

@@ -162,7 +162,7 @@ size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_m
     bytes += align256(sizeof(float) * (size_t)B * nt);    // part_s
     bytes += align256(sizeof(int32_t) * (size_t)B * nt);  // part_a
-    if (dtype == DSPARK_BF16) bytes += align256((size_t)B * r * 2);   // E
+    if (dtype == DSPARK_BF16) bytes += align256((size_t)2 * B * r * 2);   // E (the RNN head stages two parts)
     return bytes;
 }
 
@@ -176,7 +176,7 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     w.part_s = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
     w.part_a = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (size_t)B * nt);
     w.E = nullptr;
-    if (dtype == DSPARK_BF16) { w.E = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)B * r * 2); }
+    if (dtype == DSPARK_BF16) { w.E = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)2 * B * r * 2); }
     w.nTiles = (int)nt;
     return w;
 }
@@ -188,13 +188,17 @@ FinArgs fin_args(const DraftArgs &a, const DraftWs &w) {
     f.part_m = w.part_m; f.part_s = w.part_s; f.part_a = w.part_a;
     f.x_out = a.x_out; f.pd_out = a.pd_out; f.rowmax_out = a.rowmax_out; f.rowsum_out = a.rowsum_out;
     f.E = w.E; f.hdr = w.hdr;
+    f.Arec = static_cast<const __nv_bfloat16 *>(a.Arec);
+    f.H = a.H_out;
     return f;
 }
 
 cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
     DraftWs w = carve_draft_ws(ws, a.B, a.V, a.r, a.dtype);
     const FinArgs f = fin_args(a, w);
-    if (a.dtype == DSPARK_BF16) return launch_draft_tc(a, w, f, st);
+    // bf16: more than 128 requests (and every RNN-head round) on CTA pairs.
+    if (a.dtype == DSPARK_BF16)
+        return (a.B > 128 || a.H_out != nullptr) ? launch_draft_pair(a, w, f, st) : launch_draft_tc(a, w, f, st);
     cudaError_t e;
     for (int pos = 0; pos < a.G; ++pos) {
         dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);

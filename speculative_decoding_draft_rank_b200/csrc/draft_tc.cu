@@ -67,17 +67,20 @@ struct TcLayout {
 };
 
 // Every epilogue warp group owns one logit slot (segment sg of each tile goes
-// to slot sg), so a group only ever waits on phases of its own slot; the B
-// ring takes what shared memory is left (3 stages for r <= 256, 1 for r = 512).
-__host__ __device__ inline TcLayout tc_layout(int r) {
+// to slot sg), so a group only ever waits on phases of its own slot (drafting
+// only; the residual pass reads its rows from global memory); the B ring takes
+// what shared memory is left (3 stages for r <= 256, 1 for r = 512).  With the
+// RNN head's rows (residual pass only) A holds a high and a low bf16 part.
+__host__ __device__ inline TcLayout tc_layout(int r, int mode, int rnn) {
     TcLayout t;
     t.nkb = (r + kKB - 1) / kKB;
-    t.sL = kSegs;
-    const int fixed = t.nkb * kABlockBytes + t.sL * kSegBytes + 256 + 1024;
+    t.sL = mode == 0 ? kSegs : 0;
+    const int na = t.nkb * (rnn ? 2 : 1);
+    const int fixed = na * kABlockBytes + t.sL * kSegBytes + 256 + 1024;
     int sB = (227 * 1024 - fixed) / kStageBytes;
     t.sB = sB > 3 ? 3 : (sB < 1 ? 1 : sB);   // B ring depth
     t.a_off = 0;
-    t.b_off = t.a_off + t.nkb * kABlockBytes;
+    t.b_off = t.a_off + na * kABlockBytes;
     t.l_off = t.b_off + t.sB * kStageBytes;
     t.bar_off = t.l_off + t.sL * kSegBytes;
     t.total = t.bar_off + 256 + 1024;   // barriers, base alignment
@@ -90,12 +93,14 @@ enum { kEpiDraft = 0, kEpiResidual = 1 };
 struct TcEpi {
     const float *temp;
     int B, G, V, nParts;
+    long long budget;         // clock budget of the bounded waits (drains keep their own)
     WsHeader *hdr;
     FinArgs fin;              // drafting: the per-row finalize of every position
     uint32_t *grid_count;     // drafting: grid-barrier counter (zeroed before the launch)
     const __nv_bfloat16 *U;   // [V, r]: A-operand rows are U[previous token]
     const int32_t *x0;        // [B] last committed tokens
     const int32_t *x;         // [B, G] draft tokens (drafting: earlier positions of this call)
+    const float *H;           // residual, RNN head: the states [B, G, r] (A rows split high/low); else null
     const __nv_bfloat16 *L;   // drafting and residual: backbone logits [B, G, V]
     // drafting: 64-column partials per request row
     float *part_m, *part_s;
@@ -116,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                                                               int nTilesN, const TcEpi ep)
 {
     extern __shared__ unsigned char smem_raw[];
-    const TcLayout lay = tc_layout(r);
+    const int rnn = (MODE == kEpiResidual && ep.H != nullptr) ? 1 : 0;
+    const TcLayout lay = tc_layout(r, MODE, rnn);
     const uint32_t raw_u32 = tc::smem_u32(smem_raw);
     unsigned char *base = smem_raw + (((raw_u32 + 1023) & ~1023u) - raw_u32);
     unsigned char *sA = base + lay.a_off;
@@ -141,14 +147,18 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     const int B = ep.B, V = ep.V, nParts = ep.nParts;
     const int npos = (MODE == kEpiDraft) ? ep.G : 1;
     WsHeader *hdr = ep.hdr;
-    const int nMB = (B + kM - 1) / kM;
+    // Residual rows are counted on the device: the CTAs split over the
+    // M-blocks that hold queued rows only, so a round with at most 128
+    // rejections runs every CTA on one M-block.
+    const int nrows = (MODE == kEpiResidual) ? (int)*reinterpret_cast<const volatile uint32_t *>(ep.nrows) : B;
+    if (nrows <= 0) return;
+    const int nMB = (nrows + kM - 1) / kM;
     const int mb = blockIdx.x % nMB;
     const int m0 = mb * kM;
     const int first_tile = blockIdx.x / nMB;
     const int tile_step = ((int)gridDim.x - mb + nMB - 1) / nMB;
-    // Residual rows are counted on the device: m-blocks past the count leave now.
-    const int nrows = (MODE == kEpiResidual) ? (int)*reinterpret_cast<const volatile uint32_t *>(ep.nrows) : B;
-    if (m0 >= nrows) return;
+    // (Drafting grids never exceed the tile count: every CTA meets the grid barriers.)
+    if (MODE == kEpiResidual && first_tile >= nTilesN) return;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(a_full, 1);
@@ -179,12 +189,12 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             for (int pos = 0; pos < npos && ok; ++pos) {
             // Later positions stream only after the round's finalize, whose
             // dependent loads would otherwise queue behind this prefetch.
-            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, kWaitBudget);
+            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 const int n0 = t * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % SB;
-                    if (!tc::mbar_wait_bounded(&b_empty[s], ((g / SB) & 1) ^ 1, abort_flag, kWaitBudget)) {
+                    if (!tc::mbar_wait_bounded(&b_empty[s], ((g / SB) & 1) ^ 1, abort_flag, ep.budget)) {
                         ok = false;
                         break;
                     }
@@ -213,11 +223,11 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             bool ok = true;
             int g = 0, j = 0;
             for (int pos = 0; pos < npos && ok; ++pos) {
-            ok = tc::mbar_wait_bounded(a_full, pos & 1, abort_flag, kWaitBudget);
+            ok = tc::mbar_wait_bounded(a_full, pos & 1, abort_flag, ep.budget);
             tc::tc_fence_after();
             for (int t = first_tile; t < nTilesN && ok; t += tile_step, ++j) {
                 const int ab = j & 1;
-                if (!tc::mbar_wait_bounded(&acc_empty[ab], ((j >> 1) & 1) ^ 1, abort_flag, kWaitBudget)) {
+                if (!tc::mbar_wait_bounded(&acc_empty[ab], ((j >> 1) & 1) ^ 1, abort_flag, ep.budget)) {
                     ok = false;
                     break;
                 }
@@ -225,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 const uint32_t d = tmem_base + ab * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
                     const int s = g % SB;
-                    if (!tc::mbar_wait_bounded(&b_full[s], (g / SB) & 1, abort_flag, kWaitBudget)) {
+                    if (!tc::mbar_wait_bounded(&b_full[s], (g / SB) & 1, abort_flag, ep.budget)) {
                         ok = false;
                         break;
                     }
@@ -235,6 +245,10 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                         const uint64_t ad = tc::sw128_desc(a_addr + kb * kABlockBytes + kk * 32);
                         const uint64_t bd = tc::sw128_desc(b_addr + s * kStageBytes + kk * 32);
                         tc::mma_bf16(d, ad, bd, idesc, (kb | kk) != 0);
+                        if (rnn) {
+                            const uint64_t al = tc::sw128_desc(a_addr + (nkb + kb) * kABlockBytes + kk * 32);
+                            tc::mma_bf16(d, al, bd, idesc, 1u);
+                        }
                     }
                     tc::mma_commit(&b_empty[s]);
                 }
@@ -256,11 +270,11 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             int g = 0;
             bool ok = true;
             for (int pos = 0; pos < npos && ok; ++pos) {
-            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, kWaitBudget);
+            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 for (int sg = 0; sg < kSegs; ++sg, ++g) {
                     const int q = g % SL;
-                    if (!tc::mbar_wait_bounded(&l_empty[q], ((g / SL) & 1) ^ 1, abort_flag, kWaitBudget)) {
+                    if (!tc::mbar_wait_bounded(&l_empty[q], ((g / SL) & 1) ^ 1, abort_flag, ep.budget)) {
                         ok = false;
                         break;
                     }
@@ -310,6 +324,42 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             epi_sync();
             if (leader) tc::mbar_arrive(a_full);
         };
+        // RNN head's rows: the fp32 state h (row `row` of A) split into bf16
+        // high parts (k-blocks 0..nkb-1) and low parts (nkb..2nkb-1).
+        auto gather_A_state = [&](const float *hrow) {
+            for (int kb = sg; kb < nkb; kb += kSegs) {
+                unsigned char *dhi = sA + kb * kABlockBytes + row * 128;
+                unsigned char *dlo = sA + (nkb + kb) * kABlockBytes + row * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const int k = kb * kKB + c * 8;
+                    float h8[8];
+                    if (hrow != nullptr && k < r) {
+                        const float4 p0 = *reinterpret_cast<const float4 *>(hrow + k);
+                        const float4 p1 = *reinterpret_cast<const float4 *>(hrow + k + 4);
+                        h8[0] = p0.x; h8[1] = p0.y; h8[2] = p0.z; h8[3] = p0.w;
+                        h8[4] = p1.x; h8[5] = p1.y; h8[6] = p1.z; h8[7] = p1.w;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) h8[e] = 0.f;
+                    }
+                    uint32_t hi4[4], lo4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const __nv_bfloat16 a0 = __float2bfloat16_rn(h8[2 * e]), a1 = __float2bfloat16_rn(h8[2 * e + 1]);
+                        const __nv_bfloat16 b0 = __float2bfloat16_rn(h8[2 * e] - __bfloat162float(a0));
+                        const __nv_bfloat16 b1 = __float2bfloat16_rn(h8[2 * e + 1] - __bfloat162float(a1));
+                        hi4[e] = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(a1) << 16);
+                        lo4[e] = (uint32_t)__bfloat16_as_ushort(b0) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+                    }
+                    *reinterpret_cast<uint4 *>(dhi + ((c ^ (row & 7)) << 4)) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                    *reinterpret_cast<uint4 *>(dlo + ((c ^ (row & 7)) << 4)) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+                }
+            }
+            tc::fence_proxy_async_smem();
+            epi_sync();
+            if (leader) tc::mbar_arrive(a_full);
+        };
         if (MODE == kEpiDraft) {
             // ------------------------------------------ drafting epilogue
             // One online pass per 32-column chunk: y = L + Delta, chunk max,
@@ -337,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                         atomicAdd(ep.grid_count, 1u);
                         const long long t0 = clock64();
                         while (tc::ld_acquire_gpu(ep.grid_count) < target) {
-                            if (*abort_flag || clock64() - t0 > kWaitBudget) { ok = false; break; }
+                            if (*abort_flag || clock64() - t0 > ep.budget) { ok = false; break; }
                             __nanosleep(32);
                         }
                     }
@@ -378,8 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const int gl = j * kSegs + sg, q = gl % SL;
                     // Every lane waits; the vote keeps the warp converged for the
                     // warp-collective TMEM loads below even if the budget runs out.
-                    bool ok = tc::mbar_wait_bounded(&l_full[q], (gl / SL) & 1, abort_flag, kWaitBudget);
-                    ok = ok && tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
+                    bool ok = tc::mbar_wait_bounded(&l_full[q], (gl / SL) & 1, abort_flag, ep.budget);
+                    ok = ok && tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, ep.budget);
                     if (!__all_sync(0xffffffffu, ok)) break;
                     tc::tc_fence_after();
                     // This thread's 64 logits: one 128-byte row of the swizzled segment.
@@ -483,7 +533,12 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                 }
             }
         } else {
-            {
+            if (rnn) {
+                const int sidx = m0 + row;
+                const float *hrow = nullptr;
+                if (sidx < nrows) hrow = ep.H + ((size_t)ep.res_b[sidx] * ep.G + ep.res_k[sidx]) * r;
+                gather_A_state(hrow);
+            } else {
                 int prev = 0;
                 const int sidx = m0 + row;
                 if (sidx < nrows) {
@@ -513,7 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             for (int t = first_tile; t < nTilesN; t += tile_step, ++j) {
                 const int ab = j & 1;
                 const int cbase = t * kBN + sg * kSeg;
-                const bool ok = tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, kWaitBudget);
+                const bool ok = tc::mbar_wait_bounded(&acc_full[ab], (j >> 1) & 1, abort_flag, ep.budget);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 tc::tc_fence_after();
                 const uint32_t taddr = tmem_base + lane_addr + ab * kBN + sg * kSeg;
@@ -636,7 +691,7 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, const void 
     } else {
         mE = mW;   // unused
     }
-    const TcLayout lay = tc_layout(r);
+    const TcLayout lay = tc_layout(r, MODE, (MODE == kEpiResidual && ep.H != nullptr) ? 1 : 0);
     cudaError_t e = cudaFuncSetAttribute(markov_tile_tc<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)lay.total);
     if (e != cudaSuccess) return e;
@@ -677,6 +732,7 @@ cudaError_t launch_markov_tc(const void *Wt, int r, const TcEpi &ep, const void 
 cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs &f, cudaStream_t st) {
     TcEpi ep{};
     ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.nParts = w.nTiles; ep.hdr = w.hdr;
+    ep.budget = wait_budget(kWaitBudget);
     ep.U = static_cast<const __nv_bfloat16 *>(a.U); ep.x0 = a.x0; ep.x = a.x_out;
     ep.L = static_cast<const __nv_bfloat16 *>(a.L);
     ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
@@ -688,8 +744,10 @@ cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs 
 cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st) {
     TcEpi ep{};
     ep.temp = a.temp; ep.B = a.B; ep.G = a.G; ep.V = a.V; ep.nParts = a.nParts; ep.hdr = a.hdr;
+    ep.budget = wait_budget(kWaitBudget);
     ep.U = a.U; ep.x0 = a.x0; ep.x = a.x; ep.L = a.L;
     ep.nrows = a.nrows; ep.res_b = a.res_b; ep.res_k = a.res_k; ep.res_mt = a.res_mt; ep.res_zt = a.res_zt;
+    ep.H = a.H;
     ep.rowmax = a.rowmax; ep.rowsum = a.rowsum; ep.Tlog = a.Tlog; ep.rp = a.rp;
     return launch_markov_tc<kEpiResidual>(a.Wt, a.r, ep, nullptr, st);
 }

@@ -78,7 +78,13 @@ struct FinArgs {
     const int32_t *part_a;
     int32_t *x_out;
     float *pd_out, *rowmax_out, *rowsum_out;
-    __nv_bfloat16 *E;              // bf16 rounds: U[x_i] rows staged for position i + 1, else null
+    __nv_bfloat16 *E;              // bf16 rounds: the next position's A rows staged for TMA, else null
+    // RNN head (null for the Markov head): the recurrent matrix Arec [r, r]
+    // and the states H [B, G, r] fp32 (row b*G + i holds the state that
+    // biases position i); E then holds the next state split into bf16 high
+    // parts (rows 0..B-1) and low parts (rows B..2B-1).
+    const __nv_bfloat16 *Arec;
+    float *H;
     WsHeader *hdr;
 };
 
@@ -93,15 +99,33 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     const T *L = static_cast<const T *>(a.L);
     const T *U = static_cast<const T *>(a.U);
     const T *Wt = static_cast<const T *>(a.Wt);
-    const int G = a.G, V = a.V, r = a.r, nTiles = a.nTiles, TN = a.TN;
+    const int B = a.B, G = a.G, V = a.V, r = a.r, nTiles = a.nTiles, TN = a.TN;
     const int tid = g.tid, nthr = g.n;
     const size_t ro = (size_t)b * G + pos;
-    // bf16 rounds: the sampled token's U row is staged in E[b] for the next
-    // position's tensor-core pass (16-byte pieces; r is a multiple of 16).
+    // bf16 rounds: the next position's A row is staged in E for its
+    // tensor-core pass.  Markov head: the sampled token's U row (16-byte
+    // pieces; r is a multiple of 16).  RNN head: the next state
+    // h' = tanh(h A + U[x]) from this position's state h (in urow), written
+    // to H and split into bf16 high and low parts (h' = hi + lo to about 2^-17
+    // relative, so two MMAs reproduce the fp32 state's product).
     auto stage_next = [&](int x) {
-        if (a.E != nullptr && pos + 1 < G)
+        if (a.E == nullptr || pos + 1 >= G) return;
+        if (a.H == nullptr) {
             for (int q = tid; q < r / 8; q += nthr)
                 reinterpret_cast<uint4 *>(a.E + (size_t)b * r)[q] = ld_nc16(U + (size_t)x * r + q * 8);
+            return;
+        }
+        for (int c = tid; c < r; c += nthr) {
+            float acc = 0.f;
+#pragma unroll 8
+            for (int q = 0; q < r; ++q) acc = fmaf(urow[q], __bfloat162float(a.Arec[(size_t)q * r + c]), acc);
+            acc += ld_elem(U, (size_t)x * r + c);
+            const float hn = tanhf(acc);
+            a.H[(ro + 1) * r + c] = hn;
+            const __nv_bfloat16 hi = __float2bfloat16_rn(hn);
+            a.E[(size_t)b * r + c] = hi;
+            a.E[((size_t)B + b) * r + c] = __float2bfloat16_rn(hn - __bfloat162float(hi));
+        }
     };
     const float *pm = a.part_m + (size_t)b * nTiles;
     const float *ps = a.part_s + (size_t)b * nTiles;
@@ -128,11 +152,21 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     }
     const float Tb = sane_temp(a.temp[b], a.hdr);
     const float u = a.u_draft[ro];
-    const int prev = (pos == 0) ? clamp_token(a.x0[b], V, a.hdr) : a.x_out[(size_t)b * G + pos - 1];
-    // The previous token's U row (r <= 512 = 2 x 256 threads), kept in
-    // registers until after the first barrier.
-    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
-    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+    // This position's A row in fp32 (r <= 512 = 2 x 256 threads): the
+    // previous token's U row (Markov head) or the state h (RNN head).  It is
+    // published to urow by the first group barrier below.
+    float uv0, uv1;
+    if (a.H != nullptr) {
+        const float *hrow = a.H + ro * r;
+        uv0 = tid < r ? hrow[tid] : 0.f;
+        uv1 = tid + nthr < r ? hrow[tid + nthr] : 0.f;
+    } else {
+        const int prev = (pos == 0) ? clamp_token(a.x0[b], V, a.hdr) : a.x_out[(size_t)b * G + pos - 1];
+        uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
+        uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+    }
+    if (tid < r) urow[tid] = uv0;
+    if (tid + nthr < r) urow[tid + nthr] = uv1;
 
     float m = -INFINITY;
 #pragma unroll
@@ -169,10 +203,8 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
 #pragma unroll
     for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
     for (int t = t0 + kFinChunk; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
-    if (tid < r) urow[tid] = uv0;
-    if (tid + nthr < r) urow[tid + nthr] = uv1;
     float Z;
-    const float incl = grp_scan1(g, loc, sc->s_loc, &Z);   // also publishes urow
+    const float incl = grp_scan1(g, loc, sc->s_loc, &Z);
     const float target = u * Z;
     // The first thread whose inclusive prefix passes u Z owns the crossing
     // (the last thread with mass if rounding left u Z at the top).
@@ -215,6 +247,16 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     const int col = c0 + tid / tpc, part = tid % tpc;
     const bool mine = part == 0 && col < V;
     const float lval = mine ? ld_elem(L, ro * V + col) : 0.f;   // issued with the factor loads
+    // The token is one of these columns: its U row (read to stage the next
+    // position) is brought into L2 while the columns are recomputed.
+    if (a.E != nullptr && pos + 1 < G) {
+        const int nl = (r * (int)sizeof(T) + 127) / 128;   // 128-byte lines per U row
+        for (int q = tid; q < TN * nl; q += nthr) {
+            const int cc = c0 + q / nl;
+            if (cc < V)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(U + (size_t)cc * r + (q % nl) * (128 / sizeof(T))));
+        }
+    }
     float dl = 0.f;
     if (col < V) dl = dot_part(urow, Wt + (size_t)col * r, r, part, tpc);
     for (int o = tpc >> 1; o > 0; o >>= 1) dl += __shfl_xor_sync(0xffffffffu, dl, o);

@@ -1,11 +1,25 @@
 // kernels.cuh -- launch interfaces shared by the stage files of the library.
 #pragma once
 
+#include <cstdlib>
+
 #include "common.cuh"
 
 namespace dspark {
 
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Clock budget of the bounded device waits of a launch: `dflt`, or the cycle
+// count in the environment variable DSPARK_WAIT_BUDGET_CYCLES when it is set
+// to a positive number (a failure-path test hook: a budget of a few hundred
+// cycles makes the first real wait run out).  Read when the launch is
+// enqueued, so a captured graph keeps the value of its capture.
+inline long long wait_budget(long long dflt) {
+    const char *e = getenv("DSPARK_WAIT_BUDGET_CYCLES");
+    if (e == nullptr || *e == 0) return dflt;
+    const long long v = atoll(e);
+    return v > 0 ? v : dflt;
+}
 inline int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Columns per partial (max, sum, argmax) of the bf16 tensor-core drafting kernel.
@@ -19,6 +33,8 @@ struct DraftArgs {
     int B, G, V, r, dtype;
     int32_t *x_out;
     float *pd_out, *rowmax_out, *rowsum_out;
+    const void *Arec = nullptr;   // RNN head: recurrent matrix [r, r] (bf16); null for the Markov head
+    float *H_out = nullptr;       // RNN head: states [B, G, r] fp32
 };
 
 struct DraftWs {
@@ -37,6 +53,8 @@ cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st);
 struct FinArgs;
 // bf16 rounds: every position in one cooperative launch of the tensor-core kernel.
 cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs &f, cudaStream_t st);
+// bf16 rounds of more than 128 requests: the same on CTA pairs (M = 256 MMAs).
+cudaError_t launch_draft_pair(const DraftArgs &a, const DraftWs &w, const FinArgs &f, cudaStream_t st);
 
 // --------------------------------------------------------------- confidence
 cudaError_t launch_confidence(const void *h, const void *w, float bias, const float *tau, int B,
@@ -53,6 +71,7 @@ cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n
 struct VerifyArgs {
     const void *Tlog, *L, *U, *Wt;
     const int32_t *x0, *x;
+    const float *H;   // RNN head: the drafting states [B, G, r]; null for the Markov head (U, x0 used)
     const float *pd_x, *rowmax, *rowsum, *temp, *u_accept, *u_final;
     const int32_t *ell;
     int B, G, V, r, dtype;
@@ -67,6 +86,7 @@ struct ResidualTcArgs {
     const void *Wt;
     const __nv_bfloat16 *U, *L, *Tlog;
     const int32_t *x0, *x;
+    const float *H;   // RNN head: states [B, G, r] (the A rows), else null
     const float *temp, *rowmax, *rowsum, *res_mt, *res_zt;
     const int32_t *res_b, *res_k;
     const uint32_t *nrows;

@@ -11,6 +11,7 @@
 // array of fixed size that every GPU loading this library holds until exit.
 #include <mutex>
 
+#include "abi_util.cuh"
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -51,14 +52,12 @@ dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const vo
                                           const float *temp, const float *u_draft, int B, int G, int V,
                                           int r, int dtype, int32_t *x_out, float *pd_x_out,
                                           float *rowmax_out, float *rowsum_out, void *stream) {
-    if (dtype != DSPARK_F32 && dtype != DSPARK_BF16) return DSPARK_ERR_UNSUPPORTED_DTYPE;
-    if (B < 1 || B > 4096 || G < 1 || G > 16 || V < 2 || V > (1 << 20) || r < 1 || r > 512)
-        return DSPARK_ERR_INVALID_ARG;
-    if (dtype == DSPARK_BF16 && ((r % 16) != 0 || (V % 8) != 0)) return DSPARK_ERR_INVALID_ARG;
+    if (dspark_status s = dspark::injected("dspark_draft_markov_noalloc")) return s;
+    if (dspark_status s = dspark::check_common(B, G, V, r, dtype)) return s;
     if (!L || !U || !Wt || !x0 || !temp || !u_draft || !x_out || !pd_x_out || !rowmax_out || !rowsum_out)
         return DSPARK_ERR_INVALID_ARG;
-    const auto a16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-    if (dtype == DSPARK_BF16 && !(a16(L) && a16(U) && a16(Wt))) return DSPARK_ERR_INVALID_ARG;
+    if (dtype == DSPARK_BF16 && !(dspark::aligned16(L) && dspark::aligned16(U) && dspark::aligned16(Wt)))
+        return DSPARK_ERR_INVALID_ARG;
     if (dspark::draft_ws_bytes(B, G, V, r, dtype) > kNoAllocScratchBytes) return DSPARK_ERR_WORKSPACE;
     void *ws = nullptr;
     if (dspark_status s = scratch_address(&ws)) return s;
@@ -69,6 +68,20 @@ dspark_status dspark_draft_markov_noalloc(const void *L, const void *U, const vo
     if (cudaMemsetAsync(ws, 0, sizeof(dspark::WsHeader), st) != cudaSuccess) return DSPARK_ERR_CUDA;
     dspark::DraftArgs a{L, U, Wt, x0, temp, u_draft, B, G, V, r, dtype, x_out, pd_x_out, rowmax_out, rowsum_out};
     return dspark::launch_draft(a, ws, st) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+dspark_status dspark_draft_noalloc_device_status(void *stream, uint32_t *status_out) {
+    if (status_out == nullptr) return DSPARK_ERR_INVALID_ARG;
+    void *ws = nullptr;
+    if (dspark_status s = scratch_address(&ws)) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    // Stream order: the word of the last call enqueued on `stream` (calls on
+    // other streams must have been ordered before it by the caller).
+    if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSPARK_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSPARK_ERR_CUDA;
+    *status_out = v;
+    return DSPARK_OK;
 }
 
 }  // extern "C"

@@ -11,9 +11,9 @@
 // Launch sequence (fixed, graph-capturable; work counts live on the device):
 //   plan        1 CTA: row list of the admitted target rows, rows (b, k) for
 //               k = 0..ell_b (0-based), and their offsets per request.
-//   rows        persistent grid over (row, 8192-column chunk) work items,
-//               one warp per item (bf16: 32-byte loads two steps ahead):
-//               one streaming pass over each target row,
+//   rows        persistent grid over (row, 8192-column chunk) work items
+//               (bf16: chunks staged in shared memory by bulk copies, a ring
+//               of eight per SM): one streaming pass over each target row,
 //               giving per chunk the max, lowest argmax and sum of
 //               exp((t - max) / T).
 //   decide      1 CTA per request: row max / Z from the chunk partials,
@@ -245,125 +245,200 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
     }
 }
 
-// bf16 rows: one warp per (row, 8192-column chunk) work item, no block
-// barriers.  The warp walks its chunk in eight 1024-column steps; lane l owns
-// columns [l * 32, l * 32 + 32) of a step, read with two 32-byte loads (four
-// 16-byte ones when rows are not 32-byte aligned) issued two steps ahead.
-// Each lane keeps an online (max, sum of exp((t - max) / T)) -- or, for a
-// greedy row, the lowest argmax -- and a warp merge writes the chunk partial.
-constexpr int kRowsWarpThreads = 256;
-constexpr int kStep = 1024;                 // columns per warp step
-constexpr int kSteps = kChunk / kStep;      // 8
+// bf16 rows: persistent CTAs (one per SM) over the (row, 8192-column chunk)
+// work items, item q of CTA c being item c + q * grid.  One producer thread
+// streams the CTA's items into a ring of shared-memory stages with bulk copies
+// (evict-first: every target row is read once, so the transition factor that
+// drafting left in L2 stays there for the residual pass) and writes each
+// stage's item description beside it; eight consumer warps reduce a staged
+// chunk together (warp w: columns [w * 1024, w * 1024 + 1024), lane l reading
+// 16-byte pieces l, l + 32, ... of that range, bank-conflict free), release the
+// stage as soon as its values are in registers, and merge their (max, sum of
+// exp((t - max) / T), lowest argmax) after one named barrier.
+constexpr int kVrStages = 8;
+constexpr int kVrWarps = 8;
+constexpr int kVrThreads = (kVrWarps + 1) * 32;
+constexpr int kVrStageBytes = kChunk * 2;
+constexpr long long kVrWaitBudget = 4000000000LL;   // ~2 s of SM clock
 
-// 32 bf16 of a row from column c (c a multiple of 32) into w; past n reads as
-// -inf (bf16 0xff80).
-__device__ __forceinline__ void ld_row32(const __nv_bfloat16 *row, int c, int n, bool a32, uint32_t (&w)[16]) {
-    const __nv_bfloat16 *p = row + c;
-    if (a32 && c + 32 <= n) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(w[h * 8 + 0]), "=r"(w[h * 8 + 1]), "=r"(w[h * 8 + 2]), "=r"(w[h * 8 + 3]),
-                           "=r"(w[h * 8 + 4]), "=r"(w[h * 8 + 5]), "=r"(w[h * 8 + 6]), "=r"(w[h * 8 + 7])
-                         : "l"(p + h * 16));
-    } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            if (c + q * 8 + 8 <= n && ((reinterpret_cast<uintptr_t>(p + q * 8) & 15) == 0)) {
-                const uint4 v = ld_stream16(p + q * 8);
-                w[q * 4 + 0] = v.x; w[q * 4 + 1] = v.y; w[q * 4 + 2] = v.z; w[q * 4 + 3] = v.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int i0 = c + q * 8 + e * 2;
-                    const uint32_t lo = i0 < n ? (uint32_t)__bfloat16_as_ushort(p[q * 8 + e * 2]) : 0xff80u;
-                    const uint32_t hi = i0 + 1 < n ? (uint32_t)__bfloat16_as_ushort(p[q * 8 + e * 2 + 1]) : 0xff80u;
-                    w[q * 4 + e] = lo | (hi << 16);
-                }
-            }
-        }
-    }
-}
+struct VrMeta {
+    int j, c, ncols;
+    float cexp;
+};
 
-__global__ void __launch_bounds__(kRowsWarpThreads, 3) verify_rows_warp(const __nv_bfloat16 *__restrict__ Tlog,
-                                                                     const float *__restrict__ temp, int G, int V,
-                                                                     VerifyWs w) {
-    const int lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfloat16 *__restrict__ Tlog,
+                                                                 const float *__restrict__ temp, int G, int V,
+                                                                 VerifyWs w, long long budget) {
+    extern __shared__ __align__(128) unsigned char vr_smem[];
+    unsigned char *stages = vr_smem;                                                // [S][16 KB]
+    uint64_t *full = reinterpret_cast<uint64_t *>(vr_smem + kVrStages * kVrStageBytes);
+    uint64_t *empty = full + kVrStages;
+    VrMeta *meta = reinterpret_cast<VrMeta *>(empty + kVrStages);                   // [S]
+    __shared__ float pm[2][kVrWarps], ps[2][kVrWarps];
+    __shared__ int pa[2][kVrWarps];
+    __shared__ int abort_s;
+    __shared__ int stop_s[2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
     const int nwork = nrows * w.nChunks;
-    const int nwarps = gridDim.x * (blockDim.x >> 5);
-    const bool a32 = (V & 15) == 0 && (reinterpret_cast<uintptr_t>(Tlog) & 31) == 0;
-    for (int item = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); item < nwork; item += nwarps) {
-        const int j = item / w.nChunks, c = item - j * w.nChunks;
-        const int rk = w.rows[j], b = rk >> 5, kk = rk & 31;
-        const __nv_bfloat16 *row = Tlog + ((size_t)b * (G + 1) + kk) * V;
-        float Tb = temp[b];
-        Tb = Tb >= 0.f ? Tb : 0.f;
-        const float cexp = Tb > 0.f ? kLog2e / Tb : 0.f;
-        const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
-        uint32_t buf[2][16];
-        ld_row32(row, c0 + lane * 32, c1, a32, buf[0]);
-        ld_row32(row, c0 + kStep + lane * 32, c1, a32, buf[1]);
-        float m = -INFINITY, s = 0.f;
-        int am = 0x7fffffff;
-#pragma unroll
-        for (int st = 0; st < kSteps; ++st) {
-            // The step's 32 values stay packed (two bf16 per word) and are
-            // widened where used, which keeps the lane under 80 registers.
-            uint32_t v[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = buf[st & 1][i];
-            if (st + 2 < kSteps) ld_row32(row, c0 + (st + 2) * kStep + lane * 32, c1, a32, buf[st & 1]);
-            // Step maximum: four running three-input maxima over the value pairs.
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int i = 0; i < 16; ++i) m4[i & 3] = max3(m4[i & 3], bf16lo(v[i]), bf16hi(v[i]));
-            const float cm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            const int base = c0 + st * kStep + lane * 32;
-            if (cexp == 0.f) {   // greedy row: the lowest index of the largest value (warp-uniform)
-                if (cm > m) {
-                    int ix = 0;
-#pragma unroll
-                    for (int i = 15; i >= 0; --i) {
-                        if (bf16hi(v[i]) == cm) ix = 2 * i + 1;
-                        if (bf16lo(v[i]) == cm) ix = 2 * i;
+    if ((int)blockIdx.x >= nwork) return;
+    const int nmine = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    if (threadIdx.x == 0) {
+        for (int q = 0; q < kVrStages; ++q) { tc::mbar_init(&full[q], 1); tc::mbar_init(&empty[q], kVrWarps); }
+        abort_s = 0;
+        stop_s[0] = stop_s[1] = 0;
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
+    volatile int *abort_flag = &abort_s;
+
+    if (warp == kVrWarps) {
+        // ------------------------------------------------------ producer
+        // The warp loads the item descriptions 32 at a time (row ids, then
+        // temperatures); lane 0 issues the copies.
+        const uint64_t pol = tc::policy_evict_first();
+        bool ok = true;
+        int q = 0;
+        for (int q0 = 0; q0 < nmine && ok; q0 += 32) {
+            const int ql = q0 + lane;
+            int rk = 0, c = 0, j = 0;
+            float Tb = 0.f;
+            if (ql < nmine) {
+                const int item = (int)blockIdx.x + ql * (int)gridDim.x;
+                j = item / w.nChunks;
+                c = item - j * w.nChunks;
+                rk = w.rows[j];
+                Tb = temp[rk >> 5];
+            }
+            const int nb = min(32, nmine - q0);
+            for (int i = 0; i < nb; ++i, ++q) {
+                const int rki = __shfl_sync(0xffffffffu, rk, i);
+                const int ci = __shfl_sync(0xffffffffu, c, i);
+                const int ji = __shfl_sync(0xffffffffu, j, i);
+                const float Ti = __shfl_sync(0xffffffffu, Tb, i);
+                if (lane == 0) {
+                    const int s = q % kVrStages;
+                    ok = tc::mbar_wait_bounded(&empty[s], ((q / kVrStages) & 1) ^ 1, abort_flag, budget);
+                    if (ok) {
+                        const int c0 = ci * kChunk, ncols = min(kChunk, V - c0);
+                        const float T = Ti >= 0.f ? Ti : 0.f;
+                        meta[s] = VrMeta{ji, ci, ncols, T > 0.f ? kLog2e / T : 0.f};
+                        const __nv_bfloat16 *src =
+                            Tlog + ((size_t)(rki >> 5) * (G + 1) + (rki & 31)) * V + c0;
+                        tc::mbar_arrive_expect_tx(&full[s], (uint32_t)ncols * 2);
+                        tc::bulk_load(stages + s * kVrStageBytes, src, (uint32_t)ncols * 2, &full[s], pol);
                     }
-                    am = base + ix;
-                    m = cm;
                 }
-            } else if (cm > -INFINITY) {
-                // exp((t - mn) / T) = 2^(t * cexp - mn * cexp): one fused
-                // multiply-add per column.
-                const float mn = fmaxf(m, cm);
-                const float nmc = -mn * cexp;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    a4[(2 * i) & 3] += fast_exp2(fmaf(bf16lo(v[i]), cexp, nmc));
-                    a4[(2 * i + 1) & 3] += fast_exp2(fmaf(bf16hi(v[i]), cexp, nmc));
-                }
-                s = (m == -INFINITY ? 0.f : s * fast_exp2((m - mn) * cexp)) + ((a4[0] + a4[1]) + (a4[2] + a4[3]));
-                m = mn;
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
             }
         }
-        // Warp merge of (m, s, argmax) in lane order.
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float om = __shfl_xor_sync(0xffffffffu, m, o);
-            const float os = __shfl_xor_sync(0xffffffffu, s, o);
-            const int oa = __shfl_xor_sync(0xffffffffu, am, o);
-            const float nm = fmaxf(m, om);
-            if (cexp > 0.f)
-                s = (m > -INFINITY ? s * fast_exp2((m - nm) * cexp) : 0.f) +
-                    (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
-            if (om > m || (om == m && oa < am)) am = oa;
-            m = nm;
+        if (!ok && lane == 0) {
+            // Give up: wait (bounded, ignoring the abort flag) for the copies
+            // in flight so that none lands after the CTA exits.
+            int dummy = 0;
+            for (int d = 0; d < kVrStages && q - 1 - d >= 0; ++d) {
+                const int qq = q - 1 - d;
+                tc::mbar_wait_bounded(&full[qq % kVrStages], (qq / kVrStages) & 1, &dummy, kVrWaitBudget / 4);
+            }
+            flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
         }
-        if (lane == 0) {
-            const size_t o = (size_t)j * w.nChunks + c;
-            w.cm[o] = m;
-            w.cs[o] = s;
-            w.ca[o] = am;
+    } else {
+        // ------------------------------------------------------ consumers
+        // A warp whose wait ran out raises stop[q & 1] before the item's
+        // named barrier, and every consumer warp leaves after that barrier
+        // when it is set; the flags only ever go from 0 to 1, and
+        // alternate by item parity, so all eight warps take the same exit.
+        for (int q = 0; q < nmine; ++q) {
+            const int s = q % kVrStages;
+            const int par = q & 1;
+            bool ok = tc::mbar_wait_bounded(&full[s], (q / kVrStages) & 1, abort_flag, budget);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                if (lane == 0) {
+                    stop_s[par] = 1;
+                    *abort_flag = 1;
+                    flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(kVrWarps * 32) : "memory");
+                break;
+            }
+            const VrMeta md = meta[s];
+            uint4 v[4];
+            const unsigned char *src = stages + s * kVrStageBytes + warp * 2048 + lane * 16;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[s]);   // the values are in registers
+            // Column of piece i, element e: base + i * 256 + e.
+            const int base = warp * 1024 + lane * 8;
+            float t[32];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    t[i * 8 + 2 * h] = bf16lo(ww[h]);
+                    t[i * 8 + 2 * h + 1] = bf16hi(ww[h]);
+                }
+            }
+            if (md.ncols < kChunk) {   // the row's last chunk: columns past V are -inf
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (base + i * 256 + e >= md.ncols) t[i * 8 + e] = -INFINITY;
+            }
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) m4[(e >> 1) & 3] = max3(m4[(e >> 1) & 3], t[e], t[e + 1]);
+            float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            float sum = 0.f;
+            int am = 0x7fffffff;
+            const float cexp = md.cexp;
+            if (cexp == 0.f) {   // greedy row (warp-uniform): the lowest index of the largest value
+#pragma unroll
+                for (int i = 3; i >= 0; --i)
+#pragma unroll
+                    for (int e = 7; e >= 0; --e)
+                        if (t[i * 8 + e] == m) am = md.c * kChunk + base + i * 256 + e;
+            } else if (m > -INFINITY) {
+                const float nmc = -m * cexp;
+                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2(fmaf(t[e], cexp, nmc));
+                sum = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float om = __shfl_xor_sync(0xffffffffu, m, o);
+                const float os = __shfl_xor_sync(0xffffffffu, sum, o);
+                const int oa = __shfl_xor_sync(0xffffffffu, am, o);
+                const float nm = fmaxf(m, om);
+                if (cexp > 0.f)
+                    sum = (m > -INFINITY ? sum * fast_exp2((m - nm) * cexp) : 0.f) +
+                          (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
+                if (om > m || (om == m && oa < am)) am = oa;
+                m = nm;
+            }
+            if (lane == 0) { pm[par][warp] = m; ps[par][warp] = sum; pa[par][warp] = am; }
+            asm volatile("bar.sync 1, %0;" ::"r"(kVrWarps * 32) : "memory");
+            if (*reinterpret_cast<volatile int *>(&stop_s[par])) break;
+            if (warp == 0 && lane == 0) {
+                float M = pm[par][0];
+                int A = pa[par][0];
+                for (int x = 1; x < kVrWarps; ++x)
+                    if (pm[par][x] > M || (pm[par][x] == M && pa[par][x] < A)) { M = pm[par][x]; A = pa[par][x]; }
+                float S = 0.f;
+                if (cexp > 0.f)
+                    for (int x = 0; x < kVrWarps; ++x)
+                        if (pm[par][x] > -INFINITY) S += ps[par][x] * fast_exp2((pm[par][x] - M) * cexp);
+                const size_t o = (size_t)md.j * w.nChunks + md.c;
+                w.cm[o] = M;
+                w.cs[o] = S;
+                w.ca[o] = A;
+            }
         }
     }
 }
@@ -623,7 +698,7 @@ template <typename T>
 __global__ void __launch_bounds__(kRowThreads) residual_final(
     const T *__restrict__ Tlog, const T *__restrict__ L, const T *__restrict__ U,
     const T *__restrict__ Wt, const int32_t *__restrict__ x0, const int32_t *__restrict__ x,
-    const float *__restrict__ rowmax, const float *__restrict__ rowsum,
+    const float *__restrict__ H, const float *__restrict__ rowmax, const float *__restrict__ rowsum,
     const float *__restrict__ temp, const float *__restrict__ u_final, int G, int V, int r,
     VerifyWs w, int32_t *__restrict__ tokens_out) {
     extern __shared__ float res_smem[];
@@ -647,9 +722,17 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
     const float Tb = fmaxf(temp[b], 0.f), invT = 1.f / Tb;
     const float Md = rowmax[ro], Zd = rowsum[ro], Mt = w.res_mt[s], Zt = w.res_zt[s];
     const float u = u_final[b];
-    const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
-    const float uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
-    const float uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+    // The rejected position's A row in fp32: U[previous token] (Markov head)
+    // or the state that biased it (RNN head).
+    float uv0, uv1;
+    if (H != nullptr) {
+        uv0 = tid < r ? H[ro * r + tid] : 0.f;
+        uv1 = tid + nthr < r ? H[ro * r + tid + nthr] : 0.f;
+    } else {
+        const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
+        uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;
+        uv1 = tid + nthr < r ? ld_elem(U, (size_t)prev * r + tid + nthr) : 0.f;
+    }
     float loc = 0.f;
 #pragma unroll
     for (int q = 0; q < kResChunk; ++q) loc += cq[q];
@@ -736,10 +819,14 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int maxwork = a.B * (a.G + 1) * w.nChunks;
     if (a.dtype == DSPARK_BF16) {
-        // Enough resident warps to keep ~100 KB per SM of row data in flight.
-        const int grid = max(1, min((maxwork + 7) / 8, sms * 3));
-        verify_rows_warp<<<grid, kRowsWarpThreads, 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp,
-                                                            a.G, a.V, w);
+        const int grid = max(1, min(maxwork, sms));
+        const size_t smem = (size_t)kVrStages * kVrStageBytes + 2 * kVrStages * sizeof(uint64_t) +
+                            kVrStages * sizeof(VrMeta);
+        if ((e = cudaFuncSetAttribute(verify_rows_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        verify_rows_bulk<<<grid, kVrThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp, a.G,
+                                                         a.V, w, wait_budget(kVrWaitBudget));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         const int grid = max(1, min(maxwork, sms * 8));
@@ -752,7 +839,7 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.dtype == DSPARK_BF16) {
         ResidualTcArgs ra{a.Wt, static_cast<const __nv_bfloat16 *>(a.U), static_cast<const __nv_bfloat16 *>(a.L),
-                          static_cast<const __nv_bfloat16 *>(a.Tlog), a.x0, a.x, a.temp, a.rowmax, a.rowsum, w.res_mt,
+                          static_cast<const __nv_bfloat16 *>(a.Tlog), a.x0, a.x, a.H, a.temp, a.rowmax, a.rowsum, w.res_mt,
                           w.res_zt, w.res_b, w.res_k, &w.hdr->pad[1], a.B, a.G, a.V, a.r, w.nResTiles, w.rp, w.hdr};
         if ((e = launch_residual_tile_tc(ra, st)) != cudaSuccess) return e;
     } else {
@@ -770,7 +857,7 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
             return e;
     }
     fin<<<a.B, kRowThreads, smem, st>>>(Tl, static_cast<const T *>(a.L), static_cast<const T *>(a.U),
-                                       static_cast<const T *>(a.Wt), a.x0, a.x, a.rowmax, a.rowsum, a.temp,
+                                       static_cast<const T *>(a.Wt), a.x0, a.x, a.H, a.rowmax, a.rowsum, a.temp,
                                        a.u_final, a.G, a.V, a.r, w, a.tokens_out);
     return cudaGetLastError();
 }

@@ -10,7 +10,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import _lib
+from . import _lib, synth
 from .synth import RoundInputs
 
 
@@ -25,7 +25,9 @@ def _dev(arr: np.ndarray, dtype: str, device) -> torch.Tensor:
 
 class DeviceRound:
     def __init__(self, inp: RoundInputs, knots_n, knots_t, budget: int, mode: int, device="cuda",
-                 tau=None, pinned_host: bool = False):
+                 tau=None, pinned_host: bool = False, Arec=None):
+        """Arec: the RNN head's recurrent matrix [r, r] (fp32 values, sent in
+        the round's dtype); None drafts with the Markov head."""
         self.inp = inp
         self.B, self.G, self.V, self.r, self.d = inp.B, inp.G, inp.V, inp.r, inp.d
         self.dt = inp.dtype
@@ -38,6 +40,10 @@ class DeviceRound:
             "L": src("L", inp.L), "Tlog": src("Tlog", inp.Tlog), "U": src("U", inp.U), "Wt": Wt,
             "h": src("h", inp.h), "w": src("w", inp.w),
         }
+        if Arec is not None:
+            Ar = np.asarray(Arec, np.float32)
+            host["Arec"] = synth.bf16_bits(Ar) if self.dt == "bf16" else Ar
+        self.rnn = Arec is not None
         self.t = {k: _dev(v, self.dt, dev) for k, v in host.items()}
         small = {"x0": inp.x0.astype(np.int32), "temp": inp.temp.astype(np.float32),
                  "u_draft": inp.u_draft.astype(np.float32), "u_accept": inp.u_accept.astype(np.float32),
@@ -60,6 +66,8 @@ class DeviceRound:
             "acc": torch.zeros(B, **i32), "tokens": torch.zeros(B, G + 1, **i32), "nout": torch.zeros(B, **i32),
             "pt_x": torch.zeros(B, G, **f32),
         }
+        if self.rnn:
+            self.o["H"] = torch.zeros(B, G, self.r, **f32)
         dcode = _lib.DSPARK_BF16 if self.dt == "bf16" else _lib.DSPARK_F32
         need = max(_lib.dspark_draft_workspace_size(B, G, self.V, self.r, dcode),
                    _lib.dspark_schedule_workspace_size(B, G),
@@ -67,6 +75,7 @@ class DeviceRound:
         if need == 0:
             raise ValueError("round shape outside the library's limits")
         self.ws = torch.zeros((need + 255) // 256 * 256, dtype=torch.uint8, device=dev)
+        self._side = None
         self.host = None
         if pinned_host:
             self.host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in self.t.items()}
@@ -74,16 +83,54 @@ class DeviceRound:
                              for k, v in self.o.items() if k in ("tokens", "nout", "ell")}
 
     # -------------------------------------------------------------- running
-    def run(self, stream=None):
+    def run(self, stream=None, overlap_confidence: bool = True):
+        """Enqueue one round on `stream` (default: the current stream).  The
+        confidence stage does not depend on the drafted tokens, so by default
+        it runs on a side stream forked from `stream` at the start of the
+        round and joined before the scheduler (a fork and a join when the
+        round is captured in a graph)."""
         t, o = self.t, self.o
-        _lib.dspark_draft_markov(t["L"], t["U"], t["Wt"], t["x0"], t["temp"], t["u_draft"], self.ws,
-                                 o["x"], o["pd_x"], o["rowmax"], o["rowsum"], stream)
-        _lib.dspark_confidence(t["h"], t["w"], float(self.inp.bias), t["tau"], o["c"], o["S"], stream)
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+        conf = lambda st: _lib.dspark_confidence(t["h"], t["w"], float(self.inp.bias), t["tau"], o["c"], o["S"], st)
+        if overlap_confidence:
+            if self._side is None:
+                self._side = torch.cuda.Stream(device=self.device)
+                self._fork = torch.cuda.Event()
+                self._join = torch.cuda.Event()
+            self._fork.record(main)
+            self._side.wait_event(self._fork)
+            conf(self._side)
+            self._join.record(self._side)
+        self.draft(main)
+        if overlap_confidence:
+            main.wait_event(self._join)
+        else:
+            conf(main)
         _lib.dspark_schedule(o["S"], t["knots_n"], t["knots_t"], self.budget, self.mode, self.ws, o["ell"],
-                             o["n_adm"], o["theta"], o["order"], stream)
-        _lib.dspark_verify(t["Tlog"], t["L"], t["U"], t["Wt"], t["x0"], o["x"], o["pd_x"], o["rowmax"],
-                           o["rowsum"], t["temp"], t["u_accept"], t["u_final"], o["ell"], self.ws, o["acc"],
-                           o["tokens"], o["nout"], o["pt_x"], stream)
+                             o["n_adm"], o["theta"], o["order"], main)
+        self.verify(main)
+
+    def draft(self, stream=None):
+        """The drafting stage alone (Markov or RNN head)."""
+        t, o = self.t, self.o
+        if self.rnn:
+            _lib.dspark_draft_rnn(t["L"], t["U"], t["Arec"], t["Wt"], t["x0"], t["temp"], t["u_draft"], self.ws,
+                                  o["x"], o["pd_x"], o["rowmax"], o["rowsum"], o["H"], stream)
+        else:
+            _lib.dspark_draft_markov(t["L"], t["U"], t["Wt"], t["x0"], t["temp"], t["u_draft"], self.ws,
+                                     o["x"], o["pd_x"], o["rowmax"], o["rowsum"], stream)
+
+    def verify(self, stream=None):
+        """The verification stage alone, on the admitted lengths in o["ell"]."""
+        t, o = self.t, self.o
+        if self.rnn:
+            _lib.dspark_verify_rnn(t["Tlog"], t["L"], o["H"], t["Wt"], o["x"], o["pd_x"], o["rowmax"],
+                                   o["rowsum"], t["temp"], t["u_accept"], t["u_final"], o["ell"], self.ws,
+                                   o["acc"], o["tokens"], o["nout"], o["pt_x"], stream)
+        else:
+            _lib.dspark_verify(t["Tlog"], t["L"], t["U"], t["Wt"], t["x0"], o["x"], o["pd_x"], o["rowmax"],
+                               o["rowsum"], t["temp"], t["u_accept"], t["u_final"], o["ell"], self.ws, o["acc"],
+                               o["tokens"], o["nout"], o["pt_x"], stream)
 
     def upload(self, stream=None):
         """Copy every input from pinned host memory (end-to-end timing)."""

@@ -39,14 +39,16 @@ def _close(name, got, want, atol=ATOL):
                              f"gpu {got[tuple(i)]!r} oracle {want[tuple(i)]!r}")
 
 
-def check_draft(inp: synth.RoundInputs, idx, gx, gpd, grmax, grsum, rep: Report):
-    """Draft stage of requests idx against the oracle run on the same inputs."""
+def check_draft(inp: synth.RoundInputs, idx, gx, gpd, grmax, grsum, rep: Report, A=None):
+    """Draft stage of requests idx against the oracle run on the same inputs
+    (A: the RNN head's recurrent matrix, None for the Markov head)."""
     sub = synth.select_requests(inp, idx)
     gx, gpd, grmax, grsum = gx[idx], gpd[idx], grmax[idx], grsum[idx]
     B, G = gx.shape
     force = np.full((B, G), -1, np.int32)
     for _ in range(G + 1):
-        o = oracle.draft(sub.L, sub.U, sub.W, sub.x0, sub.temp, sub.u_draft.astype(np.float64), force_x=force)
+        o = oracle.draft(sub.L, sub.U, sub.W, sub.x0, sub.temp, sub.u_draft.astype(np.float64), force_x=force,
+                         A=A)
         mism = (o.x != gx) & (force < 0)
         if not mism.any():
             break
@@ -87,7 +89,12 @@ def check_schedule(gS, gell, gnadm, gtheta, gorder, knots_n, knots_t, budget, mo
             assert abs(alt.theta - o.theta) <= 1e-12 * abs(o.theta), (
                 f"admitted count gpu {gnadm} oracle {o.n_adm}: Theta {alt.theta!r} vs best {o.theta!r}")
         else:
-            assert o.margin_theta < TIE, f"admitted count gpu {gnadm} oracle {o.n_adm} (margin {o.margin_theta:.3g})"
+            # The count differs only if the comparison at the earlier of the
+            # two stop points is a near-tie (the oracle's stop, or the
+            # comparison where the GPU stopped and the oracle admitted).
+            k = min(int(gnadm), int(o.n_adm))
+            mk = o.margins[k] if k < len(o.margins) else np.inf
+            assert mk < TIE, f"admitted count gpu {gnadm} oracle {o.n_adm} (margin at {k}: {mk:.3g})"
         rep.near_ties["schedule"] += 1
         o = oracle.schedule(gS.astype(np.float64), knots_n, knots_t, budget, mode, force_n=int(gnadm))
     assert np.array_equal(o.ell, gell), "admitted prefix lengths differ"
@@ -106,9 +113,9 @@ def check_schedule(gS, gell, gnadm, gtheta, gorder, knots_n, knots_t, budget, mo
     return o
 
 
-def check_verify(inp: synth.RoundInputs, idx, gx, gell, gacc, gtok, gnout, gptx, rep: Report):
+def check_verify(inp: synth.RoundInputs, idx, gx, gell, gacc, gtok, gnout, gptx, rep: Report, A=None):
     """Verification of requests idx with the GPU's draft tokens and admitted
-    lengths; the oracle rebuilds p_d itself in fp64."""
+    lengths; the oracle rebuilds p_d itself in fp64 (A as for check_draft)."""
     sub = synth.select_requests(inp, idx)
     x, ell = gx[idx], gell[idx]
     gacc, gtok, gnout, gptx = gacc[idx], gtok[idx], gnout[idx], gptx[idx]
@@ -117,7 +124,7 @@ def check_verify(inp: synth.RoundInputs, idx, gx, gell, gacc, gtok, gnout, gptx,
     for _ in range(G + 1):
         o = oracle.verify(sub.Tlog, sub.L, sub.U, sub.W, sub.x0, x, sub.temp,
                           sub.u_accept.astype(np.float64), sub.u_final.astype(np.float64), ell,
-                          force_accept=force)
+                          force_accept=force, A=A)
         mism = o.acc != gacc
         if not mism.any():
             break

@@ -191,3 +191,61 @@ def test_injected_failure_on_variant_entries(lib, monkeypatch):
     assert lib.dspark_survival_auc(FAKE, FAKE, 64, 5, FAKE, FAKE, None) == 5
     monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_schedule_topk=4")
     assert lib.dspark_schedule_topk(FAKE, 8, 5, FAKE, -1, FAKE_WS, 1 << 20, FAKE, FAKE, None, None) == 4
+
+
+def test_injected_failure_on_verify_and_noalloc(lib, monkeypatch):
+    """Verification, allocation-free drafting and its status getter honour
+    host-side injection too (they fail before touching any pointer)."""
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_verify=4")
+    assert lib.dspark_verify(*([FAKE] * 13), 4, 5, 1024, 16, 0, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None,
+                             None) == 4
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_draft_markov_noalloc=5")
+    assert lib.dspark_draft_markov_noalloc(*([FAKE] * 6), 4, 5, 1024, 16, 0, FAKE, FAKE, FAKE, FAKE, None) == 5
+    # An injection names one entry point only.
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_draft_markov=5")
+    assert lib.dspark_draft_markov_noalloc(*([FAKE] * 6), 0, 5, 1024, 16, 0, FAKE, FAKE, FAKE, FAKE, None) == 1
+
+
+def test_noalloc_argument_checks(lib):
+    """The allocation-free entry point applies the same host checks as the
+    workspace one."""
+    f = lib.dspark_draft_markov_noalloc
+    assert f(*([FAKE] * 6), 0, 5, 1024, 16, 0, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(*([FAKE] * 6), 4, 17, 1024, 16, 0, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(*([FAKE] * 6), 4, 5, 1024, 24, 1, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert f(*([FAKE] * 6), 4, 5, 1024, 16, 7, FAKE, FAKE, FAKE, FAKE, None) == 2
+    for k in range(6):
+        args = [FAKE] * 6
+        args[k] = None
+        assert f(*args, 4, 5, 1024, 16, 0, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert lib.dspark_draft_noalloc_device_status(None, None) == 1
+
+
+def test_rnn_entry_point_checks(lib, monkeypatch):
+    """The RNN head's entry points: bf16 only, r <= 256, every pointer
+    present, 16-byte aligned bf16 arrays and states, a large enough
+    workspace; host-side injection."""
+    d = lib.dspark_draft_rnn
+    v = lib.dspark_verify_rnn
+    ok7 = [FAKE] * 7
+    assert d(*ok7, 4, 5, 1024, 16, 0, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2   # fp32
+    assert d(*ok7, 4, 5, 1024, 272, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1  # r > 256
+    assert d(*ok7, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, None, None) == 1   # no H_out
+    assert d(*ok7, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, ctypes.c_void_p(0x200008),
+             None) == 1                                                                            # misaligned H
+    assert d(*ok7, 4, 5, 1024, 16, 1, FAKE_WS, 16, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 3        # workspace
+    for k in range(7):
+        args = list(ok7)
+        args[k] = None
+        assert d(*args, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 1
+    ok12 = [FAKE] * 12
+    assert v(*ok12, 4, 5, 1024, 16, 0, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 2
+    assert v(*ok12, 4, 5, 1024, 272, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 1
+    bad = list(ok12)
+    bad[2] = None   # the states
+    assert v(*bad, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 1
+    assert v(*ok12, 4, 5, 1024, 16, 1, None, 1 << 30, FAKE, FAKE, FAKE, None, None) == 3
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_draft_rnn=4")
+    assert d(*ok7, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 4
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_verify_rnn=5")
+    assert v(*ok12, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 5

@@ -50,7 +50,9 @@ def test_round_parity_small(dtype, B, G, V, r, d):
     temps = np.tile(np.float32([1.0, 0.0, 0.6, 1.2]), B)[:B]
     inp, dr = _round(B, G, V, r, d, dtype, seed=B + V, knots_n=PROFILE[0], knots_t=PROFILE[1], temps=temps)
     out, rep = _check_round(inp, dr, *PROFILE, -1, 1)
-    assert rep.total_ties() <= max(2, B // 10)
+    # At a 1e-5 margin a counted near-tie is a rare event (about 2e-5 per
+    # decision, and a disagreement needs a far smaller margin still).
+    assert rep.total_ties() <= 1, rep.near_ties
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

@@ -50,4 +50,4 @@ def test_workload_parity(name, make, nsample):
         assert 0 <= out["tokens"][b, A] < w.V and np.all(out["tokens"][b, A + 1:] == -1)
     if w.mode == wl.MODE_ALL:
         assert np.all(out["ell"] == w.G)
-    assert rep.total_ties() <= max(2, len(idx) // 4)
+    assert rep.total_ties() <= 1, rep.near_ties

@@ -135,3 +135,49 @@ def test_rnn_mutant_is_caught(tmp_path, name, old, new):
     finally:
         oracle.use_library(oracle.build())
     assert caught, f"no RNN pin catches {name}"
+
+
+# Planted mistakes in the decision margins, caught by the margin pins.
+MARGIN_MUTANTS = [
+    ("draft_margin_unnormalised", "double m0 = u - prev, m1 = c - u;",
+     "double m0 = (u - prev) * tot, m1 = (c - u) * tot;"),
+    ("draft_margin_without_lower_edge", "*margin = m0 < m1 ? m0 : m1;", "*margin = m1;"),
+    ("draft_margin_constant", "*margin = m0 < m1 ? m0 : m1;", "*margin = 1.0;"),
+    ("greedy_margin_not_a_gap", "*gap = (V > 1) ? z[best] - second : INFINITY;",
+     "*gap = (V > 1) ? z[best] : INFINITY;"),
+    ("accept_margin_against_p_t", "margin_acc_out[o] = fabs(u_accept[o] - ratio);",
+     "margin_acc_out[o] = fabs(u_accept[o] - pt);"),
+    ("greedy_accept_margin_against_argmax", "margin_acc_out[o] = fabs(yt[xk] - best_other);",
+     "margin_acc_out[o] = gap;"),
+    ("admission_margin_absolute", "double rel = fabs(th1 - theta) / theta;", "double rel = fabs(th1 - theta);"),
+    ("admission_margin_smallest_seen",
+     "            if (margins_out) margins_out[n] = rel;\n"
+     "            if (Vn1 * t0 < Vn * t1) { /* Theta_{n+1} < Theta_n: stop */\n"
+     "                mtheta = rel;\n",
+     "            if (margins_out) margins_out[n] = rel;\n"
+     "            if (rel < mtheta) mtheta = rel;\n"
+     "            if (Vn1 * t0 < Vn * t1) { /* Theta_{n+1} < Theta_n: stop */\n"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MARGIN_MUTANTS, ids=[m[0] for m in MARGIN_MUTANTS])
+def test_margin_mutant_is_caught(tmp_path, name, old, new):
+    import test_oracle_margins as pins
+    so = _build_mutant(tmp_path, name, old, new)
+    caught = []
+    try:
+        oracle.use_library(so)
+        for pin, args in ((pins.test_draft_margin_is_the_distance_to_the_nearer_cdf_edge, (1.0,)),
+                          (pins.test_draft_margin_near_each_edge, ()),
+                          (pins.test_greedy_draft_margin_is_the_top_two_gap, ()),
+                          (pins.test_accept_and_final_margins_follow_their_definitions, ()),
+                          (pins.test_greedy_accept_margin_is_the_gap_to_the_best_other_logit, ()),
+                          (pins.test_admission_margin_is_taken_at_the_stop_point, ()),
+                          (pins.test_admission_margins_match_brute_force, (0,))):
+            try:
+                pin(*args)
+            except AssertionError:
+                caught.append(pin.__name__)
+    finally:
+        oracle.use_library(oracle.build())
+    assert caught, f"no margin pin catches {name}"

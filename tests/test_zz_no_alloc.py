@@ -38,7 +38,7 @@ def _outputs(B, G):
 
 
 @pytest.mark.parametrize("dtype,B,G,V,r", [("bf16", 256, 5, 12000, 256), ("bf16", 37, 3, 5008, 80),
-                                           ("f32", 9, 4, 3001, 16)])
+                                           ("f32", 9, 4, 3001, 16), ("bf16", 256, 5, 129280, 256)])
 def test_noalloc_matches_workspace_entry_point(dtype, B, G, V, r):
     temps = np.tile(np.float32([1.0, 0.0, 0.7, 1.3]), B)[:B]
     inp = synth.generate(B, G, V, r, 8, dtype, seed=B + V, hot=8, temps=temps)
@@ -56,6 +56,7 @@ def test_noalloc_matches_workspace_entry_point(dtype, B, G, V, r):
         for name, g, w in zip(("p_d(x)", "row max", "Z"), got[1:], ref[1:]):
             assert torch.allclose(g, w, atol=ATOL, rtol=0), f"call {call}: {name} differs"
     assert _lib.dspark_get_device_status(ws) == 0
+    assert _lib.dspark_draft_noalloc_device_status() == 0
 
 
 def test_noalloc_rejects_rounds_beyond_its_scratch():
@@ -69,3 +70,24 @@ def test_noalloc_rejects_rounds_beyond_its_scratch():
         _lib._ptr(dummy), _lib._ptr(dummy), _lib._ptr(dummy), _lib._ptr(idx), _lib._ptr(f), _lib._ptr(f), B, G, V,
         r, _lib.DSPARK_BF16, _lib._ptr(idx), _lib._ptr(f), _lib._ptr(f), _lib._ptr(f), None)
     assert st == 3  # DSPARK_ERR_WORKSPACE, before any work is enqueued
+
+
+def test_noalloc_reports_a_wait_that_ran_out(monkeypatch):
+    """A bounded wait that runs out inside the allocation-free call is
+    reported through its status getter, and the next call (which clears the
+    word) succeeds with the normal budget."""
+    B, G, V, r = 130, 3, 4104, 64
+    inp = synth.generate(B, G, V, r, 8, "bf16", seed=3, hot=8)
+    L, U, Wt, x0, temp, ud = _device_inputs(inp)
+    ws = torch.zeros(_lib.dspark_draft_workspace_size(B, G, V, r, _lib.DSPARK_BF16), dtype=torch.uint8,
+                     device="cuda")
+    ref = _outputs(B, G)
+    _lib.dspark_draft_markov(L, U, Wt, x0, temp, ud, ws, *ref)
+    monkeypatch.setenv("DSPARK_WAIT_BUDGET_CYCLES", "200")
+    got = _outputs(B, G)
+    _lib.dspark_draft_markov_noalloc(L, U, Wt, x0, temp, ud, *got)
+    assert _lib.dspark_draft_noalloc_device_status() & _lib.DEV_TIMEOUT
+    monkeypatch.delenv("DSPARK_WAIT_BUDGET_CYCLES")
+    _lib.dspark_draft_markov_noalloc(L, U, Wt, x0, temp, ud, *got)
+    assert _lib.dspark_draft_noalloc_device_status() == 0
+    assert torch.equal(got[0], ref[0])

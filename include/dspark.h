@@ -345,9 +345,22 @@ dspark_status dspark_survival_auc(const float *S, const int32_t *acc, int N, int
 
 /* Device status word of a workspace: dspark_get_device_status synchronises
  * `stream`, then copies the word to *status_out (0 = no data error since the
- * last clear).  dspark_clear_device_status enqueues a reset of the word. */
+ * last clear).  dspark_clear_device_status enqueues a reset of the word and
+ * of the near-tie counts below. */
 dspark_status dspark_get_device_status(const void *ws, void *stream, uint32_t *status_out);
 dspark_status dspark_clear_device_status(void *ws, void *stream);
+
+/* Near-tie counts of a workspace since its last clear: the sampled decisions
+ * whose uniform fell within 1e-5 of the threshold that would flip them, as
+ * the kernels evaluate them in fp32 -- a draw's uniform within 1e-5 (CDF
+ * units) of an edge of the chosen token's interval, or one that rounding left
+ * past the row's mass (drafting: *draft_out; the bonus, fresh and residual
+ * draws of verification: *verify_out), and an accept test with
+ * |u - p_t(x)/p_d(x)| < 1e-5 among the tests that decided the accepted count
+ * (*verify_out).  Such a decision can differ from an exact computation of
+ * the same round; argmax decisions (temperature 0) are not counted.
+ * Synchronises `stream`. */
+dspark_status dspark_get_near_ties(const void *ws, void *stream, uint32_t *draft_out, uint32_t *verify_out);
 
 #ifdef __cplusplus
 }

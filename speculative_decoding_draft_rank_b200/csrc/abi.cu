@@ -198,7 +198,23 @@ dspark_status dspark_get_device_status(const void *ws, void *stream, uint32_t *s
 
 dspark_status dspark_clear_device_status(void *ws, void *stream) {
     if (!ws) return DSPARK_ERR_INVALID_ARG;
-    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream)));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    WsHeader *h = static_cast<WsHeader *>(ws);
+    if (cudaMemsetAsync(&h->status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSPARK_ERR_CUDA;
+    return cuda_status(cudaMemsetAsync(&h->pad[kPadDraftTies], 0, 2 * sizeof(uint32_t), st));
+}
+
+dspark_status dspark_get_near_ties(const void *ws, void *stream, uint32_t *draft_out, uint32_t *verify_out) {
+    if (!ws || !draft_out || !verify_out) return DSPARK_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSPARK_ERR_CUDA;
+    uint32_t v[2] = {0, 0};
+    const WsHeader *h = static_cast<const WsHeader *>(ws);
+    if (cudaMemcpy(v, &h->pad[kPadDraftTies], sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return DSPARK_ERR_CUDA;
+    *draft_out = v[0];
+    *verify_out = v[1];
+    return DSPARK_OK;
 }
 
 }  // extern "C"

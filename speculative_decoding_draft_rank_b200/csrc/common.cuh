@@ -24,6 +24,15 @@ __device__ __forceinline__ void flag_status(WsHeader *h, uint32_t bit) {
     atomicOr(&h->status, bit);
 }
 
+// Near-tie counters in the workspace header: sampled decisions whose uniform
+// fell within kNearTie (CDF units) of an edge of the chosen interval, or of
+// the accept threshold p_t / p_d.  Drafting counts into pad[8], verification
+// into pad[9]; dspark_clear_device_status zeroes both.
+constexpr int kPadDraftTies = 8;
+constexpr int kPadVerifyTies = 9;
+constexpr float kNearTie = 1e-5f;
+__device__ __forceinline__ void count_near_tie(WsHeader *h, int slot) { atomicAdd(&h->pad[slot], 1u); }
+
 // Element loads: fp32 or bf16 widened exactly to fp32.
 __device__ __forceinline__ float ld_elem(const float *p, size_t i) { return __ldg(p + i); }
 __device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) {

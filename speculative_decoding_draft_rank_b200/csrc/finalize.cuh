@@ -209,7 +209,8 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     // The first thread whose inclusive prefix passes u Z owns the crossing
     // (the last thread with mass if rounding left u Z at the top).
     int owner = grp_min1(g, (incl > target && loc > 0.f) ? tid : 0x7fffffff, sc->s_own);
-    if (owner == 0x7fffffff) owner = max(0, grp_max1_i(g, loc > 0.f ? tid : -1, sc->s_own2));
+    const bool past_mass = owner == 0x7fffffff;   // rounding left u Z at the top: a tie by definition
+    if (past_mass) owner = max(0, grp_max1_i(g, loc > 0.f ? tid : -1, sc->s_own2));
     if (tid == owner) {
         float run = incl - loc, run_last = run;
         int ts = -1, last = t1 - 1;
@@ -264,7 +265,8 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     float ttot;
     const float inc = grp_scan1(g, e, sc->s_col, &ttot);
     int xs = grp_min1(g, (mine && inc > rem) ? col : 0x7fffffff, sc->s_x);
-    if (xs == 0x7fffffff) {  // the recomputed mass fell short: last positive column
+    const bool fell_short = xs == 0x7fffffff;
+    if (fell_short) {  // the recomputed mass fell short: last positive column
         xs = grp_max1_i(g, (mine && e > 0.f) ? col : -1, sc->s_x2);
         if (xs < 0) xs = min(c0 + TN, V) - 1;
     }
@@ -273,6 +275,10 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
         a.pd_out[ro] = e / Z;
         a.rowmax_out[ro] = M;
         a.rowsum_out[ro] = Z;
+        // The draw's margin: u Z to the nearer edge of the token's interval
+        // [inc - e, inc) (mass units, relative to the crossing slice), over Z.
+        const float margin = (past_mass || fell_short) ? 0.f : fminf(rem - (inc - e), inc - rem) / Z;
+        if (margin < kNearTie) count_near_tie(a.hdr, kPadDraftTies);
     }
     stage_next(xs);
     g.sync();

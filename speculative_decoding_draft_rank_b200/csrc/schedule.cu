@@ -79,8 +79,10 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 {
     extern __shared__ __align__(16) unsigned char sched_smem[];
     const int N = B * G;
+    int n2 = 64;
+    while (n2 < N) n2 <<= 1;
     unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [n2]
-    int *ell_s = reinterpret_cast<int *>(keys + kSchedMaxN);                          // [B]
+    int *ell_s = reinterpret_cast<int *>(keys + n2);                                  // [B]
     __shared__ int kn_s[kSchedMaxP];
     __shared__ double kt_s[kSchedMaxP];
     __shared__ int red_i[33];
@@ -110,8 +112,6 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     // Unique 64-bit keys: ~bits(S) (ascending = S descending, valid for
     // S >= 0) above the position-major id, so an ascending sort is the stable
     // sort by S descending.  Padding keys sort last.
-    int n2 = 64;
-    while (n2 < N) n2 <<= 1;
     for (int id = tid; id < n2; id += blockDim.x) {
         unsigned long long k = ~0ull;
         if (id < N) {
@@ -255,13 +255,20 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
 
 size_t schedule_ws_bytes(int, int) { return sizeof(WsHeader); }
 
+// Dynamic shared memory of one call: the padded keys and the per-request counts.
+static size_t sched_smem_bytes(int B, int G) {
+    int n2 = 64;
+    while (n2 < B * G) n2 <<= 1;
+    return sizeof(unsigned long long) * (size_t)n2 + sizeof(int) * (size_t)B;
+}
+
 cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
                             const double *knots_t, int P, int budget, int mode, float threshold, void *,
                             int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
                             int32_t *order_out, cudaStream_t st) {
-    const size_t smem = sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096;
+    const size_t smem = sched_smem_bytes(B, G);
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+                                         (int)(sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096));
     if (e != cudaSuccess) return e;
     schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, threshold,
                                                     nullptr, nullptr, ell_out, n_adm_out, theta_out, order_out);
@@ -270,9 +277,9 @@ cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n
 
 cudaError_t launch_schedule_topk(const float *S, int B, int G, const int32_t *capacity, int budget, void *ws,
                                  int32_t *ell_out, int32_t *n_adm_out, int32_t *order_out, cudaStream_t st) {
-    const size_t smem = sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096;
+    const size_t smem = sched_smem_bytes(B, G);
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+                                         (int)(sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096));
     if (e != cudaSuccess) return e;
     schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_TOPK, 0.f,
                                                     capacity, static_cast<WsHeader *>(ws), ell_out, n_adm_out,

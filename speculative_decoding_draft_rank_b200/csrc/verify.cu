@@ -482,7 +482,8 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
     float tot;
     const float inc = block_scan1(wc, s_c, &tot);
     int ch = block_min1((tid < w.nChunks && inc > target) ? tid : 0x7fffffff, s_i0);
-    if (ch == 0x7fffffff) {
+    const bool past_mass = ch == 0x7fffffff;   // rounding left u Z at the top: a tie by definition
+    if (past_mass) {
         ch = block_max1_i((tid < w.nChunks && wc > 0.f) ? tid : -1, s_i1);
         if (ch < 0) ch = w.nChunks - 1;
     }
@@ -508,19 +509,25 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
     float rt;
     const float incl = block_scan1(run, s_e, &rt);
     int owner = block_min1((incl > rem && run > 0.f) ? tid : 0x7fffffff, s_i2);
-    if (owner == 0x7fffffff) owner = max(0, block_max1_i(run > 0.f ? tid : -1, s_i3));
+    const bool short_slice = owner == 0x7fffffff;
+    if (short_slice) owner = max(0, block_max1_i(run > 0.f ? tid : -1, s_i3));
     if (tid == owner) {
         float p = incl - run;
         int f = -1, lastpos = -1;
+        float margin = 0.f;
 #pragma unroll
         for (int t = 0; t < 32; ++t) {
             if (f < 0 && e[t] > 0.f) {
                 lastpos = i0 + t;
                 p += e[t];
-                if (p > rem) f = i0 + t;
+                if (p > rem) {
+                    f = i0 + t;
+                    margin = fminf(rem - (p - e[t]), p - rem) / Z;   // u Z to the nearer edge, over Z
+                }
             }
         }
         if (f < 0) f = lastpos >= 0 ? lastpos : c1 - 1;
+        if (past_mass || short_slice || !(margin >= kNearTie)) count_near_tie(w.hdr, kPadVerifyTies);
         col_s = f;
     }
     __syncthreads();
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     int32_t *__restrict__ nout_out, float *__restrict__ pt_x_out) {
     __shared__ float rM[17], rZ[17];
     __shared__ int rA[17];
-    __shared__ int acc_s[16];
+    __shared__ int acc_s[16], tie_s[16];
     __shared__ int A_s;
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const float Tb = sane_temp(temp[b], w.hdr);
@@ -568,23 +575,29 @@ __global__ void __launch_bounds__(kRowThreads) verify_decide(
     __syncthreads();
     if (tid < G) {
         float pt = -1.f;
-        int acc = 0;
+        int acc = 0, tie = 0;
         if (tid < lb) {
             if (Tb == 0.f) {
                 acc = rA[tid] == xk;
                 pt = acc ? 1.f : 0.f;
             } else {
                 pt = exp_e((tk - rM[tid]) * invT) / rZ[tid];
-                acc = uk < pt / pdk;
+                const float ratio = pt / pdk;
+                acc = uk < ratio;
+                tie = !(fabsf(uk - ratio) >= kNearTie);
             }
         }
         acc_s[tid] = acc;
+        tie_s[tid] = tie;
         if (pt_x_out != nullptr) pt_x_out[o] = pt;
     }
     __syncthreads();
     if (tid == 0) {
         int A = 0;
         while (A < lb && acc_s[A]) ++A;   // the first rejection discards the rest
+        // Near-ties among the tests that decided A (later ones are discarded).
+        for (int k = 0; k < lb && k <= A; ++k)
+            if (tie_s[k]) count_near_tie(w.hdr, kPadVerifyTies);
         A_s = A;
         acc_out[b] = A;
         nout_out[b] = A + 1;
@@ -747,7 +760,8 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
     } else {
         const float target = u * Q;
         int owner = block_min1((incl > target && loc > 0.f) ? tid : 0x7fffffff, s_own);
-        if (owner == 0x7fffffff) owner = max(0, block_max1_i(loc > 0.f ? tid : -1, s_own2));
+        const bool past_mass = owner == 0x7fffffff;   // rounding left u Q at the top: a tie by definition
+        if (past_mass) owner = max(0, block_max1_i(loc > 0.f ? tid : -1, s_own2));
         if (tid == owner) {
             float run = incl - loc, run_last = run;
             int ts = -1, last = t1 - 1;
@@ -798,9 +812,15 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
         float tot;
         const float inc = block_scan1(qv, s_col, &tot);
         int ys = block_min1((mine && qv > 0.f && inc > rem) ? col : 0x7fffffff, s_y);
-        if (ys == 0x7fffffff) {
+        const bool fell_short = ys == 0x7fffffff;
+        if (fell_short) {
             ys = block_max1_i((mine && qv > 0.f) ? col : -1, s_y2);
             if (ys < 0) ys = min(c0 + TN, V) - 1;
+        }
+        if (mine && col == ys) {
+            // The residual draw's margin: u Q to the nearer edge of the token's interval, over Q.
+            const float margin = (past_mass || fell_short) ? 0.f : fminf(rem - (inc - qv), inc - rem) / Q;
+            if (margin < kNearTie) count_near_tie(w.hdr, kPadVerifyTies);
         }
         y = ys;
     }

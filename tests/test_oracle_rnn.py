@@ -128,3 +128,22 @@ def test_states_match_the_drafting_bias():
     h = oracle.rnn_states(U, A, x0, d.x)
     np.testing.assert_allclose(d.rowmax, h.max(axis=2), rtol=0, atol=1e-15)
     assert np.array_equal(d.x, h.argmax(axis=2))
+
+
+def test_rnn_states_refuse_tokens_outside_the_vocabulary():
+    """The states entry indexes U by token: a token outside [0, V) (either
+    the committed one or a drafted one) or an empty batch is an argument
+    error, not an out-of-bounds read."""
+    rng = np.random.default_rng(3)
+    V, r, G = 6, 4, 3
+    U = rng.normal(0, 1, (V, r)).astype(np.float32)
+    A = np.zeros((r, r), np.float32)
+    ok_x0, ok_x = np.array([1, 2], np.int32), np.array([[0, 5, 3], [1, 1, 1]], np.int32)
+    oracle.rnn_states(U, A, ok_x0, ok_x)
+    for x0, x in ((np.array([6, 2], np.int32), ok_x), (np.array([-1, 2], np.int32), ok_x),
+                  (ok_x0, np.array([[0, 6, 3], [1, 1, 1]], np.int32)),
+                  (ok_x0, np.array([[0, 1, 3], [-2, 1, 1]], np.int32))):
+        with pytest.raises(ValueError):
+            oracle.rnn_states(U, A, x0, x)
+    with pytest.raises(ValueError):
+        oracle.rnn_states(U, A, np.zeros(0, np.int32), np.zeros((0, G), np.int32))

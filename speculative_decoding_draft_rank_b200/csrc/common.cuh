@@ -59,6 +59,14 @@ __device__ __forceinline__ uint4 ld_nc16(const void *p) {
     return r;
 }
 
+// v rounded to bf16, plus the remainder rounded to bf16: the value a product
+// of the two bf16 parts of v (a high and a low part) multiplies by.
+__device__ __forceinline__ float split_bf16_sum(float v) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float h = __bfloat162float(hi);
+    return h + __bfloat162float(__float2bfloat16_rn(v - h));
+}
+
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
@@ -88,6 +96,31 @@ __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
     return r;
 }
+// 2^x for two arguments x <= 0 on the FMA pipe, to share the exponential work
+// of a softmax with the MUFU unit: x = n + f with n = rint(x) (by the 1.5 * 2^23
+// rounding constant, no conversion instruction) and f in [-1/2, 1/2]; 2^f from
+// the degree-5 polynomial interpolating it at the six Chebyshev nodes of
+// [-1/2, 1/2] (coefficients computed offline; max relative error 2.4e-7 in
+// fp32 Horner form, about that of ex2.approx); 2^n added to the exponent
+// bits.  Arguments below -125 are raised to -125 (a value of ~1e-38 in place
+// of a smaller one).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    const float2 lo = make_float2(-125.f, -125.f);
+    x = make_float2(fmaxf(x.x, lo.x), fmaxf(x.y, lo.y));
+    const float2 big = make_float2(12582912.f, 12582912.f);
+    const float2 t = add2(x, big);                       // n in the low mantissa bits
+    const float2 f = add2(x, add2(big, make_float2(-t.x, -t.y)));   // x - n
+    float2 p = make_float2(0.0013390863314270973f, 0.0013390863314270973f);
+    p = fma2(p, f, make_float2(0.009676031768321991f, 0.009676031768321991f));
+    p = fma2(p, f, make_float2(0.055503569543361664f, 0.055503569543361664f));
+    p = fma2(p, f, make_float2(0.2402210682630539f, 0.2402210682630539f));
+    p = fma2(p, f, make_float2(0.6931471824645996f, 0.6931471824645996f));
+    p = fma2(p, f, make_float2(1.0000001192092896f, 1.0000001192092896f));
+    const int nx = __float_as_int(t.x) - 0x4B400000, ny = __float_as_int(t.y) - 0x4B400000;
+    return make_float2(__int_as_float(__float_as_int(p.x) + (nx << 23)),
+                       __int_as_float(__float_as_int(p.y) + (ny << 23)));
+}
+
 // max(a, b, c) in one instruction.
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;

@@ -157,9 +157,11 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     // published to urow by the first group barrier below.
     float uv0, uv1;
     if (a.H != nullptr) {
+        // The state as the tensor-core product saw it: its high and low bf16
+        // parts summed, so the recomputed slice agrees with the tile partials.
         const float *hrow = a.H + ro * r;
-        uv0 = tid < r ? hrow[tid] : 0.f;
-        uv1 = tid + nthr < r ? hrow[tid + nthr] : 0.f;
+        uv0 = tid < r ? split_bf16_sum(hrow[tid]) : 0.f;
+        uv1 = tid + nthr < r ? split_bf16_sum(hrow[tid + nthr]) : 0.f;
     } else {
         const int prev = (pos == 0) ? clamp_token(a.x0[b], V, a.hdr) : a.x_out[(size_t)b * G + pos - 1];
         uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;

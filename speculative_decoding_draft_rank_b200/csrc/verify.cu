@@ -738,9 +738,9 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
     // The rejected position's A row in fp32: U[previous token] (Markov head)
     // or the state that biased it (RNN head).
     float uv0, uv1;
-    if (H != nullptr) {
-        uv0 = tid < r ? H[ro * r + tid] : 0.f;
-        uv1 = tid + nthr < r ? H[ro * r + tid + nthr] : 0.f;
+    if (H != nullptr) {   // as the residual tile pass's split product saw it
+        uv0 = tid < r ? split_bf16_sum(H[ro * r + tid]) : 0.f;
+        uv1 = tid + nthr < r ? split_bf16_sum(H[ro * r + tid + nthr]) : 0.f;
     } else {
         const int prev = min(max((k == 0) ? x0[b] : x[ro - 1], 0), V - 1);
         uv0 = tid < r ? ld_elem(U, (size_t)prev * r + tid) : 0.f;

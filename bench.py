@@ -695,6 +695,7 @@ def main():
     nout_sum = int(dr.o["nout"].sum().item())
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    _lib.dspark_clear_device_status(dr.ws, stream)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
         barrier()
@@ -708,6 +709,9 @@ def main():
                 step_ms.append(e0.elapsed_time(e1))
         torch.cuda.synchronize()
         barrier()
+    # Decisions within 1e-5 of their threshold, as the kernels counted them
+    # over the timed rounds (the same inputs every round).
+    ties_d, ties_v = _lib.dspark_get_near_ties(dr.ws, stream)
     # Stage breakdown (not the headline): each stage's graph between events.
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     with torch.cuda.stream(stream):
@@ -794,7 +798,9 @@ def main():
                   "rounds_per_s": world * 1e3 / ms, "emitted_tokens_per_s": nout_tot / (ms * 1e-3),
                   "algorithmic_bytes": round_bytes,
                   "hbm_roofline_frac": (round_bytes / (ms * 1e-3) / 1e9) / hbm_gbs,
-                  "stage_ms": dict(zip(stage_names, stage_means))},
+                  "stage_ms": dict(zip(stage_names, stage_means)),
+                  "near_ties_per_round": {"draft": ties_d / max(1, args.steps),
+                                          "verify": ties_v / max(1, args.steps)}},
         "roofline": {"kernel": stage_kernels[dom], "bound": "hbm", "achieved": ach,
                      "peak": hbm_gbs, "unit": "GB/s", "frac": ach / hbm_gbs,
                      "traffic": profiled_traffic(w.name) if dom == 0 else None,

@@ -6,11 +6,12 @@
 // calibrated left to right by sequential temperature scaling):
 //   c[b,i] = sigmoid((w . h[b,i,:] + bias) / tau[i]),  S[b,i] = prod_{j<=i} c[b,j].
 //
-// One CTA per request; each position's row is split over P = 32 / G warps
-// (at most 8) so that every 16-byte load of the batch is in flight at once
-// (the stage is latency-bound otherwise: a few KB per row).  The warps'
-// partial dot products are folded in a fixed order, then the first thread
-// forms the running product.  HBM-bound: B*G*d*esize bytes.
+// One CTA per request, one warp per position (G warps, at most 40 registers
+// a thread): small enough to share an SM with the drafting kernel, which it
+// runs beside on a side stream of the round (it does not depend on the
+// drafted tokens).  Each lane keeps four 16-byte loads of h in flight; the
+// warp's partial dot products are folded in a fixed order, then the first
+// thread forms the running product.  HBM-bound: B*G*d*esize bytes.
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -77,7 +78,7 @@ __device__ __forceinline__ float dot_part8(const float *__restrict__ h, const fl
 }
 
 template <typename T>
-__global__ void __launch_bounds__(1024) confidence_kernel(const T *__restrict__ h, const T *__restrict__ w,
+__global__ void __launch_bounds__(512, 3) confidence_kernel(const T *__restrict__ h, const T *__restrict__ w,
                                                           float bias, const float *__restrict__ tau, int B, int G,
                                                           int d, int P, float *__restrict__ c_out,
                                                           float *__restrict__ S_out) {
@@ -114,8 +115,7 @@ __global__ void __launch_bounds__(1024) confidence_kernel(const T *__restrict__ 
 
 cudaError_t launch_confidence(const void *h, const void *w, float bias, const float *tau, int B,
                               int G, int d, int dtype, float *c_out, float *S_out, cudaStream_t st) {
-    int P = 32 / G;                      // warps per position (G <= 16)
-    P = P > 8 ? 8 : P;
+    const int P = 1;                     // one warp per position
     const int threads = 32 * G * P;
     if (dtype == DSPARK_BF16)
         confidence_kernel<__nv_bfloat16><<<B, threads, 0, st>>>(

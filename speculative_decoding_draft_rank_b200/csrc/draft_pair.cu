@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // This CTA's A rows are in: the even CTA's MMA counts one arrival per CTA.
         auto a_arrive = [&]() {
             if (even) tc::mbar_arrive(a_full);
-            else tc::mbar_arrive_remote(a_full0);
+            else tc::mbar_arrive_remote_release(a_full0);
         };
         const int b = m0 + row;
         const bool rowok = b < B;
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     if (HEAD == kHeadRnn)   // the low parts sit B rows below the high parts
                         tc::tma_load_2d_pair(sA + (nkb + kb) * kPABytes, &mapE, a_full0, kb * kPKB, B + m0, once);
                 }
-                if (!even) tc::mbar_arrive_remote(a_full0);
+                if (!even) tc::mbar_arrive_remote_release(a_full0);
                 tc::mbar_arrive(go);
             }
         }
@@ -603,25 +603,8 @@ cudaError_t launch_pair(const DraftArgs &a, const DraftWs &w, const FinArgs &f, 
     const int pairs = std::max(ep.nPB, std::min(maxc, ep.nPB * nTilesN));
     cfg.gridDim = dim3(2 * pairs);
     if ((e = cudaMemsetAsync(ep.grid_count, 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
-    // Cooperative cluster launches are tried once outside stream capture; where
-    // the combination is refused (or first seen inside a capture) the pairs are
-    // launched as plain clusters, whose grid fits the GPU by the check above.
-    static int coop = -1;   // -1 unknown, 0 refused, 1 accepted
-    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-    if ((e = cudaStreamIsCapturing(st, &cap)) != cudaSuccess) return e;
-    if (coop != 0 && (coop == 1 || cap == cudaStreamCaptureStatusNone)) {
-        attr[1].id = cudaLaunchAttributeCooperative;
-        attr[1].val.cooperative = 1;
-        cfg.numAttrs = 2;
-        e = cudaLaunchKernelEx(&cfg, markov_pair_tc<HEAD>, mW, mL, mE, a.r, nTilesN, ep);
-        if (e == cudaSuccess || coop == 1) {
-            coop = e == cudaSuccess ? 1 : coop;
-            return e;
-        }
-        (void)cudaGetLastError();
-        coop = 0;
-    }
-    cfg.numAttrs = 1;
+    // A plain cluster launch: the grid fits the GPU at once by the check
+    // above, and every CTA waits on the grid barriers with a bounded spin.
     return cudaLaunchKernelEx(&cfg, markov_pair_tc<HEAD>, mW, mL, mE, a.r, nTilesN, ep);
 }
 

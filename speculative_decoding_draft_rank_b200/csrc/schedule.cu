@@ -6,19 +6,21 @@
 // summary, Appendix A: stop as soon as the objective drops, so admitting
 // token k never looks at information from after x_k is drawn).
 //
-// One CTA of 1024 threads does the whole stage:
-//   1. 64-bit keys (~bits(S) above the position-major candidate id i*B + b)
-//      are sorted ascending by a bitonic sort; the keys are unique, so this
-//      is the stable sort by S descending with ties going to the lower id.
-//      Compare-exchange stages with a partner distance of 64 or more go
-//      through shared memory, one barrier each; a warp holds each 64-key
-//      chunk in registers (two keys per lane) for the stages below that and
-//      exchanges with shuffles;
-//   2. fp64 block scan of the sorted survivals gives V_n = B + sum_{j<n} S_(j);
-//   3. every candidate n evaluates the stop test
-//      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index
-//      (or the budget) is the admitted count;
-//   4. admitted candidates are counted per request in shared memory -> ell.
+// The stage runs as one launch of CTAs of 1024 threads:
+//   1. rank by counting, spread over the CTAs: every CTA holds the survivals
+//      (position-major, candidate id i*B + b) in shared memory and each warp
+//      takes one candidate c at a time: its rank in the order "S descending,
+//      ties by the lower id" is #{j : S_j > S_c} + #{j : S_j = S_c, j < c},
+//      counted by the 32 lanes over all candidates (ranks are unique, so the
+//      candidates land in a permutation); the candidate's 64-bit key
+//      (~bits(S) above the id) is written at its rank in the workspace;
+//   2. the last CTA to finish (an arrival counter in the workspace header,
+//      zeroed by a memset before the launch) reads the sorted keys and
+//      admits: fp64 block scan of the sorted survivals gives
+//      V_n = B + sum_{j<n} S_(j); every candidate n evaluates the stop test
+//      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index (or
+//      the budget) is the admitted count;
+//   3. admitted candidates are counted per request in shared memory -> ell.
 // Variants (menfem.com KB entry, "Key Contributions"; paperlayer.ai summary,
 // Appendix A): the offline global search admits the count that maximises
 // Theta(n) = V_n / t(n) over every n up to the budget (lowest n on ties) --
@@ -31,6 +33,8 @@
 // candidates, K read from device memory -- written there by an earlier
 // schedule call on an earlier round -- so one captured graph serves every
 // capacity.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "schedule_variants.cuh"
@@ -53,45 +57,29 @@ __device__ __forceinline__ double profile_at(const int *kn, const double *kt, in
     return kt[lo] + (n - (double)kn[lo]) * slope;
 }
 
-// One bitonic compare-exchange stage (block size k, partner distance j <= 32)
-// on the 64-key chunk a warp holds: lane l has keys e0 = base + 2l and e0 + 1.
-__device__ __forceinline__ void bitonic_warp_step(unsigned long long &v0, unsigned long long &v1, int e0, int k,
-                                                  int j) {
-    const bool up = (e0 & k) == 0;   // the same for e0 and e0 + 1 (k >= 2)
-    if (j == 1) {
-        if ((v0 > v1) == up) { const unsigned long long t = v0; v0 = v1; v1 = t; }
-        return;
-    }
-    const int lane = threadIdx.x & 31, o = j >> 1;   // partner keys sit in lane ^ (j / 2), same slot
-    const unsigned long long o0 = __shfl_xor_sync(0xffffffffu, v0, o);
-    const unsigned long long o1 = __shfl_xor_sync(0xffffffffu, v1, o);
-    const bool keep_min = ((lane & o) == 0) == up;
-    v0 = keep_min ? (v0 < o0 ? v0 : o0) : (v0 > o0 ? v0 : o0);
-    v1 = keep_min ? (v1 < o1 ? v1 : o1) : (v1 > o1 ? v1 : o1);
-}
-
 __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
     const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
-    const int32_t *__restrict__ capacity, WsHeader *hdr,
+    const int32_t *__restrict__ capacity, WsHeader *hdr, unsigned long long *__restrict__ sorted,
     int32_t *__restrict__ ell_out, int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
     int32_t *__restrict__ order_out)
 {
     extern __shared__ __align__(16) unsigned char sched_smem[];
     const int N = B * G;
-    int n2 = 64;
-    while (n2 < N) n2 <<= 1;
-    unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [n2]
-    int *ell_s = reinterpret_cast<int *>(keys + n2);                                  // [B]
+    // Shared memory: the survivals (phase 1), then the sorted keys [N] and the
+    // per-request counts [B] (the admitting CTA).
+    int *ell_s = reinterpret_cast<int *>(sched_smem + sizeof(unsigned long long) * (size_t)N);
+    __shared__ int last_s;
     __shared__ int kn_s[kSchedMaxP];
     __shared__ double kt_s[kSchedMaxP];
     __shared__ int red_i[33];
     __shared__ double red_d[33];
 
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
     for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
 
-    if (mode == DSPARK_SCHED_ALL) {
+    if (mode == DSPARK_SCHED_ALL) {   // one CTA: no order to find
+        if (blockIdx.x != 0) return;
         double acc = 0.0;
         for (int j = tid; j < N; j += blockDim.x) acc += (double)S[j];
         acc = warp_sum_d(acc);
@@ -109,50 +97,37 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
         return;
     }
 
-    // Unique 64-bit keys: ~bits(S) (ascending = S descending, valid for
-    // S >= 0) above the position-major id, so an ascending sort is the stable
-    // sort by S descending.  Padding keys sort last.
-    for (int id = tid; id < n2; id += blockDim.x) {
-        unsigned long long k = ~0ull;
-        if (id < N) {
-            const int i = id / B, b = id - i * B;
-            float s = S[(size_t)b * G + i];
-            if (!(s >= 0.f)) s = 0.f;  // NaN or negative survival ranks last
-            k = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)id;
-        }
-        keys[id] = k;
+    // Phase 1: ranks by counting.  sv holds the survivals position-major
+    // (NaN or negative survivals rank last, as 0).
+    float *sv = reinterpret_cast<float *>(sched_smem);
+    for (int id = tid; id < N; id += blockDim.x) {
+        const int i = id / B, b = id - i * B;
+        float s = S[(size_t)b * G + i];
+        if (!(s >= 0.f)) s = 0.f;
+        sv[id] = s;
     }
     __syncthreads();
-    const int nchunks = n2 >> 6, nwarps = blockDim.x >> 5;
-    // Block sizes 2..64: every stage stays inside one 64-key chunk.
-    for (int c = wid; c < nchunks; c += nwarps) {
-        const int e0 = c * 64 + 2 * lane;
-        unsigned long long v0 = keys[e0], v1 = keys[e0 + 1];
-        for (int k = 2; k <= 64; k <<= 1)
-            for (int j = k >> 1; j > 0; j >>= 1) bitonic_warp_step(v0, v1, e0, k, j);
-        keys[e0] = v0;
-        keys[e0 + 1] = v1;
+    for (int c = (int)blockIdx.x * nwarps + wid; c < N; c += (int)gridDim.x * nwarps) {
+        const float s = sv[c];
+        int cnt = 0;
+        for (int j = lane; j < N; j += 32) {
+            const float t = sv[j];
+            cnt += (t > s) | ((t == s) & (j < c));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) sorted[cnt] = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)c;
     }
+    // The last CTA to finish its candidates admits.
+    __threadfence();
     __syncthreads();
-    for (int k = 128; k <= n2; k <<= 1) {
-        for (int j = k >> 1; j >= 64; j >>= 1) {
-            for (int i = tid; i < (n2 >> 1); i += blockDim.x) {
-                const int lo = 2 * i - (i & (j - 1)), hi = lo + j;
-                const bool up = (lo & k) == 0;
-                const unsigned long long a = keys[lo], c = keys[hi];
-                if ((a > c) == up) { keys[lo] = c; keys[hi] = a; }
-            }
-            __syncthreads();
-        }
-        for (int c = wid; c < nchunks; c += nwarps) {
-            const int e0 = c * 64 + 2 * lane;
-            unsigned long long v0 = keys[e0], v1 = keys[e0 + 1];
-            for (int j = 32; j > 0; j >>= 1) bitonic_warp_step(v0, v1, e0, k, j);
-            keys[e0] = v0;
-            keys[e0 + 1] = v1;
-        }
-        __syncthreads();
-    }
+    if (tid == 0) last_s = atomicAdd(&hdr->pad[kPadSchedArrive], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [N]
+    for (int n = tid; n < N; n += blockDim.x) keys[n] = __ldcg(sorted + n);
+    __syncthreads();
 
     // fp64 prefix of the sorted survivals: V_n = B + sum_{j<n} S_(j).  Thread t
     // owns the contiguous ranks [c0, c1).
@@ -253,38 +228,52 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     }
 }
 
-size_t schedule_ws_bytes(int, int) { return sizeof(WsHeader); }
+// Workspace: the header (status word, arrival counter) and the sorted keys.
+size_t schedule_ws_bytes(int B, int G) { return sizeof(WsHeader) + align256(sizeof(unsigned long long) * (size_t)B * G); }
 
-// Dynamic shared memory of one call: the padded keys and the per-request counts.
+// Dynamic shared memory of one call: the sorted keys (which reuse the
+// survivals' space) and the per-request counts.
 static size_t sched_smem_bytes(int B, int G) {
-    int n2 = 64;
-    while (n2 < B * G) n2 <<= 1;
-    return sizeof(unsigned long long) * (size_t)n2 + sizeof(int) * (size_t)B;
+    return sizeof(unsigned long long) * (size_t)B * G + sizeof(int) * (size_t)B;
 }
 
-cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
-                            const double *knots_t, int P, int budget, int mode, float threshold, void *,
-                            int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
-                            int32_t *order_out, cudaStream_t st) {
+static cudaError_t launch_sched(const float *S, int B, int G, const int32_t *knots_n, const double *knots_t, int P,
+                                int budget, int mode, float threshold, const int32_t *capacity, void *ws,
+                                int32_t *ell_out, int32_t *n_adm_out, double *theta_out, int32_t *order_out,
+                                cudaStream_t st) {
     const size_t smem = sched_smem_bytes(B, G);
     cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096));
     if (e != cudaSuccess) return e;
-    schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, threshold,
-                                                    nullptr, nullptr, ell_out, n_adm_out, theta_out, order_out);
+    WsHeader *hdr = static_cast<WsHeader *>(ws);
+    unsigned long long *sorted = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + sizeof(WsHeader));
+    int grid = 1;
+    if (mode != DSPARK_SCHED_ALL) {
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int warps = kSchedThreads / 32;
+        grid = std::max(1, std::min(sms, (B * G + warps - 1) / warps));   // about one candidate per warp
+        if ((e = cudaMemsetAsync(&hdr->pad[kPadSchedArrive], 0, sizeof(uint32_t), st)) != cudaSuccess) return e;
+    }
+    schedule_kernel<<<grid, kSchedThreads, smem, st>>>(S, B, G, knots_n, knots_t, P, budget, mode, threshold,
+                                                       capacity, hdr, sorted, ell_out, n_adm_out, theta_out,
+                                                       order_out);
     return cudaGetLastError();
+}
+
+cudaError_t launch_schedule(const float *S, int B, int G, const int32_t *knots_n,
+                            const double *knots_t, int P, int budget, int mode, float threshold, void *ws,
+                            int32_t *ell_out, int32_t *n_adm_out, double *theta_out,
+                            int32_t *order_out, cudaStream_t st) {
+    return launch_sched(S, B, G, knots_n, knots_t, P, budget, mode, threshold, nullptr, ws, ell_out, n_adm_out,
+                        theta_out, order_out, st);
 }
 
 cudaError_t launch_schedule_topk(const float *S, int B, int G, const int32_t *capacity, int budget, void *ws,
                                  int32_t *ell_out, int32_t *n_adm_out, int32_t *order_out, cudaStream_t st) {
-    const size_t smem = sched_smem_bytes(B, G);
-    cudaError_t e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(sizeof(unsigned long long) * kSchedMaxN + sizeof(int) * 4096));
-    if (e != cudaSuccess) return e;
-    schedule_kernel<<<1, kSchedThreads, smem, st>>>(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_TOPK, 0.f,
-                                                    capacity, static_cast<WsHeader *>(ws), ell_out, n_adm_out,
-                                                    nullptr, order_out);
-    return cudaGetLastError();
+    return launch_sched(S, B, G, nullptr, nullptr, 0, budget, DSPARK_SCHED_TOPK, 0.f, capacity, ws, ell_out,
+                        n_adm_out, nullptr, order_out, st);
 }
 
 }  // namespace dspark

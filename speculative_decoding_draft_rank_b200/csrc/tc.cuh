@@ -48,14 +48,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
                                                   long long budget) {
     const long long t0 = clock64();
-    for (uint32_t it = 0;; ++it) {
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u) {
-            if (*abort) return false;
-            if (clock64() - t0 > budget) {
-                *abort = 1;
-                return false;
-            }
+        if (*abort) return false;
+        if (clock64() - t0 > budget) {
+            *abort = 1;
+            return false;
         }
     }
 }
@@ -202,8 +200,17 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t a, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
     return r;
 }
-// Arrive once on an mbarrier given by its shared::cluster address (this CTA's or the peer's).
+// Arrive once on an mbarrier given by its shared::cluster address (this CTA's
+// or the peer's), with the default (CTA-scope release) semantics: for
+// arrivals that publish no memory to the other CTA (an accumulator drained
+// into registers), so no cluster-wide ordering of this thread's earlier
+// global stores is waited for.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// The same with a cluster-scope release: for arrivals that publish this
+// CTA's shared-memory writes to work the other CTA starts.
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 // Every thread of both CTAs (an unbounded hardware barrier: each thread

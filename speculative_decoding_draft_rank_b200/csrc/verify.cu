@@ -11,9 +11,9 @@
 // Launch sequence (fixed, graph-capturable; work counts live on the device):
 //   plan        1 CTA: row list of the admitted target rows, rows (b, k) for
 //               k = 0..ell_b (0-based), and their offsets per request.
-//   rows        persistent grid over (row, 8192-column chunk) work items
-//               (bf16: chunks staged in shared memory by bulk copies, a ring
-//               of eight per SM): one streaming pass over each target row,
+//   rows        persistent grid over (row, 4096-column chunk) work items
+//               (bf16: chunks staged in shared memory by bulk copies, two per
+//               consumer warp): one streaming pass over each target row,
 //               giving per chunk the max, lowest argmax and sum of
 //               exp((t - max) / T).
 //   decide      1 CTA per request: row max / Z from the chunk partials,
@@ -30,8 +30,10 @@
 
 namespace dspark {
 
-constexpr int kChunk = 8192;          // columns per row work item
+constexpr int kChunk = 4096;          // columns per row work item
 constexpr int kRowThreads = 256;      // threads of the row and decide kernels
+constexpr int kRowQ = kChunk / (kRowThreads * 8);   // 8-column groups per thread in a chunk (fp32 rows pass)
+constexpr int kColsPerThread = kChunk / kRowThreads;   // columns per thread when a block rescans a chunk
 constexpr int kResRows = 32;          // queued rows per residual tile CTA
 constexpr int kResCols = 256;         // columns per residual tile (fp32, CUDA cores)
 
@@ -142,20 +144,20 @@ __global__ void verify_plan(const int32_t *__restrict__ ell, int B, int G, Verif
 }
 
 // ----------------------------------------------------------------- rows
-// One work item = one 8192-column chunk of one admitted target row.  Each
-// thread owns 32 columns (4 groups of 8 contiguous columns), loads them with
+// One work item = one 4096-column chunk of one admitted target row.  Each
+// thread owns 16 columns (2 groups of 8 contiguous columns), loads them with
 // 16-byte streaming loads one item ahead of the one it reduces, and keeps an
 // online (max, sum of exp((t - max) / T)); the greedy argmax is only tracked
 // for T = 0 rows.  One block merge per item writes the chunk partial.
 template <typename T>
 __device__ __forceinline__ void rows_load(const T *__restrict__ Tlog, const VerifyWs &w, int G, int V, int item,
-                                          float (&v)[4][8]) {
+                                          float (&v)[kRowQ][8]) {
     const int j = item / w.nChunks, c = item - j * w.nChunks;
     const int rk = w.rows[j], b = rk >> 5, k = rk & 31;
     const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
     const int c0 = c * kChunk, c1 = min(V, c0 + kChunk);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kRowQ; ++q) {
         const int i = c0 + (q * kRowThreads + threadIdx.x) * 8;
         if (i < c1) {
             load8(row, i, c1, v[q]);
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
     const int nwork = nrows * w.nChunks;
     int item = blockIdx.x;
     if (item >= nwork) return;
-    float cur[4][8], nxt[4][8];
+    float cur[kRowQ][8], nxt[kRowQ][8];
     rows_load(Tlog, w, G, V, item, cur);
     for (; item < nwork; item += gridDim.x) {
         const int next = item + gridDim.x;
@@ -189,20 +191,20 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
         const float cexp = Tb > 0.f ? kLog2e / Tb : 0.f;
         float m = -INFINITY;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < kRowQ; ++q)
 #pragma unroll
             for (int e = 0; e < 8; ++e) m = fmaxf(m, cur[q][e]);
         int am = 0x7fffffff;
         float s = 0.f;
         if (Tb == 0.f) {   // whole item is one row: the branch is block-uniform
 #pragma unroll
-            for (int q = 3; q >= 0; --q)
+            for (int q = kRowQ - 1; q >= 0; --q)
 #pragma unroll
                 for (int e = 7; e >= 0; --e)
                     if (cur[q][e] == m) am = c * kChunk + (q * kRowThreads + tid) * 8 + e;
         } else if (m > -INFINITY) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kRowQ; ++q)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) s += fast_exp2((cur[q][e] - m) * cexp);
         }
@@ -238,27 +240,30 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
         __syncthreads();
         if (next < nwork) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
+            for (int q = 0; q < kRowQ; ++q)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) cur[q][e] = nxt[q][e];
         }
     }
 }
 
-// bf16 rows: persistent CTAs (one per SM) over the (row, 8192-column chunk)
+// bf16 rows: persistent CTAs (one per SM) over the (row, 4096-column chunk)
 // work items, item q of CTA c being item c + q * grid.  One producer thread
-// streams the CTA's items into a ring of shared-memory stages with bulk copies
+// streams the CTA's items into shared-memory stages with bulk copies
 // (evict-first: every target row is read once, so the transition factor that
 // drafting left in L2 stays there for the residual pass) and writes each
-// stage's item description beside it; eight consumer warps reduce a staged
-// chunk together (warp w: columns [w * 1024, w * 1024 + 1024), lane l reading
-// 16-byte pieces l, l + 32, ... of that range, bank-conflict free), release the
-// stage as soon as its values are in registers, and merge their (max, sum of
-// exp((t - max) / T), lowest argmax) after one named barrier.
-constexpr int kVrStages = 8;
+// stage's item description beside it.  Item q belongs to consumer warp
+// q % 8, which owns two stages and alternates between them, so its next chunk
+// lands while it reduces the current one; it releases a stage as soon as the
+// values are in registers, reduces its 4096 columns to (max, sum of
+// exp((t - max) / T), lowest argmax) and writes the chunk partial itself -- no
+// block barrier and no cross-warp merge.  Lane l reads the 16-byte pieces
+// l, l + 32, ... of the chunk (bank-conflict free).
 constexpr int kVrWarps = 8;
+constexpr int kVrStages = 2 * kVrWarps;
 constexpr int kVrThreads = (kVrWarps + 1) * 32;
-constexpr int kVrStageBytes = kChunk * 2;
+constexpr int kVrStageBytes = kChunk * 2;          // 8 KB
+constexpr int kVrPieces = kVrStageBytes / 16 / 32;   // 16-byte pieces per lane (16)
 constexpr long long kVrWaitBudget = 4000000000LL;   // ~2 s of SM clock
 
 struct VrMeta {
@@ -270,27 +275,25 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
                                                                  const float *__restrict__ temp, int G, int V,
                                                                  VerifyWs w, long long budget) {
     extern __shared__ __align__(128) unsigned char vr_smem[];
-    unsigned char *stages = vr_smem;                                                // [S][16 KB]
+    unsigned char *stages = vr_smem;                                                // [S][8 KB]
     uint64_t *full = reinterpret_cast<uint64_t *>(vr_smem + kVrStages * kVrStageBytes);
     uint64_t *empty = full + kVrStages;
     VrMeta *meta = reinterpret_cast<VrMeta *>(empty + kVrStages);                   // [S]
-    __shared__ float pm[2][kVrWarps], ps[2][kVrWarps];
-    __shared__ int pa[2][kVrWarps];
     __shared__ int abort_s;
-    __shared__ int stop_s[2];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
     const int nwork = nrows * w.nChunks;
     if ((int)blockIdx.x >= nwork) return;
     const int nmine = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     if (threadIdx.x == 0) {
-        for (int q = 0; q < kVrStages; ++q) { tc::mbar_init(&full[q], 1); tc::mbar_init(&empty[q], kVrWarps); }
+        for (int q = 0; q < kVrStages; ++q) { tc::mbar_init(&full[q], 1); tc::mbar_init(&empty[q], 1); }
         abort_s = 0;
-        stop_s[0] = stop_s[1] = 0;
         tc::fence_barrier_init();
     }
     __syncthreads();
     volatile int *abort_flag = &abort_s;
+    // Item q: warp q % 8, stage q % 8 + 8 * ((q / 8) & 1), use (q / 16) of that stage.
+    auto stage_of = [](int q) { return (q % kVrWarps) + kVrWarps * ((q / kVrWarps) & 1); };
 
     if (warp == kVrWarps) {
         // ------------------------------------------------------ producer
@@ -317,8 +320,8 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
                 const int ji = __shfl_sync(0xffffffffu, j, i);
                 const float Ti = __shfl_sync(0xffffffffu, Tb, i);
                 if (lane == 0) {
-                    const int s = q % kVrStages;
-                    ok = tc::mbar_wait_bounded(&empty[s], ((q / kVrStages) & 1) ^ 1, abort_flag, budget);
+                    const int s = stage_of(q), use = q / kVrStages;
+                    ok = tc::mbar_wait_bounded(&empty[s], (use & 1) ^ 1, abort_flag, budget);
                     if (ok) {
                         const int c0 = ci * kChunk, ncols = min(kChunk, V - c0);
                         const float T = Ti >= 0.f ? Ti : 0.f;
@@ -339,76 +342,88 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
             int dummy = 0;
             for (int d = 0; d < kVrStages && q - 1 - d >= 0; ++d) {
                 const int qq = q - 1 - d;
-                tc::mbar_wait_bounded(&full[qq % kVrStages], (qq / kVrStages) & 1, &dummy, kVrWaitBudget / 4);
+                tc::mbar_wait_bounded(&full[stage_of(qq)], (qq / kVrStages) & 1, &dummy, kVrWaitBudget / 4);
             }
             flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
         }
     } else {
         // ------------------------------------------------------ consumers
-        // A warp whose wait ran out raises stop[q & 1] before the item's
-        // named barrier, and every consumer warp leaves after that barrier
-        // when it is set; the flags only ever go from 0 to 1, and
-        // alternate by item parity, so all eight warps take the same exit.
-        for (int q = 0; q < nmine; ++q) {
-            const int s = q % kVrStages;
-            const int par = q & 1;
-            bool ok = tc::mbar_wait_bounded(&full[s], (q / kVrStages) & 1, abort_flag, budget);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) {
+        for (int q = warp; q < nmine; q += kVrWarps) {
+            const int s = stage_of(q), use = q / kVrStages;
+            bool ok = tc::mbar_wait_bounded(&full[s], use & 1, abort_flag, budget);
+            if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) {
-                    stop_s[par] = 1;
                     *abort_flag = 1;
                     flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
                 }
-                asm volatile("bar.sync 1, %0;" ::"r"(kVrWarps * 32) : "memory");
                 break;
             }
             const VrMeta md = meta[s];
-            uint4 v[4];
-            const unsigned char *src = stages + s * kVrStageBytes + warp * 2048 + lane * 16;
+            uint4 v[kVrPieces];
+            const unsigned char *src = stages + s * kVrStageBytes + lane * 16;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
+            for (int i = 0; i < kVrPieces; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
             tc::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&empty[s]);   // the values are in registers
-            // Column of piece i, element e: base + i * 256 + e.
-            const int base = warp * 1024 + lane * 8;
-            float t[32];
+            // Column of piece i, element e: i * 256 + lane * 8 + e.
+            const int cexp_zero = md.cexp == 0.f;
+            const float cexp = md.cexp;
+            if (md.ncols < kChunk) {   // the row's last chunk: columns past V are -inf (bf16 0xff80)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t ww[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                for (int i = 0; i < kVrPieces; ++i) {
+                    uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    t[i * 8 + 2 * h] = bf16lo(ww[h]);
-                    t[i * 8 + 2 * h + 1] = bf16hi(ww[h]);
+                    for (int h = 0; h < 4; ++h) {
+                        const int col = i * 256 + lane * 8 + 2 * h;
+                        if (col >= md.ncols) wq[h] = (wq[h] & 0xffff0000u) | 0xff80u;
+                        if (col + 1 >= md.ncols) wq[h] = (wq[h] & 0x0000ffffu) | 0xff800000u;
+                    }
+                    v[i] = make_uint4(wq[0], wq[1], wq[2], wq[3]);
                 }
             }
-            if (md.ncols < kChunk) {   // the row's last chunk: columns past V are -inf
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (base + i * 256 + e >= md.ncols) t[i * 8 + e] = -INFINITY;
-            }
+            // Maximum: running three-input maxima over the value pairs.
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) m4[(e >> 1) & 3] = max3(m4[(e >> 1) & 3], t[e], t[e + 1]);
+            for (int i = 0; i < kVrPieces; ++i) {
+                m4[0] = max3(m4[0], bf16lo(v[i].x), bf16hi(v[i].x));
+                m4[1] = max3(m4[1], bf16lo(v[i].y), bf16hi(v[i].y));
+                m4[2] = max3(m4[2], bf16lo(v[i].z), bf16hi(v[i].z));
+                m4[3] = max3(m4[3], bf16lo(v[i].w), bf16hi(v[i].w));
+            }
             float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             float sum = 0.f;
             int am = 0x7fffffff;
-            const float cexp = md.cexp;
-            if (cexp == 0.f) {   // greedy row (warp-uniform): the lowest index of the largest value
+            if (cexp_zero) {   // greedy row (warp-uniform): the lowest index of the largest value
 #pragma unroll
-                for (int i = 3; i >= 0; --i)
+                for (int i = kVrPieces - 1; i >= 0; --i) {
+                    const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-                    for (int e = 7; e >= 0; --e)
-                        if (t[i * 8 + e] == m) am = md.c * kChunk + base + i * 256 + e;
+                    for (int h = 3; h >= 0; --h) {
+                        if (bf16hi(wq[h]) == m) am = md.c * kChunk + i * 256 + lane * 8 + 2 * h + 1;
+                        if (bf16lo(wq[h]) == m) am = md.c * kChunk + i * 256 + lane * 8 + 2 * h;
+                    }
+                }
             } else if (m > -INFINITY) {
+                // exp((t - m) / T) = 2^(t * cexp - m * cexp): one paired fused
+                // multiply-add per two columns, then the two ex2.
+                const float2 c2 = make_float2(cexp, cexp);
                 const float nmc = -m * cexp;
-                float a4[4] = {0.f, 0.f, 0.f, 0.f};
+                const float2 n2 = make_float2(nmc, nmc);
+                float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int e = 0; e < 32; ++e) a4[e & 3] += fast_exp2(fmaf(t[e], cexp, nmc));
-                sum = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+                for (int i = 0; i < kVrPieces; ++i) {
+                    const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float2 arg = fma2(make_float2(bf16lo(wq[h]), bf16hi(wq[h])), c2, n2);
+                        s2[h] = add2(s2[h], make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
+                    }
+                }
+                const float2 p01 = add2(s2[0], s2[1]), p23 = add2(s2[2], s2[3]);
+                const float2 pall = add2(p01, p23);
+                sum = pall.x + pall.y;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -416,28 +431,17 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
                 const float os = __shfl_xor_sync(0xffffffffu, sum, o);
                 const int oa = __shfl_xor_sync(0xffffffffu, am, o);
                 const float nm = fmaxf(m, om);
-                if (cexp > 0.f)
+                if (!cexp_zero)
                     sum = (m > -INFINITY ? sum * fast_exp2((m - nm) * cexp) : 0.f) +
                           (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
                 if (om > m || (om == m && oa < am)) am = oa;
                 m = nm;
             }
-            if (lane == 0) { pm[par][warp] = m; ps[par][warp] = sum; pa[par][warp] = am; }
-            asm volatile("bar.sync 1, %0;" ::"r"(kVrWarps * 32) : "memory");
-            if (*reinterpret_cast<volatile int *>(&stop_s[par])) break;
-            if (warp == 0 && lane == 0) {
-                float M = pm[par][0];
-                int A = pa[par][0];
-                for (int x = 1; x < kVrWarps; ++x)
-                    if (pm[par][x] > M || (pm[par][x] == M && pa[par][x] < A)) { M = pm[par][x]; A = pa[par][x]; }
-                float S = 0.f;
-                if (cexp > 0.f)
-                    for (int x = 0; x < kVrWarps; ++x)
-                        if (pm[par][x] > -INFINITY) S += ps[par][x] * fast_exp2((pm[par][x] - M) * cexp);
+            if (lane == 0) {
                 const size_t o = (size_t)md.j * w.nChunks + md.c;
-                w.cm[o] = M;
-                w.cs[o] = S;
-                w.ca[o] = A;
+                w.cm[o] = m;
+                w.cs[o] = sum;
+                w.ca[o] = am;
             }
         }
     }
@@ -477,7 +481,7 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
     const float *cm = w.cm + (size_t)j * w.nChunks;
     const float *cs = w.cs + (size_t)j * w.nChunks;
     const float target = u * Z;
-    // Prefix over chunk sums (nChunks <= 128 for V <= 2^20; kRowThreads >= that).
+    // Prefix over chunk sums (nChunks <= 256 for V <= 2^20; kRowThreads >= that).
     const float wc = tid < w.nChunks ? cs[tid] * exp_e((cm[tid] - M) * invT) : 0.f;
     float tot;
     const float inc = block_scan1(wc, s_c, &tot);
@@ -492,11 +496,11 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
     const float rem = target - excl_s;
     const T *row = Tlog + ((size_t)b * (G + 1) + k) * V;
     const int c0 = ch * kChunk, c1 = min(V, c0 + kChunk);
-    const int i0 = c0 + tid * 32;   // this thread's 32 consecutive columns
-    float e[32];
+    const int i0 = c0 + tid * kColsPerThread;   // this thread's consecutive columns
+    float e[kColsPerThread];
     float run = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kColsPerThread / 8; ++q) {
         float v[8];
         const int i = i0 + q * 8;
         if (i < c1) load8(row, i, c1, v);
@@ -516,7 +520,7 @@ __device__ int sample_target_row(const T *__restrict__ Tlog, const VerifyWs &w, 
         int f = -1, lastpos = -1;
         float margin = 0.f;
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
+        for (int t = 0; t < kColsPerThread; ++t) {
             if (f < 0 && e[t] > 0.f) {
                 lastpos = i0 + t;
                 p += e[t];

@@ -12,8 +12,8 @@
 //   plan        1 CTA: row list of the admitted target rows, rows (b, k) for
 //               k = 0..ell_b (0-based), and their offsets per request.
 //   rows        persistent grid over (row, 4096-column chunk) work items
-//               (bf16: chunks staged in shared memory by bulk copies, two per
-//               consumer warp): one streaming pass over each target row,
+//               (bf16: chunks staged in shared memory by bulk copies, two
+//               stages per warp): one streaming pass over each target row,
 //               giving per chunk the max, lowest argmax and sum of
 //               exp((t - max) / T).
 //   decide      1 CTA per request: row max / Z from the chunk partials,
@@ -248,37 +248,34 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
 }
 
 // bf16 rows: persistent CTAs (one per SM) over the (row, 4096-column chunk)
-// work items, item q of CTA c being item c + q * grid.  One producer thread
-// streams the CTA's items into shared-memory stages with bulk copies
-// (evict-first: every target row is read once, so the transition factor that
-// drafting left in L2 stays there for the residual pass) and writes each
-// stage's item description beside it.  Item q belongs to consumer warp
-// q % 8, which owns two stages and alternates between them, so its next chunk
-// lands while it reduces the current one; it releases a stage as soon as the
-// values are in registers, reduces its 4096 columns to (max, sum of
-// exp((t - max) / T), lowest argmax) and writes the chunk partial itself -- no
-// block barrier and no cross-warp merge.  Lane l reads the 16-byte pieces
-// l, l + 32, ... of the chunk (bank-conflict free).
+// work items, item q of CTA c being item c + q * grid.  Warp w of the CTA
+// takes items q = w, w + 8, ... and streams them itself: it owns two
+// shared-memory stages and keeps a bulk copy in flight into one while it
+// reduces the other (evict-first: every target row is read once, so the
+// transition factor that drafting left in L2 stays there for the residual
+// pass).  As soon as a chunk's values are in registers the warp issues the
+// copy two items ahead into the stage it just read, reduces its 4096 columns
+// to (max, sum of exp((t - max) / T), lowest argmax) and writes the chunk
+// partial -- no block barrier, no producer to wait for.  The row of an item
+// comes from the compacted row list, read 32 items ahead; temperatures are
+// staged in shared memory.  Lane l reads the 16-byte pieces l, l + 32, ...
+// of the chunk (bank-conflict free).
 constexpr int kVrWarps = 8;
-constexpr int kVrStages = 2 * kVrWarps;
-constexpr int kVrThreads = (kVrWarps + 1) * 32;
-constexpr int kVrStageBytes = kChunk * 2;          // 8 KB
+constexpr int kVrThreads = kVrWarps * 32;
+constexpr int kVrStageBytes = kChunk * 2;            // 8 KB
 constexpr int kVrPieces = kVrStageBytes / 16 / 32;   // 16-byte pieces per lane (16)
 constexpr long long kVrWaitBudget = 4000000000LL;   // ~2 s of SM clock
 
-struct VrMeta {
-    int j, c, ncols;
-    float cexp;
-};
+__host__ inline size_t vr_smem_bytes(int B) {
+    return (size_t)kVrWarps * 2 * kVrStageBytes + (size_t)kVrWarps * 2 * sizeof(uint64_t) + sizeof(float) * (size_t)B;
+}
 
 __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfloat16 *__restrict__ Tlog,
-                                                                 const float *__restrict__ temp, int G, int V,
+                                                                 const float *__restrict__ temp, int B, int G, int V,
                                                                  VerifyWs w, long long budget) {
     extern __shared__ __align__(128) unsigned char vr_smem[];
-    unsigned char *stages = vr_smem;                                                // [S][8 KB]
-    uint64_t *full = reinterpret_cast<uint64_t *>(vr_smem + kVrStages * kVrStageBytes);
-    uint64_t *empty = full + kVrStages;
-    VrMeta *meta = reinterpret_cast<VrMeta *>(empty + kVrStages);                   // [S]
+    uint64_t *full = reinterpret_cast<uint64_t *>(vr_smem + kVrWarps * 2 * kVrStageBytes);   // [warp][2]
+    float *temp_s = reinterpret_cast<float *>(full + kVrWarps * 2);                            // [B]
     __shared__ int abort_s;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
@@ -286,163 +283,151 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
     if ((int)blockIdx.x >= nwork) return;
     const int nmine = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     if (threadIdx.x == 0) {
-        for (int q = 0; q < kVrStages; ++q) { tc::mbar_init(&full[q], 1); tc::mbar_init(&empty[q], 1); }
+        for (int q = 0; q < kVrWarps * 2; ++q) tc::mbar_init(&full[q], 1);
         abort_s = 0;
         tc::fence_barrier_init();
     }
+    for (int b = threadIdx.x; b < B; b += blockDim.x) temp_s[b] = temp[b];
     __syncthreads();
     volatile int *abort_flag = &abort_s;
-    // Item q: warp q % 8, stage q % 8 + 8 * ((q / 8) & 1), use (q / 16) of that stage.
-    auto stage_of = [](int q) { return (q % kVrWarps) + kVrWarps * ((q / kVrWarps) & 1); };
-
-    if (warp == kVrWarps) {
-        // ------------------------------------------------------ producer
-        // The warp loads the item descriptions 32 at a time (row ids, then
-        // temperatures); lane 0 issues the copies.
-        const uint64_t pol = tc::policy_evict_first();
-        bool ok = true;
-        int q = 0;
-        for (int q0 = 0; q0 < nmine && ok; q0 += 32) {
-            const int ql = q0 + lane;
-            int rk = 0, c = 0, j = 0;
-            float Tb = 0.f;
-            if (ql < nmine) {
-                const int item = (int)blockIdx.x + ql * (int)gridDim.x;
-                j = item / w.nChunks;
-                c = item - j * w.nChunks;
-                rk = w.rows[j];
-                Tb = temp[rk >> 5];
-            }
-            const int nb = min(32, nmine - q0);
-            for (int i = 0; i < nb; ++i, ++q) {
-                const int rki = __shfl_sync(0xffffffffu, rk, i);
-                const int ci = __shfl_sync(0xffffffffu, c, i);
-                const int ji = __shfl_sync(0xffffffffu, j, i);
-                const float Ti = __shfl_sync(0xffffffffu, Tb, i);
-                if (lane == 0) {
-                    const int s = stage_of(q), use = q / kVrStages;
-                    ok = tc::mbar_wait_bounded(&empty[s], (use & 1) ^ 1, abort_flag, budget);
-                    if (ok) {
-                        const int c0 = ci * kChunk, ncols = min(kChunk, V - c0);
-                        const float T = Ti >= 0.f ? Ti : 0.f;
-                        meta[s] = VrMeta{ji, ci, ncols, T > 0.f ? kLog2e / T : 0.f};
-                        const __nv_bfloat16 *src =
-                            Tlog + ((size_t)(rki >> 5) * (G + 1) + (rki & 31)) * V + c0;
-                        tc::mbar_arrive_expect_tx(&full[s], (uint32_t)ncols * 2);
-                        tc::bulk_load(stages + s * kVrStageBytes, src, (uint32_t)ncols * 2, &full[s], pol);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-            }
+    unsigned char *stage0 = vr_smem + warp * 2 * kVrStageBytes;
+    uint64_t *myfull = full + warp * 2;
+    const int nk = (nmine - warp + kVrWarps - 1) / kVrWarps;   // this warp's items: k = 0..nk-1
+    auto item_of = [&](int k) { return (int)blockIdx.x + (warp + kVrWarps * k) * (int)gridDim.x; };
+    auto load_rk = [&](int k) { return k < nk ? w.rows[item_of(k) / w.nChunks] : 0; };
+    // Row ids of items base .. base + 63: lane l holds items base + l (cur) and base + 32 + l (nxt).
+    int base = 0, cur = load_rk(lane), nxt = load_rk(32 + lane);
+    auto rk_of = [&](int k) {
+        const int a = __shfl_sync(0xffffffffu, cur, (k - base) & 31);
+        const int b2 = __shfl_sync(0xffffffffu, nxt, (k - base) & 31);
+        return (k - base) < 32 ? a : b2;
+    };
+    const uint64_t pol = tc::policy_evict_first();
+    auto issue = [&](int k) {
+        const int rk = rk_of(k);
+        if (lane == 0) {
+            const int item = item_of(k);
+            const int c = item % w.nChunks;
+            const int c0 = c * kChunk, ncols = min(kChunk, V - c0);
+            const __nv_bfloat16 *src = Tlog + ((size_t)(rk >> 5) * (G + 1) + (rk & 31)) * V + c0;
+            tc::mbar_arrive_expect_tx(&myfull[k & 1], (uint32_t)ncols * 2);
+            tc::bulk_load(stage0 + (k & 1) * kVrStageBytes, src, (uint32_t)ncols * 2, &myfull[k & 1], pol);
         }
-        if (!ok && lane == 0) {
-            // Give up: wait (bounded, ignoring the abort flag) for the copies
-            // in flight so that none lands after the CTA exits.
-            int dummy = 0;
-            for (int d = 0; d < kVrStages && q - 1 - d >= 0; ++d) {
-                const int qq = q - 1 - d;
-                tc::mbar_wait_bounded(&full[stage_of(qq)], (qq / kVrStages) & 1, &dummy, kVrWaitBudget / 4);
-            }
-            flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
+    };
+    if (nk > 0) issue(0);
+    if (nk > 1) issue(1);
+    int issued = min(nk, 2);
+    for (int k = 0; k < nk; ++k) {
+        if (k - base == 32) {   // slide the row-id window by 32 items
+            cur = nxt;
+            base += 32;
+            nxt = load_rk(base + 32 + lane);
         }
-    } else {
-        // ------------------------------------------------------ consumers
-        for (int q = warp; q < nmine; q += kVrWarps) {
-            const int s = stage_of(q), use = q / kVrStages;
-            bool ok = tc::mbar_wait_bounded(&full[s], use & 1, abort_flag, budget);
-            if (!__all_sync(0xffffffffu, ok)) {
-                if (lane == 0) {
-                    *abort_flag = 1;
-                    flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
-                }
-                break;
+        const bool ok = tc::mbar_wait_bounded(&myfull[k & 1], (k >> 1) & 1, abort_flag, budget);
+        if (!__all_sync(0xffffffffu, ok)) {
+            // Give up: wait (bounded, ignoring the abort flag) for this warp's
+            // copies in flight so that none lands after the CTA exits.
+            if (lane == 0) {
+                int dummy = 0;
+                for (int kk = k; kk < issued; ++kk)
+                    tc::mbar_wait_bounded(&myfull[kk & 1], (kk >> 1) & 1, &dummy, kVrWaitBudget / 4);
+                *abort_flag = 1;
+                flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
             }
-            const VrMeta md = meta[s];
-            uint4 v[kVrPieces];
-            const unsigned char *src = stages + s * kVrStageBytes + lane * 16;
+            break;
+        }
+        uint4 v[kVrPieces];
+        const unsigned char *src = stage0 + (k & 1) * kVrStageBytes + lane * 16;
 #pragma unroll
-            for (int i = 0; i < kVrPieces; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&empty[s]);   // the values are in registers
-            // Column of piece i, element e: i * 256 + lane * 8 + e.
-            const int cexp_zero = md.cexp == 0.f;
-            const float cexp = md.cexp;
-            if (md.ncols < kChunk) {   // the row's last chunk: columns past V are -inf (bf16 0xff80)
-#pragma unroll
-                for (int i = 0; i < kVrPieces; ++i) {
-                    uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const int col = i * 256 + lane * 8 + 2 * h;
-                        if (col >= md.ncols) wq[h] = (wq[h] & 0xffff0000u) | 0xff80u;
-                        if (col + 1 >= md.ncols) wq[h] = (wq[h] & 0x0000ffffu) | 0xff800000u;
-                    }
-                    v[i] = make_uint4(wq[0], wq[1], wq[2], wq[3]);
-                }
-            }
-            // Maximum: running three-input maxima over the value pairs.
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        for (int i = 0; i < kVrPieces; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
+        const int rk = rk_of(k);
+        // The stage is free once every lane's reads are done: the next copy may
+        // land in it (generic reads, then async-proxy writes).
+        tc::fence_proxy_async_smem();
+        __syncwarp();
+        if (k + 2 < nk) {
+            issue(k + 2);
+            issued = k + 3;
+        }
+        const int item = item_of(k);
+        const int jrow = item / w.nChunks, ch = item - jrow * w.nChunks;
+        const int ncols = min(kChunk, V - ch * kChunk);
+        float T = temp_s[rk >> 5];
+        T = T >= 0.f ? T : 0.f;
+        const float cexp = T > 0.f ? kLog2e / T : 0.f;
+        if (ncols < kChunk) {   // the row's last chunk: columns past V are -inf (bf16 0xff80)
 #pragma unroll
             for (int i = 0; i < kVrPieces; ++i) {
-                m4[0] = max3(m4[0], bf16lo(v[i].x), bf16hi(v[i].x));
-                m4[1] = max3(m4[1], bf16lo(v[i].y), bf16hi(v[i].y));
-                m4[2] = max3(m4[2], bf16lo(v[i].z), bf16hi(v[i].z));
-                m4[3] = max3(m4[3], bf16lo(v[i].w), bf16hi(v[i].w));
-            }
-            float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            float sum = 0.f;
-            int am = 0x7fffffff;
-            if (cexp_zero) {   // greedy row (warp-uniform): the lowest index of the largest value
+                uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
-                for (int i = kVrPieces - 1; i >= 0; --i) {
-                    const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-                    for (int h = 3; h >= 0; --h) {
-                        if (bf16hi(wq[h]) == m) am = md.c * kChunk + i * 256 + lane * 8 + 2 * h + 1;
-                        if (bf16lo(wq[h]) == m) am = md.c * kChunk + i * 256 + lane * 8 + 2 * h;
-                    }
+                for (int h = 0; h < 4; ++h) {
+                    const int col = i * 256 + lane * 8 + 2 * h;
+                    if (col >= ncols) wq[h] = (wq[h] & 0xffff0000u) | 0xff80u;
+                    if (col + 1 >= ncols) wq[h] = (wq[h] & 0x0000ffffu) | 0xff800000u;
                 }
-            } else if (m > -INFINITY) {
-                // exp((t - m) / T) = 2^(t * cexp - m * cexp): one paired fused
-                // multiply-add per two columns, then the two ex2.
-                const float2 c2 = make_float2(cexp, cexp);
-                const float nmc = -m * cexp;
-                const float2 n2 = make_float2(nmc, nmc);
-                float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                make_float2(0.f, 0.f)};
+                v[i] = make_uint4(wq[0], wq[1], wq[2], wq[3]);
+            }
+        }
+        // Maximum: running three-input maxima over the value pairs.
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-                for (int i = 0; i < kVrPieces; ++i) {
-                    const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+        for (int i = 0; i < kVrPieces; ++i) {
+            m4[0] = max3(m4[0], bf16lo(v[i].x), bf16hi(v[i].x));
+            m4[1] = max3(m4[1], bf16lo(v[i].y), bf16hi(v[i].y));
+            m4[2] = max3(m4[2], bf16lo(v[i].z), bf16hi(v[i].z));
+            m4[3] = max3(m4[3], bf16lo(v[i].w), bf16hi(v[i].w));
+        }
+        float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        float sum = 0.f;
+        int am = 0x7fffffff;
+        if (cexp == 0.f) {   // greedy row (warp-uniform): the lowest index of the largest value
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float2 arg = fma2(make_float2(bf16lo(wq[h]), bf16hi(wq[h])), c2, n2);
-                        s2[h] = add2(s2[h], make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
-                    }
+            for (int i = kVrPieces - 1; i >= 0; --i) {
+                const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int h = 3; h >= 0; --h) {
+                    if (bf16hi(wq[h]) == m) am = ch * kChunk + i * 256 + lane * 8 + 2 * h + 1;
+                    if (bf16lo(wq[h]) == m) am = ch * kChunk + i * 256 + lane * 8 + 2 * h;
                 }
-                const float2 p01 = add2(s2[0], s2[1]), p23 = add2(s2[2], s2[3]);
-                const float2 pall = add2(p01, p23);
-                sum = pall.x + pall.y;
             }
+        } else if (m > -INFINITY) {
+            // exp((t - m) / T) = 2^(t * cexp - m * cexp): one paired fused
+            // multiply-add per two columns, then the two ex2.
+            const float2 c2 = make_float2(cexp, cexp);
+            const float nmc = -m * cexp;
+            const float2 n2 = make_float2(nmc, nmc);
+            float2 s2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float om = __shfl_xor_sync(0xffffffffu, m, o);
-                const float os = __shfl_xor_sync(0xffffffffu, sum, o);
-                const int oa = __shfl_xor_sync(0xffffffffu, am, o);
-                const float nm = fmaxf(m, om);
-                if (!cexp_zero)
-                    sum = (m > -INFINITY ? sum * fast_exp2((m - nm) * cexp) : 0.f) +
-                          (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
-                if (om > m || (om == m && oa < am)) am = oa;
-                m = nm;
+            for (int i = 0; i < kVrPieces; ++i) {
+                const uint32_t wq[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const float2 arg = fma2(make_float2(bf16lo(wq[h]), bf16hi(wq[h])), c2, n2);
+                    s2[h] = add2(s2[h], make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
+                }
             }
-            if (lane == 0) {
-                const size_t o = (size_t)md.j * w.nChunks + md.c;
-                w.cm[o] = m;
-                w.cs[o] = sum;
-                w.ca[o] = am;
-            }
+            const float2 p01 = add2(s2[0], s2[1]), p23 = add2(s2[2], s2[3]);
+            const float2 pall = add2(p01, p23);
+            sum = pall.x + pall.y;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, m, o);
+            const float os = __shfl_xor_sync(0xffffffffu, sum, o);
+            const int oa = __shfl_xor_sync(0xffffffffu, am, o);
+            const float nm = fmaxf(m, om);
+            if (cexp > 0.f)
+                sum = (m > -INFINITY ? sum * fast_exp2((m - nm) * cexp) : 0.f) +
+                      (om > -INFINITY ? os * fast_exp2((om - nm) * cexp) : 0.f);
+            if (om > m || (om == m && oa < am)) am = oa;
+            m = nm;
+        }
+        if (lane == 0) {
+            const size_t o = (size_t)jrow * w.nChunks + ch;
+            w.cm[o] = m;
+            w.cs[o] = sum;
+            w.ca[o] = am;
         }
     }
 }
@@ -844,13 +829,12 @@ static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaS
     const int maxwork = a.B * (a.G + 1) * w.nChunks;
     if (a.dtype == DSPARK_BF16) {
         const int grid = max(1, min(maxwork, sms));
-        const size_t smem = (size_t)kVrStages * kVrStageBytes + 2 * kVrStages * sizeof(uint64_t) +
-                            kVrStages * sizeof(VrMeta);
+        const size_t smem = vr_smem_bytes(a.B);
         if ((e = cudaFuncSetAttribute(verify_rows_bulk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
             cudaSuccess)
             return e;
-        verify_rows_bulk<<<grid, kVrThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp, a.G,
-                                                         a.V, w, wait_budget(kVrWaitBudget));
+        verify_rows_bulk<<<grid, kVrThreads, smem, st>>>(static_cast<const __nv_bfloat16 *>(a.Tlog), a.temp, a.B,
+                                                         a.G, a.V, w, wait_budget(kVrWaitBudget));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     } else {
         const int grid = max(1, min(maxwork, sms * 8));

@@ -49,6 +49,6 @@ def test_fullsize_wide_sample(make, n, capsys):
                             rep)
     residual = int(np.sum(o.final_kind == 0))
     with capsys.disabled():
-        print(f"\n{w.name}: {len(idx)} requests, {residual} residual draws, near-ties {rep.near_ties}")
+        print(f"\n{w.name}: {len(idx)} requests, {residual} residual draws; {rep.summary()}")
     assert residual >= 20
-    assert rep.total_ties() <= 1, rep.near_ties
+    parity.assert_few_ties(rep)

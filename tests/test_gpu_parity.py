@@ -52,7 +52,7 @@ def test_round_parity_small(dtype, B, G, V, r, d):
     out, rep = _check_round(inp, dr, *PROFILE, -1, 1)
     # At a 1e-5 margin a counted near-tie is a rare event (about 2e-5 per
     # decision, and a disagreement needs a far smaller margin still).
-    assert rep.total_ties() <= 1, rep.near_ties
+    parity.assert_few_ties(rep)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

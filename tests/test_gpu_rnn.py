@@ -61,7 +61,7 @@ def test_rnn_round_parity(B, G, V, r):
                           *PROFILE, -1, 1, G, rep)
     parity.check_verify(inp, idx, out["x"], out["ell"], out["acc"], out["tokens"], out["nout"], out["pt_x"], rep,
                         A=A)
-    assert rep.total_ties() <= 1, rep.near_ties
+    parity.assert_few_ties(rep)
 
 
 def test_rnn_verify_everything():
@@ -77,7 +77,7 @@ def test_rnn_verify_everything():
     o = parity.check_verify(inp, idx, out["x"], out["ell"], out["acc"], out["tokens"], out["nout"], out["pt_x"],
                             rep, A=A)
     assert int(np.sum(o.final_kind == 0)) >= 20
-    assert rep.total_ties() <= 1, rep.near_ties
+    parity.assert_few_ties(rep)
 
 
 def test_rnn_head_differs_from_markov_head():

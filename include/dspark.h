@@ -362,6 +362,15 @@ dspark_status dspark_clear_device_status(void *ws, void *stream);
  * Synchronises `stream`. */
 dspark_status dspark_get_near_ties(const void *ws, void *stream, uint32_t *draft_out, uint32_t *verify_out);
 
+/* Diagnostics: y[i] = 2^x[i] by the FMA-pipe polynomial that shares the
+ * exponentials of the verification row pass with the special-function unit
+ * (x = n + f, n = rint(x), f in [-1/2, 1/2]; 2^f from a degree-5 polynomial;
+ * 2^n added to the exponent bits).  Relative error within 4e-7 of 2^x for
+ * -125 <= x <= 0; arguments below -125 give 2^-125.  x, y: device arrays of n
+ * floats (n >= 0), enqueued on `stream`.  DSPARK_ERR_INVALID_ARG for a null
+ * pointer with n > 0 or a negative n. */
+dspark_status dspark_exp2_fma(const float *x, float *y, int n, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,7 +32,8 @@ EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov
            "dspark_verify", "dspark_get_device_status", "dspark_clear_device_status",
            "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold",
            "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc", "dspark_schedule_topk",
-           "dspark_draft_noalloc_device_status", "dspark_draft_rnn", "dspark_verify_rnn", "dspark_get_near_ties")
+           "dspark_draft_noalloc_device_status", "dspark_draft_rnn", "dspark_verify_rnn", "dspark_get_near_ties",
+           "dspark_exp2_fma")
 
 
 class DsparkError(RuntimeError):
@@ -73,6 +74,8 @@ def load() -> ctypes.CDLL:
     lib.dspark_verify.argtypes = [_vp] * 13 + [_i] * 5 + [_vp, _sz] + [_vp] * 5
     lib.dspark_get_device_status.restype = _i
     lib.dspark_get_device_status.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]
+    lib.dspark_exp2_fma.restype = _i
+    lib.dspark_exp2_fma.argtypes = [_vp, _vp, _i, _vp]
     lib.dspark_get_near_ties.restype = _i
     lib.dspark_get_near_ties.argtypes = [_vp, _vp, ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]
     lib.dspark_clear_device_status.restype = _i
@@ -270,6 +273,11 @@ def dspark_get_near_ties(ws, stream=None):
     d, v = ctypes.c_uint32(0), ctypes.c_uint32(0)
     _call("dspark_get_near_ties", _ptr(ws), _stream(stream), ctypes.byref(d), ctypes.byref(v))
     return int(d.value), int(v.value)
+
+
+def dspark_exp2_fma(x, y, stream=None):
+    """y = 2^x (float32 device tensors of equal size) by the library's FMA-pipe polynomial."""
+    _call("dspark_exp2_fma", _ptr(x), _ptr(y), int(x.numel()), _stream(stream))
 
 
 def dspark_clear_device_status(ws, stream=None):

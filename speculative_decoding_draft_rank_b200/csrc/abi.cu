@@ -204,6 +204,12 @@ dspark_status dspark_clear_device_status(void *ws, void *stream) {
     return cuda_status(cudaMemsetAsync(&h->pad[kPadDraftTies], 0, 2 * sizeof(uint32_t), st));
 }
 
+dspark_status dspark_exp2_fma(const float *x, float *y, int n, void *stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return DSPARK_ERR_INVALID_ARG;
+    if (n == 0) return DSPARK_OK;
+    return cuda_status(launch_exp2_fma(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 dspark_status dspark_get_near_ties(const void *ws, void *stream, uint32_t *draft_out, uint32_t *verify_out) {
     if (!ws || !draft_out || !verify_out) return DSPARK_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -96,5 +96,7 @@ struct ResidualTcArgs {
 };
 cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st);
 cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st);
+// y = 2^x by the FMA-pipe polynomial of common.cuh (diagnostics).
+cudaError_t launch_exp2_fma(const float *x, float *y, int n, cudaStream_t st);
 
 }  // namespace dspark

@@ -249,7 +249,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
 
 // bf16 rows: persistent CTAs (one per SM) over the (row, 4096-column chunk)
 // work items, item q of CTA c being item c + q * grid.  Warp w of the CTA
-// takes items q = w, w + 8, ... and streams them itself: it owns two
+// takes items q = w, w + 12, ... and streams them itself: it owns two
 // shared-memory stages and keeps a bulk copy in flight into one while it
 // reduces the other (evict-first: every target row is read once, so the
 // transition factor that drafting left in L2 stays there for the residual
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
 // comes from the compacted row list, read 32 items ahead; temperatures are
 // staged in shared memory.  Lane l reads the 16-byte pieces l, l + 32, ...
 // of the chunk (bank-conflict free).
-constexpr int kVrWarps = 8;
+constexpr int kVrWarps = 12;
 constexpr int kVrThreads = kVrWarps * 32;
 constexpr int kVrStageBytes = kChunk * 2;            // 8 KB
 constexpr int kVrPieces = kVrStageBytes / 16 / 32;   // 16-byte pieces per lane (16)
@@ -404,7 +404,9 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const float2 arg = fma2(make_float2(bf16lo(wq[h]), bf16hi(wq[h])), c2, n2);
-                    s2[h] = add2(s2[h], make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
+                    // One column pair in four goes through the FMA-pipe polynomial
+                    // instead of the special-function unit, which is the busier pipe.
+                    s2[h] = add2(s2[h], h == 3 ? exp2_poly2(arg) : make_float2(fast_exp2(arg.x), fast_exp2(arg.y)));
                 }
             }
             const float2 p01 = add2(s2[0], s2[1]), p23 = add2(s2[2], s2[3]);
@@ -817,6 +819,24 @@ __global__ void __launch_bounds__(kRowThreads) residual_final(
 }
 
 // ----------------------------------------------------------------- host
+// ----------------------------------------------------------------- diagnostics
+__global__ void exp2_fma_kernel(const float *__restrict__ x, float *__restrict__ y, int n) {
+    const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
+    if (i + 1 < n) {
+        const float2 v = exp2_poly2(make_float2(x[i], x[i + 1]));
+        y[i] = v.x;
+        y[i + 1] = v.y;
+    } else if (i < n) {
+        y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+    }
+}
+
+cudaError_t launch_exp2_fma(const float *x, float *y, int n, cudaStream_t st) {
+    const int pairs = (n + 1) / 2;
+    exp2_fma_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n);
+    return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaStream_t st) {
     const T *Tl = static_cast<const T *>(a.Tlog);

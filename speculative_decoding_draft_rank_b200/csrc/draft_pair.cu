@@ -29,7 +29,10 @@
 //               y = L + Delta; Delta never leaves the SM.
 // Positions are separated by a grid barrier, the per-row finalize (inverse
 // CDF, token, U row staged for the next position) and a second grid barrier,
-// as in the single-CTA kernel of draft_tc.cu.  Every mbarrier and grid-barrier
+// as in the single-CTA kernel of draft_tc.cu.  The two producers do not wait
+// for that window: the logits and the factor do not depend on the drawn
+// tokens, so they fill the free ring slots with the next position's first
+// tiles while the rows are finalized.  Every mbarrier and grid-barrier
 // wait is bounded; a CTA that gives up raises DSPARK_DEV_TIMEOUT, lets its
 // copies in flight land, and both CTAs of the pair meet at a cluster barrier
 // before the pair's tensor memory is freed.
@@ -70,8 +73,10 @@ struct PairLayout {
     uint32_t a_off, b_off, l_off, bar_off, total;
 };
 
-// The B ring takes what is left under ~200 KB (2 to 6 stages), so a small
-// kernel can still share the SM.
+// The B ring takes what is left under ~200 KB (2 to 6 stages; deeper rings
+// under the full 227 KB measured slower).  Each of the four logit consumer
+// groups (one per 64-column segment) owns one slot: with fewer slots than
+// groups a slot would pass between groups whose parity waits can alias.
 __host__ __device__ inline PairLayout pair_layout(int r, int head) {
     PairLayout t;
     t.nkb = (r + kPKB - 1) / kPKB;
@@ -124,8 +129,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint64_t *acc_full = l_empty + SL;       // 2, each CTA: an accumulator is complete
     uint64_t *acc_empty = acc_full + 2;      // 2, even CTA: both CTAs' 32 epilogue warps drained it
     uint64_t *drain = acc_empty + 2;         // 1, even CTA
-    uint64_t *go = drain + 1;                // 1, local: position p >= 1 may start streaming
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(go + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     __shared__ int epi_flag;
@@ -147,7 +151,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
         for (int q = 0; q < SL; ++q) { tc::mbar_init(&l_full[q], 1); tc::mbar_init(&l_empty[q], 4); }
         for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], 2 * kPEpiWarps); }
         tc::mbar_init(drain, 1);
-        tc::mbar_init(go, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -172,7 +175,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
             int g = 0;
             bool ok = true;
             for (int pos = 0; pos < ep.G && ok; ++pos) {
-                if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
                 for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                     const int n0 = t * kPBN + (int)rank * kPHalf;
                     for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -248,7 +250,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
             int g = 0;
             bool ok = true;
             for (int pos = 0; pos < ep.G && ok; ++pos) {
-                if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
                 for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                     for (int sg = 0; sg < kPSegs; ++sg, ++g) {
                         const int q = g % SL;
@@ -492,7 +493,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         tc::tma_load_2d_pair(sA + (nkb + kb) * kPABytes, &mapE, a_full0, kb * kPKB, B + m0, once);
                 }
                 if (!even) tc::mbar_arrive_remote_release(a_full0);
-                tc::mbar_arrive(go);
             }
         }
     }

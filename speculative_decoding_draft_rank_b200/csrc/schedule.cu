@@ -21,6 +21,10 @@
 //      (V_n + S_(n)) t(n) < V_n t(n+1) in parallel; the first true index (or
 //      the budget) is the admitted count;
 //   3. admitted candidates are counted per request in shared memory -> ell.
+// Batches of at most 4096 candidates run as a single cluster of 16 CTAs (8
+// where the GPU refuses 16): the CTAs rank as in 1. but store each key
+// straight into the first CTA's shared memory, and one cluster barrier
+// replaces the workspace round trip, the arrival counter and its reset.
 // Variants (menfem.com KB entry, "Key Contributions"; paperlayer.ai summary,
 // Appendix A): the offline global search admits the count that maximises
 // Theta(n) = V_n / t(n) over every n up to the budget (lowest n on ties) --
@@ -38,12 +42,14 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "schedule_variants.cuh"
+#include "tc.cuh"
 
 namespace dspark {
 
 constexpr int kSchedThreads = 1024;
 constexpr int kSchedMaxN = 16384;
 constexpr int kSchedMaxP = 64;
+constexpr int kSchedClusterMaxN = 4096;   // batches ranked by one cluster of CTAs
 
 // Piecewise-linear profile through (kn[j], kt[j]) continued with the last slope.
 __device__ __forceinline__ double profile_at(const int *kn, const double *kt, int P, double n) {
@@ -57,78 +63,19 @@ __device__ __forceinline__ double profile_at(const int *kn, const double *kt, in
     return kt[lo] + (n - (double)kn[lo]) * slope;
 }
 
-__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
-    const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
-    const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
-    const int32_t *__restrict__ capacity, WsHeader *hdr, unsigned long long *__restrict__ sorted,
-    int32_t *__restrict__ ell_out, int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
-    int32_t *__restrict__ order_out)
-{
-    extern __shared__ __align__(16) unsigned char sched_smem[];
-    const int N = B * G;
-    // Shared memory: the survivals (phase 1), then the sorted keys [N] and the
-    // per-request counts [B] (the admitting CTA).
-    int *ell_s = reinterpret_cast<int *>(sched_smem + sizeof(unsigned long long) * (size_t)N);
-    __shared__ int last_s;
-    __shared__ int kn_s[kSchedMaxP];
-    __shared__ double kt_s[kSchedMaxP];
+// Admission over the sorted keys [N] in shared memory (one CTA): the fp64
+// prefix of the sorted survivals, the mode's count, the per-request lengths,
+// the order and the objective at the admitted count.  ell_s: [B] ints of
+// shared memory.
+__device__ void admit_sorted(const unsigned long long *keys, int *ell_s, int B, int G, const int *kn_s,
+                             const double *kt_s, int P, int budget, int mode, float threshold,
+                             const int32_t *__restrict__ capacity, WsHeader *hdr, int32_t *__restrict__ ell_out,
+                             int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
+                             int32_t *__restrict__ order_out) {
     __shared__ int red_i[33];
     __shared__ double red_d[33];
-
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
-    for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
-
-    if (mode == DSPARK_SCHED_ALL) {   // one CTA: no order to find
-        if (blockIdx.x != 0) return;
-        double acc = 0.0;
-        for (int j = tid; j < N; j += blockDim.x) acc += (double)S[j];
-        acc = warp_sum_d(acc);
-        if (lane == 0) red_d[wid] = acc;
-        __syncthreads();
-        if (tid == 0) {
-            double t = 0.0;
-            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red_d[w];
-            *n_adm_out = N;
-            *theta_out = ((double)B + t) / profile_at(kn_s, kt_s, P, (double)N);
-        }
-        for (int b = tid; b < B; b += blockDim.x) ell_out[b] = G;
-        if (order_out != nullptr)
-            for (int j = tid; j < N; j += blockDim.x) order_out[j] = j;
-        return;
-    }
-
-    // Phase 1: ranks by counting.  sv holds the survivals position-major
-    // (NaN or negative survivals rank last, as 0).
-    float *sv = reinterpret_cast<float *>(sched_smem);
-    for (int id = tid; id < N; id += blockDim.x) {
-        const int i = id / B, b = id - i * B;
-        float s = S[(size_t)b * G + i];
-        if (!(s >= 0.f)) s = 0.f;
-        sv[id] = s;
-    }
-    __syncthreads();
-    for (int c = (int)blockIdx.x * nwarps + wid; c < N; c += (int)gridDim.x * nwarps) {
-        const float s = sv[c];
-        int cnt = 0;
-        for (int j = lane; j < N; j += 32) {
-            const float t = sv[j];
-            cnt += (t > s) | ((t == s) & (j < c));
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) sorted[cnt] = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)c;
-    }
-    // The last CTA to finish its candidates admits.
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) last_s = atomicAdd(&hdr->pad[kPadSchedArrive], 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!last_s) return;
-    __threadfence();
-    unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [N]
-    for (int n = tid; n < N; n += blockDim.x) keys[n] = __ldcg(sorted + n);
-    __syncthreads();
-
+    const int N = B * G;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     // fp64 prefix of the sorted survivals: V_n = B + sum_{j<n} S_(j).  Thread t
     // owns the contiguous ranks [c0, c1).
     const int cpt = (N + blockDim.x - 1) / blockDim.x;
@@ -228,6 +175,131 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     }
 }
 
+__global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
+    const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
+    const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
+    const int32_t *__restrict__ capacity, WsHeader *hdr, unsigned long long *__restrict__ sorted,
+    int32_t *__restrict__ ell_out, int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out,
+    int32_t *__restrict__ order_out)
+{
+    extern __shared__ __align__(16) unsigned char sched_smem[];
+    const int N = B * G;
+    // Shared memory: the survivals (phase 1), then the sorted keys [N] and the
+    // per-request counts [B] (the admitting CTA).
+    int *ell_s = reinterpret_cast<int *>(sched_smem + sizeof(unsigned long long) * (size_t)N);
+    __shared__ int last_s;
+    __shared__ int kn_s[kSchedMaxP];
+    __shared__ double kt_s[kSchedMaxP];
+    __shared__ double red_d[33];
+
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
+
+    if (mode == DSPARK_SCHED_ALL) {   // one CTA: no order to find
+        if (blockIdx.x != 0) return;
+        double acc = 0.0;
+        for (int j = tid; j < N; j += blockDim.x) acc += (double)S[j];
+        acc = warp_sum_d(acc);
+        if (lane == 0) red_d[wid] = acc;
+        __syncthreads();
+        if (tid == 0) {
+            double t = 0.0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red_d[w];
+            *n_adm_out = N;
+            *theta_out = ((double)B + t) / profile_at(kn_s, kt_s, P, (double)N);
+        }
+        for (int b = tid; b < B; b += blockDim.x) ell_out[b] = G;
+        if (order_out != nullptr)
+            for (int j = tid; j < N; j += blockDim.x) order_out[j] = j;
+        return;
+    }
+
+    // Phase 1: ranks by counting.  sv holds the survivals position-major
+    // (NaN or negative survivals rank last, as 0).
+    float *sv = reinterpret_cast<float *>(sched_smem);
+    for (int id = tid; id < N; id += blockDim.x) {
+        const int i = id / B, b = id - i * B;
+        float s = S[(size_t)b * G + i];
+        if (!(s >= 0.f)) s = 0.f;
+        sv[id] = s;
+    }
+    __syncthreads();
+    for (int c = (int)blockIdx.x * nwarps + wid; c < N; c += (int)gridDim.x * nwarps) {
+        const float s = sv[c];
+        int cnt = 0;
+        for (int j = lane; j < N; j += 32) {
+            const float t = sv[j];
+            cnt += (t > s) | ((t == s) & (j < c));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) sorted[cnt] = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)c;
+    }
+    // The last CTA to finish its candidates admits.
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last_s = atomicAdd(&hdr->pad[kPadSchedArrive], 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!last_s) return;
+    __threadfence();
+    unsigned long long *keys = reinterpret_cast<unsigned long long *>(sched_smem);   // [N]
+    for (int n = tid; n < N; n += blockDim.x) keys[n] = __ldcg(sorted + n);
+    __syncthreads();
+
+    admit_sorted(keys, ell_s, B, G, kn_s, kt_s, P, budget, mode, threshold, capacity, hdr, ell_out, n_adm_out,
+                 theta_out, order_out);
+}
+
+// Batches of at most kSchedClusterMaxN candidates: the grid is one cluster.
+// Every CTA holds the survivals and ranks its share of the candidates by
+// counting, as above, but writes each key straight into the first CTA's
+// shared memory (distributed shared memory); after one cluster barrier the
+// first CTA admits -- no workspace round trip and no arrival counter.
+__global__ void __launch_bounds__(kSchedThreads) schedule_cluster_kernel(
+    const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
+    const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
+    const int32_t *__restrict__ capacity, WsHeader *hdr, int32_t *__restrict__ ell_out,
+    int32_t *__restrict__ n_adm_out, double *__restrict__ theta_out, int32_t *__restrict__ order_out)
+{
+    extern __shared__ __align__(16) unsigned char sched_smem[];
+    const int N = B * G;
+    // Shared memory: the survivals [N] (every CTA), then the sorted keys [N]
+    // and the per-request counts [B] (used in the first CTA).
+    float *sv = reinterpret_cast<float *>(sched_smem);
+    unsigned long long *keys =
+        reinterpret_cast<unsigned long long *>(sched_smem + ((sizeof(float) * (size_t)N + 15) & ~(size_t)15));
+    int *ell_s = reinterpret_cast<int *>(keys + N);
+    __shared__ int kn_s[kSchedMaxP];
+    __shared__ double kt_s[kSchedMaxP];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
+    for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
+    for (int id = tid; id < N; id += blockDim.x) {
+        const int i = id / B, b = id - i * B;
+        float s = S[(size_t)b * G + i];
+        if (!(s >= 0.f)) s = 0.f;
+        sv[id] = s;
+    }
+    __syncthreads();
+    const int rank = (int)tc::cluster_ctarank();
+    const uint32_t keys0 = tc::mapa_shared(tc::smem_u32(keys), 0);
+    for (int c = rank * nwarps + wid; c < N; c += (int)gridDim.x * nwarps) {
+        const float s = sv[c];
+        int cnt = 0;
+        for (int j = lane; j < N; j += 32) {
+            const float t = sv[j];
+            cnt += (t > s) | ((t == s) & (j < c));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0)
+            tc::st_cluster_u64(keys0 + 8u * (uint32_t)cnt, ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)c);
+    }
+    tc::cluster_sync();   // release / acquire: every key is in the first CTA
+    if (rank != 0) return;
+    admit_sorted(keys, ell_s, B, G, kn_s, kt_s, P, budget, mode, threshold, capacity, hdr, ell_out, n_adm_out,
+                 theta_out, order_out);
+}
+
 // Workspace: the header (status word, arrival counter) and the sorted keys.
 size_t schedule_ws_bytes(int B, int G) { return sizeof(WsHeader) + align256(sizeof(unsigned long long) * (size_t)B * G); }
 
@@ -247,6 +319,45 @@ static cudaError_t launch_sched(const float *S, int B, int G, const int32_t *kno
     if (e != cudaSuccess) return e;
     WsHeader *hdr = static_cast<WsHeader *>(ws);
     unsigned long long *sorted = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + sizeof(WsHeader));
+    if (mode != DSPARK_SCHED_ALL && B * G <= kSchedClusterMaxN) {
+        static int cluster = -1;   // CTAs of the ranking cluster (16 where the GPU allows, else 8)
+        const size_t csmem = ((sizeof(float) * (size_t)B * G + 15) & ~(size_t)15) +
+                             sizeof(unsigned long long) * (size_t)B * G + sizeof(int) * (size_t)B;
+        if ((e = cudaFuncSetAttribute(schedule_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)(((sizeof(float) * kSchedClusterMaxN + 15) & ~(size_t)15) +
+                                            sizeof(unsigned long long) * kSchedClusterMaxN +
+                                            sizeof(int) * kSchedClusterMaxN))) != cudaSuccess)
+            return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(kSchedThreads);
+        cfg.dynamicSmemBytes = csmem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cluster < 0) {
+            cluster = 8;
+            if (cudaFuncSetAttribute(schedule_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+                int n = 0;
+                attr[0].val.clusterDim.x = 16;
+                cfg.gridDim = dim3(16);
+                if (cudaOccupancyMaxActiveClusters(&n, schedule_cluster_kernel, &cfg) == cudaSuccess && n >= 1)
+                    cluster = 16;
+            }
+            cudaGetLastError();   // a refused query leaves no error behind
+        }
+        attr[0].val.clusterDim.x = cluster;
+        cfg.gridDim = dim3(cluster);
+        if ((e = cudaLaunchKernelEx(&cfg, schedule_cluster_kernel, S, B, G, knots_n, knots_t, P, budget, mode,
+                                    threshold, capacity, hdr, ell_out, n_adm_out, theta_out, order_out)) !=
+            cudaSuccess)
+            return e;
+        return cudaGetLastError();
+    }
     int grid = 1;
     if (mode != DSPARK_SCHED_ALL) {
         int dev = 0, sms = 148;

@@ -215,6 +215,10 @@ __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t bar) {
 }
 // Every thread of both CTAs (an unbounded hardware barrier: each thread
 // reaches it exactly twice, after set-up and before tear-down).
+// 64-bit store to a shared::cluster address (another CTA's shared memory).
+__device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
+}
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

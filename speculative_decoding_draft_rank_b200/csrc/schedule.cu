@@ -59,8 +59,19 @@ __device__ __forceinline__ double profile_at(const int *kn, const double *kt, in
         int mid = (lo + hi + 1) >> 1;
         if ((double)kn[mid] <= n) lo = mid; else hi = mid - 1;
     }
-    const double slope = (kt[lo + 1] - kt[lo]) / (double)(kn[lo + 1] - kn[lo]);
-    return kt[lo] + (n - (double)kn[lo]) * slope;
+    return kt[lo] + (n - (double)kn[lo]) * kt[kSchedMaxP + lo];   // the segment's slope, stored by load_profile
+}
+
+// Knots and per-segment slopes into shared memory: kt[j] = t(kn[j]) and
+// kt[kSchedMaxP + j] = (t(kn[j+1]) - t(kn[j])) / (kn[j+1] - kn[j]), so that
+// the admission scan evaluates the profile without a division.
+__device__ __forceinline__ void load_profile(const int32_t *__restrict__ knots_n, const double *__restrict__ knots_t,
+                                             int P, int *kn, double *kt) {
+    for (int j = threadIdx.x; j < P; j += blockDim.x) {
+        kn[j] = knots_n[j];
+        kt[j] = knots_t[j];
+        if (j + 1 < P) kt[kSchedMaxP + j] = (knots_t[j + 1] - knots_t[j]) / (double)(knots_n[j + 1] - knots_n[j]);
+    }
 }
 
 // Admission over the sorted keys [N] in shared memory (one CTA): the fp64
@@ -189,11 +200,11 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
     int *ell_s = reinterpret_cast<int *>(sched_smem + sizeof(unsigned long long) * (size_t)N);
     __shared__ int last_s;
     __shared__ int kn_s[kSchedMaxP];
-    __shared__ double kt_s[kSchedMaxP];
+    __shared__ double kt_s[2 * kSchedMaxP];
     __shared__ double red_d[33];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
-    for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
+    load_profile(knots_n, knots_t, P, kn_s, kt_s);
 
     if (mode == DSPARK_SCHED_ALL) {   // one CTA: no order to find
         if (blockIdx.x != 0) return;
@@ -270,9 +281,9 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_cluster_kernel(
         reinterpret_cast<unsigned long long *>(sched_smem + ((sizeof(float) * (size_t)N + 15) & ~(size_t)15));
     int *ell_s = reinterpret_cast<int *>(keys + N);
     __shared__ int kn_s[kSchedMaxP];
-    __shared__ double kt_s[kSchedMaxP];
+    __shared__ double kt_s[2 * kSchedMaxP];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
-    for (int j = tid; j < P; j += blockDim.x) { kn_s[j] = knots_n[j]; kt_s[j] = knots_t[j]; }
+    load_profile(knots_n, knots_t, P, kn_s, kt_s);
     for (int id = tid; id < N; id += blockDim.x) {
         const int i = id / B, b = id - i * B;
         float s = S[(size_t)b * G + i];

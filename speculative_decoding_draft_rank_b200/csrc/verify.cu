@@ -24,6 +24,8 @@
 //               as in drafting) fused with q = max(0, p_t - p_d) tile sums.
 //   res_final   1 CTA per queued row: prefix over tile sums, one tile
 //               recomputed and scanned to the replacement token.
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tc.cuh"
@@ -840,7 +842,7 @@ cudaError_t launch_exp2_fma(const float *x, float *y, int n, cudaStream_t st) {
 template <typename T>
 static cudaError_t launch_verify_t(const VerifyArgs &a, const VerifyWs &w, cudaStream_t st) {
     const T *Tl = static_cast<const T *>(a.Tlog);
-    verify_plan<<<1, 1024, 0, st>>>(a.ell, a.B, a.G, w);
+    verify_plan<<<1, std::min(1024, (a.B + 31) / 32 * 32), 0, st>>>(a.ell, a.B, a.G, w);   // one thread per request
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;

@@ -138,8 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
     uint64_t *acc_full = l_empty + SL;       // 2
     uint64_t *acc_empty = acc_full + 2;      // 2 (16 warps)
     uint64_t *drain = acc_empty + 2;         // 1
-    uint64_t *go = drain + 1;                // 1: drafting position p >= 1 may start streaming (phase p - 1)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(go + 1);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
 
     __shared__ int epi_flag;                 // epilogue-wide verdict of the last grid barrier
@@ -166,7 +165,6 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
         for (int q = 0; q < SL; ++q) { tc::mbar_init(&l_full[q], 1); tc::mbar_init(&l_empty[q], 4); }
         for (int q = 0; q < 2; ++q) { tc::mbar_init(&acc_full[q], 1); tc::mbar_init(&acc_empty[q], kEpiWarps); }
         tc::mbar_init(drain, 1);
-        tc::mbar_init(go, 1);
         *abort_flag = 0;
         tc::fence_barrier_init();
     }
@@ -186,10 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             const uint64_t keep = tc::policy_evict_last();
             int g = 0;
             bool ok = true;
+            // The factor does not depend on the drawn tokens: the ring runs on
+            // into the next position while the rows are finalized.
             for (int pos = 0; pos < npos && ok; ++pos) {
-            // Later positions stream only after the round's finalize, whose
-            // dependent loads would otherwise queue behind this prefetch.
-            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 const int n0 = t * kBN;
                 for (int kb = 0; kb < nkb; ++kb, ++g) {
@@ -269,8 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
             const uint64_t stream = tc::policy_evict_first();
             int g = 0;
             bool ok = true;
-            for (int pos = 0; pos < npos && ok; ++pos) {
-            if (pos > 0) ok = tc::mbar_wait_bounded(go, (pos - 1) & 1, abort_flag, ep.budget);
+            for (int pos = 0; pos < npos && ok; ++pos) {   // (the logits neither)
             for (int t = first_tile; t < nTilesN && ok; t += tile_step) {
                 for (int sg = 0; sg < kSegs; ++sg, ++g) {
                     const int q = g % SL;
@@ -529,7 +525,6 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const uint64_t once = tc::policy_evict_first();
                     for (int kb = 0; kb < nkb; ++kb)
                         tc::tma_load_2d(sA + kb * kABlockBytes, &mapE, a_full, kb * kKB, m0, once);
-                    tc::mbar_arrive(go);   // the producers may stream position pos + 1
                 }
             }
         } else {

@@ -22,9 +22,10 @@
 //      the budget) is the admitted count;
 //   3. admitted candidates are counted per request in shared memory -> ell.
 // Batches of at most 4096 candidates run as a single cluster of 16 CTAs (8
-// where the GPU refuses 16): the CTAs rank as in 1. but store each key
-// straight into the first CTA's shared memory, and one cluster barrier
-// replaces the workspace round trip, the arrival counter and its reset.
+// where the GPU refuses 16) that ranks through sorted position columns
+// (schedule_cluster_kernel below) and gathers the sorted keys in the first
+// CTA's shared memory: cluster barriers replace the workspace round trip, the
+// arrival counter and its reset.
 // Variants (menfem.com KB entry, "Key Contributions"; paperlayer.ai summary,
 // Appendix A): the offline global search admits the count that maximises
 // Theta(n) = V_n / t(n) over every n up to the budget (lowest n on ties) --
@@ -261,11 +262,21 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_kernel(
                  theta_out, order_out);
 }
 
-// Batches of at most kSchedClusterMaxN candidates: the grid is one cluster.
-// Every CTA holds the survivals and ranks its share of the candidates by
-// counting, as above, but writes each key straight into the first CTA's
-// shared memory (distributed shared memory); after one cluster barrier the
-// first CTA admits -- no workspace round trip and no arrival counter.
+// Batches of at most kSchedClusterMaxN candidates: the grid is one cluster,
+// and the rank is found in two steps instead of by comparing all pairs.  The
+// order is that of the unique 64-bit keys (~bits(S) above the candidate id),
+// so a candidate's rank is the number of smaller keys, summed over the G
+// position columns of B candidates each:
+//   1. column ranks -- each CTA takes a share of the candidates and counts,
+//      within the candidate's own column, the smaller keys (B comparisons,
+//      one warp per candidate); the key is stored at that place of the
+//      sorted column in every CTA of the cluster (distributed shared memory);
+//   2. after a cluster barrier, global ranks -- for its candidates each CTA
+//      adds the G lower bounds of the key in the sorted columns (one lane per
+//      column, a binary search each) and stores the key at that rank in the
+//      first CTA; after a second barrier the first CTA admits.
+// That is N (B + G log B) comparisons where counting over all pairs takes N^2,
+// with no workspace round trip and no arrival counter.
 __global__ void __launch_bounds__(kSchedThreads) schedule_cluster_kernel(
     const float *__restrict__ S, int B, int G, const int32_t *__restrict__ knots_n,
     const double *__restrict__ knots_t, int P, int budget, int mode, float threshold,
@@ -274,38 +285,60 @@ __global__ void __launch_bounds__(kSchedThreads) schedule_cluster_kernel(
 {
     extern __shared__ __align__(16) unsigned char sched_smem[];
     const int N = B * G;
-    // Shared memory: the survivals [N] (every CTA), then the sorted keys [N]
-    // and the per-request counts [B] (used in the first CTA).
-    float *sv = reinterpret_cast<float *>(sched_smem);
-    unsigned long long *keys =
-        reinterpret_cast<unsigned long long *>(sched_smem + ((sizeof(float) * (size_t)N + 15) & ~(size_t)15));
+    // Shared memory: every candidate's key [N] (position-major), the sorted
+    // columns [G][B], then (used in the first CTA) the sorted keys [N] and the
+    // per-request counts [B].
+    unsigned long long *kall = reinterpret_cast<unsigned long long *>(sched_smem);
+    unsigned long long *col = kall + N;
+    unsigned long long *keys = col + N;
     int *ell_s = reinterpret_cast<int *>(keys + N);
     __shared__ int kn_s[kSchedMaxP];
     __shared__ double kt_s[2 * kSchedMaxP];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
+    tc::cluster_arrive_relaxed();   // this CTA runs; waited for before the first remote store
     load_profile(knots_n, knots_t, P, kn_s, kt_s);
     for (int id = tid; id < N; id += blockDim.x) {
         const int i = id / B, b = id - i * B;
         float s = S[(size_t)b * G + i];
-        if (!(s >= 0.f)) s = 0.f;
-        sv[id] = s;
+        if (!(s >= 0.f)) s = 0.f;   // NaN or negative survivals rank last, as 0
+        kall[id] = ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)id;
     }
     __syncthreads();
-    const int rank = (int)tc::cluster_ctarank();
-    const uint32_t keys0 = tc::mapa_shared(tc::smem_u32(keys), 0);
-    for (int c = rank * nwarps + wid; c < N; c += (int)gridDim.x * nwarps) {
-        const float s = sv[c];
+    tc::cluster_wait();             // every CTA of the cluster has started
+    const int rank = (int)tc::cluster_ctarank(), ncta = (int)gridDim.x;
+    const int step = ncta * nwarps;
+    // 1. Column ranks, broadcast into every CTA's sorted columns.
+    const uint32_t col_u32 = tc::smem_u32(col);
+    for (int c = rank * nwarps + wid; c < N; c += step) {
+        const unsigned long long k = kall[c];
+        const int i = c / B;
+        const unsigned long long *cc = kall + (size_t)i * B;
         int cnt = 0;
-        for (int j = lane; j < N; j += 32) {
-            const float t = sv[j];
-            cnt += (t > s) | ((t == s) & (j < c));
-        }
+        for (int j = lane; j < B; j += 32) cnt += cc[j] < k;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0)
-            tc::st_cluster_u64(keys0 + 8u * (uint32_t)cnt, ((unsigned long long)(~__float_as_uint(s)) << 32) | (unsigned)c);
+        if (lane < ncta) tc::st_cluster_u64(tc::mapa_shared(col_u32 + 8u * (uint32_t)(i * B + cnt), lane), k);
     }
-    tc::cluster_sync();   // release / acquire: every key is in the first CTA
+    tc::cluster_sync();   // every CTA holds all G sorted columns
+    // 2. Global ranks: lane i < G counts the keys below k in sorted column i.
+    const uint32_t keys0 = tc::mapa_shared(tc::smem_u32(keys), 0);
+    for (int c = rank * nwarps + wid; c < N; c += step) {
+        const unsigned long long k = kall[c];
+        int below = 0;
+        if (lane < G) {
+            const unsigned long long *cc = col + (size_t)lane * B;
+            int lo = 0, hi = B;   // first index with cc[idx] >= k
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (cc[mid] < k) lo = mid + 1; else hi = mid;
+            }
+            below = lo;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+        if (lane == 0) tc::st_cluster_u64(keys0 + 8u * (uint32_t)below, k);
+    }
+    tc::cluster_sync();   // every key is in the first CTA, in order
     if (rank != 0) return;
     admit_sorted(keys, ell_s, B, G, kn_s, kt_s, P, budget, mode, threshold, capacity, hdr, ell_out, n_adm_out,
                  theta_out, order_out);
@@ -332,11 +365,10 @@ static cudaError_t launch_sched(const float *S, int B, int G, const int32_t *kno
     unsigned long long *sorted = reinterpret_cast<unsigned long long *>(static_cast<char *>(ws) + sizeof(WsHeader));
     if (mode != DSPARK_SCHED_ALL && B * G <= kSchedClusterMaxN) {
         static int cluster = -1;   // CTAs of the ranking cluster (16 where the GPU allows, else 8)
-        const size_t csmem = ((sizeof(float) * (size_t)B * G + 15) & ~(size_t)15) +
-                             sizeof(unsigned long long) * (size_t)B * G + sizeof(int) * (size_t)B;
+        // keys, sorted columns and sorted keys [3 N] u64, the counts [B] int
+        const size_t csmem = 3 * sizeof(unsigned long long) * (size_t)B * G + sizeof(int) * (size_t)B;
         if ((e = cudaFuncSetAttribute(schedule_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      (int)(((sizeof(float) * kSchedClusterMaxN + 15) & ~(size_t)15) +
-                                            sizeof(unsigned long long) * kSchedClusterMaxN +
+                                      (int)(3 * sizeof(unsigned long long) * kSchedClusterMaxN +
                                             sizeof(int) * kSchedClusterMaxN))) != cudaSuccess)
             return e;
         cudaLaunchConfig_t cfg = {};

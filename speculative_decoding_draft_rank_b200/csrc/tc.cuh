@@ -219,6 +219,11 @@ __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t bar) {
 __device__ __forceinline__ void st_cluster_u64(uint32_t addr, unsigned long long v) {
     asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(addr), "l"(v) : "memory");
 }
+// Split cluster barrier: arrive (relaxed) early, wait (acquire) later.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

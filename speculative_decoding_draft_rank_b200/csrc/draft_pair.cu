@@ -471,9 +471,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const int p = t * kPSegs + sg;
                 if (rowok && p < nParts) {
                     const size_t o = (size_t)b * nParts + p;
-                    ep.part_m[o] = m;
-                    ep.part_s[o] = s;
-                    ep.part_a[o] = am;
+                    ep.part_m[o] = m;   // the finalize reads Z's terms for sampled rows, the argmax for greedy ones
+                    if (invT > 0.f) ep.part_s[o] = s;
+                    else ep.part_a[o] = am;
                 }
             }
             if (!grid_sync(nblk * (2u * pos + 1u))) break;

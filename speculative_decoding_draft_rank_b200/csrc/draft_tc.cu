@@ -507,9 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const int p = t * kSegs + sg;
                     if (rowok && p < nParts) {
                         const size_t o = (size_t)b * nParts + p;
-                        ep.part_m[o] = m;
-                        ep.part_s[o] = s;
-                        ep.part_a[o] = am;
+                        ep.part_m[o] = m;   // the finalize reads Z's terms for sampled rows, the argmax for greedy ones
+                        if (invT > 0.f) ep.part_s[o] = s;
+                        else ep.part_a[o] = am;
                     }
                 }
                 // Every CTA's partials of this position are written.

@@ -133,21 +133,24 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
 
     // Every load that depends on nothing else goes out first (the partials
-    // as 16-byte pieces when the thread's eight are whole and aligned).
+    // as 16-byte pieces when the thread's eight are whole and aligned).  The
+    // partials are rewritten at every position by other CTAs of the same
+    // launch, so they are read past L1 (ld.global.cg), never through the
+    // read-only path.
     float cm[kFinChunk], cs[kFinChunk];
     if (t0 + kFinChunk <= t1 && ((reinterpret_cast<uintptr_t>(pm + t0) | reinterpret_cast<uintptr_t>(ps + t0)) & 15) == 0) {
-        const float4 m0 = __ldg(reinterpret_cast<const float4 *>(pm + t0));
-        const float4 m1 = __ldg(reinterpret_cast<const float4 *>(pm + t0 + 4));
-        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(ps + t0));
-        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(ps + t0 + 4));
+        const float4 m0 = __ldcg(reinterpret_cast<const float4 *>(pm + t0));
+        const float4 m1 = __ldcg(reinterpret_cast<const float4 *>(pm + t0 + 4));
+        const float4 s0 = __ldcg(reinterpret_cast<const float4 *>(ps + t0));
+        const float4 s1 = __ldcg(reinterpret_cast<const float4 *>(ps + t0 + 4));
         cm[0] = m0.x; cm[1] = m0.y; cm[2] = m0.z; cm[3] = m0.w; cm[4] = m1.x; cm[5] = m1.y; cm[6] = m1.z; cm[7] = m1.w;
         cs[0] = s0.x; cs[1] = s0.y; cs[2] = s0.z; cs[3] = s0.w; cs[4] = s1.x; cs[5] = s1.y; cs[6] = s1.z; cs[7] = s1.w;
     } else {
 #pragma unroll
         for (int q = 0; q < kFinChunk; ++q) {
             const bool in = t0 + q < t1;
-            cm[q] = in ? pm[t0 + q] : -INFINITY;
-            cs[q] = in ? ps[t0 + q] : 0.f;
+            cm[q] = in ? __ldcg(pm + t0 + q) : -INFINITY;
+            cs[q] = in ? __ldcg(ps + t0 + q) : 0.f;
         }
     }
     const float Tb = sane_temp(a.temp[b], a.hdr);
@@ -173,20 +176,20 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     float m = -INFINITY;
 #pragma unroll
     for (int q = 0; q < kFinChunk; ++q) m = fmaxf(m, cm[q]);
-    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, pm[t]);   // very large vocabularies only
+    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, __ldcg(pm + t));   // very large vocabularies only
     const float M = grp_max1(g, m, sc->s_max);
 
     if (Tb == 0.f) {   // greedy row (group-uniform): lowest argmax over the partials
         int first = 0x7fffffff;
         for (int t = t1 - 1; t >= t0 + kFinChunk; --t)
-            if (pm[t] == M) first = t;
+            if (__ldcg(pm + t) == M) first = t;
 #pragma unroll
         for (int q = kFinChunk - 1; q >= 0; --q)
             if (t0 + q < t1 && cm[q] == M) first = t0 + q;
         first = grp_min1(g, first, sc->s_own);
         if (tid == 0) {
             if (first >= nTiles) first = 0;  // no partial matched (non-finite inputs)
-            int x = a.part_a[(size_t)b * nTiles + first];
+            int x = __ldcg(a.part_a + (size_t)b * nTiles + first);
             if (x < 0 || x >= V) x = 0;
             a.x_out[ro] = x;
             a.pd_out[ro] = 1.f;
@@ -204,7 +207,7 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     float loc = 0.f;
 #pragma unroll
     for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
-    for (int t = t0 + kFinChunk; t < t1; ++t) loc += ps[t] * fast_exp2((pm[t] - M) * cexp);
+    for (int t = t0 + kFinChunk; t < t1; ++t) loc += __ldcg(ps + t) * fast_exp2((__ldcg(pm + t) - M) * cexp);
     float Z;
     const float incl = grp_scan1(g, loc, sc->s_loc, &Z);
     const float target = u * Z;
@@ -229,7 +232,7 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
             }
         }
         for (int t = t0 + kFinChunk; t < t1 && ts < 0; ++t) {
-            const float wt = ps[t] * fast_exp2((pm[t] - M) * cexp);
+            const float wt = __ldcg(ps + t) * fast_exp2((__ldcg(pm + t) - M) * cexp);
             if (run + wt > target) {
                 ts = t;
             } else {

@@ -33,14 +33,14 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
     const T *__restrict__ L, const T *__restrict__ U, const T *__restrict__ Wt,
     const int32_t *__restrict__ x0, const int32_t *__restrict__ xprev_base,
     const float *__restrict__ temp, int B, int G, int V, int r, int pos, int nTiles,
-    float *__restrict__ part_m, float *__restrict__ part_s, int32_t *__restrict__ part_a,
-    WsHeader *hdr)
+    float2 *__restrict__ part, WsHeader *hdr)
 {
     __shared__ float Es[kSimtRows][33];
     __shared__ int prev_s[kSimtRows];
     __shared__ float red_v[8][kSimtRows];
     __shared__ int red_i[8][kSimtRows];
     __shared__ float row_m[kSimtRows];
+    __shared__ int row_a[kSimtRows];
     __shared__ float row_invT[kSimtRows];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
@@ -113,11 +113,7 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
             if (ov > v || (ov == v && oi < ix)) { v = ov; ix = oi; }
         }
         row_m[tid] = v;
-        int b = row0 + tid;
-        if (b < B) {
-            part_m[(size_t)b * nTiles + tile] = v;
-            part_a[(size_t)b * nTiles + tile] = ix;
-        }
+        row_a[tid] = ix;
     }
     __syncthreads();
     // Phase 2: sum of exp(((L - m) + Delta) / T) over the tile.
@@ -133,7 +129,8 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
     if (tid < kSimtRows && row0 + tid < B) {
         float s = 0.f;
         for (int w = 0; w < 8; ++w) s += red_v[w][tid];
-        part_s[(size_t)(row0 + tid) * nTiles + tile] = s;
+        part[(size_t)(row0 + tid) * nTiles + tile] =
+            make_float2(row_m[tid], row_invT[tid] > 0.f ? s : __int_as_float(row_a[tid]));
     }
 }
 
@@ -159,9 +156,7 @@ int draft_tile_cols(int dtype) { return dtype == DSPARK_BF16 ? kTcTileN : kSimtC
 size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
     size_t nt = draft_tiles(V, dtype);
     size_t bytes = sizeof(WsHeader);
-    bytes += align256(sizeof(float) * (size_t)B * nt);    // part_m
-    bytes += align256(sizeof(float) * (size_t)B * nt);    // part_s
-    bytes += align256(sizeof(int32_t) * (size_t)B * nt);  // part_a
+    bytes += align256(sizeof(float2) * (size_t)B * nt);   // part
     if (dtype == DSPARK_BF16) bytes += align256((size_t)2 * B * r * 2);   // E (the RNN head stages two parts)
     return bytes;
 }
@@ -172,9 +167,7 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     char *p = static_cast<char *>(ws);
     w.hdr = reinterpret_cast<WsHeader *>(p);
     p += sizeof(WsHeader);
-    w.part_m = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
-    w.part_s = reinterpret_cast<float *>(p); p += align256(sizeof(float) * (size_t)B * nt);
-    w.part_a = reinterpret_cast<int32_t *>(p); p += align256(sizeof(int32_t) * (size_t)B * nt);
+    w.part = reinterpret_cast<float2 *>(p); p += align256(sizeof(float2) * (size_t)B * nt);
     w.E = nullptr;
     if (dtype == DSPARK_BF16) { w.E = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)2 * B * r * 2); }
     w.nTiles = (int)nt;
@@ -185,7 +178,7 @@ FinArgs fin_args(const DraftArgs &a, const DraftWs &w) {
     FinArgs f{};
     f.L = a.L; f.U = a.U; f.Wt = a.Wt; f.x0 = a.x0; f.temp = a.temp; f.u_draft = a.u_draft;
     f.B = a.B; f.G = a.G; f.V = a.V; f.r = a.r; f.nTiles = w.nTiles; f.TN = draft_tile_cols(a.dtype);
-    f.part_m = w.part_m; f.part_s = w.part_s; f.part_a = w.part_a;
+    f.part = w.part;
     f.x_out = a.x_out; f.pd_out = a.pd_out; f.rowmax_out = a.rowmax_out; f.rowsum_out = a.rowsum_out;
     f.E = w.E; f.hdr = w.hdr;
     f.Arec = static_cast<const __nv_bfloat16 *>(a.Arec);
@@ -204,7 +197,7 @@ cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
         dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);
         draft_tile_simt<float><<<grid, 256, 0, st>>>(
             static_cast<const float *>(a.L), static_cast<const float *>(a.U), static_cast<const float *>(a.Wt),
-            a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos, w.nTiles, w.part_m, w.part_s, w.part_a, w.hdr);
+            a.x0, a.x_out, a.temp, a.B, a.G, a.V, a.r, pos, w.nTiles, w.part, w.hdr);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         draft_finalize<float><<<a.B, kFinThreads, 0, st>>>(f, pos);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -102,8 +102,7 @@ struct PairEpi {
     uint32_t *grid_count;
     const __nv_bfloat16 *U;
     const int32_t *x0;
-    float *part_m, *part_s;
-    int32_t *part_a;
+    float2 *part;
 };
 
 template <int HEAD>
@@ -471,9 +470,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 const int p = t * kPSegs + sg;
                 if (rowok && p < nParts) {
                     const size_t o = (size_t)b * nParts + p;
-                    ep.part_m[o] = m;   // the finalize reads Z's terms for sampled rows, the argmax for greedy ones
-                    if (invT > 0.f) ep.part_s[o] = s;
-                    else ep.part_a[o] = am;
+                    // One 8-byte record: the finalize reads Z's terms for a sampled row,
+                    // the argmax for a greedy one.
+                    ep.part[o] = make_float2(m, invT > 0.f ? s : __int_as_float(am));
                 }
             }
             if (!grid_sync(nblk * (2u * pos + 1u))) break;
@@ -565,7 +564,7 @@ cudaError_t launch_pair(const DraftArgs &a, const DraftWs &w, const FinArgs &f, 
     ep.grid_count = &w.hdr->pad[2];
     ep.U = static_cast<const __nv_bfloat16 *>(a.U);
     ep.x0 = a.x0;
-    ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
+    ep.part = w.part;
     const int nMB = (a.B + kPM - 1) / kPM;
     ep.nPB = (nMB + 1) / 2;
     CUtensorMap mW, mL, mE;

@@ -103,8 +103,7 @@ struct TcEpi {
     const float *H;           // residual, RNN head: the states [B, G, r] (A rows split high/low); else null
     const __nv_bfloat16 *L;   // drafting and residual: backbone logits [B, G, V]
     // drafting: 64-column partials per request row
-    float *part_m, *part_s;
-    int32_t *part_a;
+    float2 *part;
     // residual: rows are the queued rejections; per 64 columns the sum of
     // max(0, p_t - p_d) with p_d rebuilt from L + Delta and the drafting stats
     const uint32_t *nrows;
@@ -507,9 +506,9 @@ __global__ void __launch_bounds__(kThreads, 1) markov_tile_tc(const __grid_const
                     const int p = t * kSegs + sg;
                     if (rowok && p < nParts) {
                         const size_t o = (size_t)b * nParts + p;
-                        ep.part_m[o] = m;   // the finalize reads Z's terms for sampled rows, the argmax for greedy ones
-                        if (invT > 0.f) ep.part_s[o] = s;
-                        else ep.part_a[o] = am;
+                        // One 8-byte record: the finalize reads Z's terms for a sampled row,
+                        // the argmax for a greedy one.
+                        ep.part[o] = make_float2(m, invT > 0.f ? s : __int_as_float(am));
                     }
                 }
                 // Every CTA's partials of this position are written.
@@ -730,7 +729,7 @@ cudaError_t launch_draft_tc(const DraftArgs &a, const DraftWs &w, const FinArgs 
     ep.budget = wait_budget(kWaitBudget);
     ep.U = static_cast<const __nv_bfloat16 *>(a.U); ep.x0 = a.x0; ep.x = a.x_out;
     ep.L = static_cast<const __nv_bfloat16 *>(a.L);
-    ep.part_m = w.part_m; ep.part_s = w.part_s; ep.part_a = w.part_a;
+    ep.part = w.part;
     ep.fin = f;
     ep.grid_count = &w.hdr->pad[2];
     return launch_markov_tc<kEpiDraft>(a.Wt, a.r, ep, w.E, st);

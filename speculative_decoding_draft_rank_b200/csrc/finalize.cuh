@@ -74,8 +74,7 @@ struct FinArgs {
     const int32_t *x0;
     const float *temp, *u_draft;
     int B, G, V, r, nTiles, TN;   // TN: columns per partial
-    const float *part_m, *part_s;
-    const int32_t *part_a;
+    const float2 *part;            // [B, nTiles] (max, sum of exps or argmax bits)
     int32_t *x_out;
     float *pd_out, *rowmax_out, *rowsum_out;
     __nv_bfloat16 *E;              // bf16 rounds: the next position's A rows staged for TMA, else null
@@ -127,8 +126,7 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
             a.E[((size_t)B + b) * r + c] = __float2bfloat16_rn(hn - __bfloat162float(hi));
         }
     };
-    const float *pm = a.part_m + (size_t)b * nTiles;
-    const float *ps = a.part_s + (size_t)b * nTiles;
+    const float2 *pp = a.part + (size_t)b * nTiles;
     const int K = (nTiles + nthr - 1) / nthr;
     const int t0 = min(nTiles, tid * K), t1 = min(nTiles, t0 + K);
 
@@ -137,20 +135,20 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     // partials are rewritten at every position by other CTAs of the same
     // launch, so they are read past L1 (ld.global.cg), never through the
     // read-only path.
-    float cm[kFinChunk], cs[kFinChunk];
-    if (t0 + kFinChunk <= t1 && ((reinterpret_cast<uintptr_t>(pm + t0) | reinterpret_cast<uintptr_t>(ps + t0)) & 15) == 0) {
-        const float4 m0 = __ldcg(reinterpret_cast<const float4 *>(pm + t0));
-        const float4 m1 = __ldcg(reinterpret_cast<const float4 *>(pm + t0 + 4));
-        const float4 s0 = __ldcg(reinterpret_cast<const float4 *>(ps + t0));
-        const float4 s1 = __ldcg(reinterpret_cast<const float4 *>(ps + t0 + 4));
-        cm[0] = m0.x; cm[1] = m0.y; cm[2] = m0.z; cm[3] = m0.w; cm[4] = m1.x; cm[5] = m1.y; cm[6] = m1.z; cm[7] = m1.w;
-        cs[0] = s0.x; cs[1] = s0.y; cs[2] = s0.z; cs[3] = s0.w; cs[4] = s1.x; cs[5] = s1.y; cs[6] = s1.z; cs[7] = s1.w;
+    float cm[kFinChunk], cs[kFinChunk];   // cs: sums of exps (sampled rows) or argmax bits (greedy rows)
+    if (t0 + kFinChunk <= t1 && (reinterpret_cast<uintptr_t>(pp + t0) & 15) == 0) {
+#pragma unroll
+        for (int q = 0; q < kFinChunk / 2; ++q) {
+            const float4 v = __ldcg(reinterpret_cast<const float4 *>(pp + t0 + 2 * q));
+            cm[2 * q] = v.x; cs[2 * q] = v.y; cm[2 * q + 1] = v.z; cs[2 * q + 1] = v.w;
+        }
     } else {
 #pragma unroll
         for (int q = 0; q < kFinChunk; ++q) {
             const bool in = t0 + q < t1;
-            cm[q] = in ? __ldcg(pm + t0 + q) : -INFINITY;
-            cs[q] = in ? __ldcg(ps + t0 + q) : 0.f;
+            const float2 v = in ? __ldcg(pp + t0 + q) : make_float2(-INFINITY, 0.f);
+            cm[q] = v.x;
+            cs[q] = v.y;
         }
     }
     const float Tb = sane_temp(a.temp[b], a.hdr);
@@ -176,20 +174,20 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     float m = -INFINITY;
 #pragma unroll
     for (int q = 0; q < kFinChunk; ++q) m = fmaxf(m, cm[q]);
-    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, __ldcg(pm + t));   // very large vocabularies only
+    for (int t = t0 + kFinChunk; t < t1; ++t) m = fmaxf(m, __ldcg(pp + t).x);   // very large vocabularies only
     const float M = grp_max1(g, m, sc->s_max);
 
     if (Tb == 0.f) {   // greedy row (group-uniform): lowest argmax over the partials
         int first = 0x7fffffff;
         for (int t = t1 - 1; t >= t0 + kFinChunk; --t)
-            if (__ldcg(pm + t) == M) first = t;
+            if (__ldcg(pp + t).x == M) first = t;
 #pragma unroll
         for (int q = kFinChunk - 1; q >= 0; --q)
             if (t0 + q < t1 && cm[q] == M) first = t0 + q;
         first = grp_min1(g, first, sc->s_own);
         if (tid == 0) {
             if (first >= nTiles) first = 0;  // no partial matched (non-finite inputs)
-            int x = __ldcg(a.part_a + (size_t)b * nTiles + first);
+            int x = __float_as_int(__ldcg(pp + first).y);
             if (x < 0 || x >= V) x = 0;
             a.x_out[ro] = x;
             a.pd_out[ro] = 1.f;
@@ -207,7 +205,10 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
     float loc = 0.f;
 #pragma unroll
     for (int q = 0; q < kFinChunk; ++q) loc += cs[q] * fast_exp2((cm[q] - M) * cexp);
-    for (int t = t0 + kFinChunk; t < t1; ++t) loc += __ldcg(ps + t) * fast_exp2((__ldcg(pm + t) - M) * cexp);
+    for (int t = t0 + kFinChunk; t < t1; ++t) {
+        const float2 v = __ldcg(pp + t);
+        loc += v.y * fast_exp2((v.x - M) * cexp);
+    }
     float Z;
     const float incl = grp_scan1(g, loc, sc->s_loc, &Z);
     const float target = u * Z;
@@ -232,7 +233,8 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
             }
         }
         for (int t = t0 + kFinChunk; t < t1 && ts < 0; ++t) {
-            const float wt = __ldcg(ps + t) * fast_exp2((__ldcg(pm + t) - M) * cexp);
+            const float2 v = __ldcg(pp + t);
+            const float wt = v.y * fast_exp2((v.x - M) * cexp);
             if (run + wt > target) {
                 ts = t;
             } else {

@@ -39,8 +39,10 @@ struct DraftArgs {
 
 struct DraftWs {
     WsHeader *hdr;
-    float *part_m, *part_s;
-    int32_t *part_a;
+    // Per (row, 64-column segment) partial of the drafting softmax: x = the
+    // segment's max, y = its sum of exp((y - max) / T) for a sampled row, or
+    // the bits of its lowest argmax (int) for a greedy row.
+    float2 *part;
     __nv_bfloat16 *E;   // bf16 only: [B, r] rows U[x_i] staged for the next position's MMA
     int nTiles;
 };

@@ -277,7 +277,7 @@ dspark_status dspark_verify_rnn(const void *Tlog, const void *L, const float *H,
  * this library holds until the process exits.  Rounds whose drafting
  * workspace (dspark_draft_workspace_size) would exceed that size are rejected
  * with DSPARK_ERR_WORKSPACE before any work is enqueued; the headline shape
- * B = 256, G = 5, V = 129280, r = 256 needs 4,399,360 bytes.  No call
+ * B = 256, G = 5, V = 129280, r = 256 needs 4,530,432 bytes.  No call
  * allocates: no cudaMalloc, cudaFree or allocating library routine.
  *
  * The first call on each device looks up the array's device address (with

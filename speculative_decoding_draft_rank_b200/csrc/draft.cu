@@ -134,6 +134,22 @@ __global__ void __launch_bounds__(256) draft_tile_simt(
     }
 }
 
+// out[c][q] = in[q][c] for an n x n bf16 matrix (32 x 32 tiles through shared
+// memory, 32 x 8 threads).
+__global__ void transpose_bf16(const __nv_bfloat16 *__restrict__ in, __nv_bfloat16 *__restrict__ out, int n) {
+    __shared__ __nv_bfloat16 tile[32][33];
+    const int x0 = blockIdx.x * 32, y0 = blockIdx.y * 32;
+    for (int j = threadIdx.y; j < 32; j += 8) {
+        const int y = y0 + j, x = x0 + threadIdx.x;
+        if (y < n && x < n) tile[j][threadIdx.x] = in[(size_t)y * n + x];
+    }
+    __syncthreads();
+    for (int j = threadIdx.y; j < 32; j += 8) {
+        const int y = x0 + j, x = y0 + threadIdx.x;   // out row = in column
+        if (y < n && x < n) out[(size_t)y * n + x] = tile[threadIdx.x][j];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Finalize (fp32 rounds): one CTA of kFinThreads threads per request row, the
 // row work in finalize.cuh.
@@ -158,6 +174,7 @@ size_t draft_ws_bytes(int B, int G, int V, int r, int dtype) {
     size_t bytes = sizeof(WsHeader);
     bytes += align256(sizeof(float2) * (size_t)B * nt);   // part
     if (dtype == DSPARK_BF16) bytes += align256((size_t)2 * B * r * 2);   // E (the RNN head stages two parts)
+    if (dtype == DSPARK_BF16) bytes += align256((size_t)r * r * 2);       // the RNN head's transposed A
     return bytes;
 }
 
@@ -169,7 +186,9 @@ DraftWs carve_draft_ws(void *ws, int B, int V, int r, int dtype) {
     p += sizeof(WsHeader);
     w.part = reinterpret_cast<float2 *>(p); p += align256(sizeof(float2) * (size_t)B * nt);
     w.E = nullptr;
+    w.AT = nullptr;
     if (dtype == DSPARK_BF16) { w.E = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)2 * B * r * 2); }
+    if (dtype == DSPARK_BF16) { w.AT = reinterpret_cast<__nv_bfloat16 *>(p); p += align256((size_t)r * r * 2); }
     w.nTiles = (int)nt;
     return w;
 }
@@ -182,6 +201,7 @@ FinArgs fin_args(const DraftArgs &a, const DraftWs &w) {
     f.x_out = a.x_out; f.pd_out = a.pd_out; f.rowmax_out = a.rowmax_out; f.rowsum_out = a.rowsum_out;
     f.E = w.E; f.hdr = w.hdr;
     f.Arec = static_cast<const __nv_bfloat16 *>(a.Arec);
+    f.ArecT = w.AT;
     f.H = a.H_out;
     return f;
 }
@@ -189,9 +209,17 @@ FinArgs fin_args(const DraftArgs &a, const DraftWs &w) {
 cudaError_t launch_draft(const DraftArgs &a, void *ws, cudaStream_t st) {
     DraftWs w = carve_draft_ws(ws, a.B, a.V, a.r, a.dtype);
     const FinArgs f = fin_args(a, w);
-    // bf16: more than 128 requests (and every RNN-head round) on CTA pairs.
-    if (a.dtype == DSPARK_BF16)
+    // bf16: more than 128 requests (and every RNN-head round) on CTA pairs;
+    // the RNN head's recurrent matrix is transposed into the workspace first.
+    if (a.dtype == DSPARK_BF16) {
+        if (a.H_out != nullptr) {
+            dim3 grid((a.r + 31) / 32, (a.r + 31) / 32);
+            transpose_bf16<<<grid, dim3(32, 8), 0, st>>>(static_cast<const __nv_bfloat16 *>(a.Arec), w.AT, a.r);
+            cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
         return (a.B > 128 || a.H_out != nullptr) ? launch_draft_pair(a, w, f, st) : launch_draft_tc(a, w, f, st);
+    }
     cudaError_t e;
     for (int pos = 0; pos < a.G; ++pos) {
         dim3 grid(w.nTiles, (a.B + kSimtRows - 1) / kSimtRows);

@@ -83,6 +83,7 @@ struct FinArgs {
     // biases position i); E then holds the next state split into bf16 high
     // parts (rows 0..B-1) and low parts (rows B..2B-1).
     const __nv_bfloat16 *Arec;
+    const __nv_bfloat16 *ArecT;    // its transpose [r, r] (row c = column c), staged per launch
     float *H;
     WsHeader *hdr;
 };
@@ -115,9 +116,10 @@ __device__ void finalize_row(const Grp &g, FinScratch *sc, float *urow, const Fi
             return;
         }
         for (int c = tid; c < r; c += nthr) {
-            float acc = 0.f;
-#pragma unroll 8
-            for (int q = 0; q < r; ++q) acc = fmaf(urow[q], __bfloat162float(a.Arec[(size_t)q * r + c]), acc);
+            // (h A)[c] as the dot product of h with column c of A, a row of
+            // the transposed copy: 16-byte loads, eight in flight, summed in
+            // index order.
+            float acc = dot_part(urow, a.ArecT + (size_t)c * r, r, 0, 1);
             acc += ld_elem(U, (size_t)x * r + c);
             const float hn = tanhf(acc);
             a.H[(ro + 1) * r + c] = hn;

@@ -43,7 +43,8 @@ struct DraftWs {
     // segment's max, y = its sum of exp((y - max) / T) for a sampled row, or
     // the bits of its lowest argmax (int) for a greedy row.
     float2 *part;
-    __nv_bfloat16 *E;   // bf16 only: [B, r] rows U[x_i] staged for the next position's MMA
+    __nv_bfloat16 *E;
+    __nv_bfloat16 *AT;   // bf16 only: the RNN head's recurrent matrix transposed [r, r] (row c = column c of A)   // bf16 only: [B, r] rows U[x_i] staged for the next position's MMA
     int nTiles;
 };
 

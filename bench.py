@@ -741,23 +741,23 @@ def main():
         ell_tot, nout_tot = float(ell_sum), float(nout_sum)
     value = ell_tot / (ms * 1e-3)
 
-    # End to end through the public API: per-round inputs from pinned host
-    # memory, the round, and the emitted tokens back to pinned host memory.
+    # End to end through the public API (DeviceRound.run_from_host): the
+    # round's draft-side inputs from pinned host memory, drafting, confidence
+    # and scheduling, the target rows verification reads (rows 0..ell_b per
+    # request, pulled from pinned host memory by one kernel that reads ell on
+    # the device), verification, and the emitted tokens, counts and lengths
+    # back to pinned host memory.
     e2e_ms = []
-    per_round_inputs = ("L", "Tlog", "h", "x0", "temp", "u_draft", "u_accept", "u_final")
-    h2d = sum(dr.host[k].numel() * dr.host[k].element_size() for k in per_round_inputs)
-    d2h = dr.d2h_bytes()
+    h2d = d2h = 0
     with torch.cuda.stream(stream):
         for i in range(max(2, args.steps // 2) + 1):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for k in per_round_inputs:
-                dr.t[k].copy_(dr.host[k], non_blocking=True)
-            dr.run(stream)
-            dr.download(stream)
+            dr.run_from_host(stream)
             e1.record(stream)
             stream.synchronize()
+            h2d, d2h = dr.host_round_bytes()
             if i > 0:
                 e2e_ms.append(e0.elapsed_time(e1))
     e2e = statistics.mean(e2e_ms)

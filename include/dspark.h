@@ -263,6 +263,34 @@ dspark_status dspark_verify_rnn(const void *Tlog, const void *L, const float *H,
                                 void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Target rows from host memory.  [PL] §2: the target model checks the drafted
+ * tokens in one forward pass; [KB] Key Contributions: the scheduler prunes
+ * low-confidence tokens from verification.  The target forward therefore
+ * yields rows only for the admitted positions: of Tlog [B,G+1,V] a round
+ * needs rows 0..ell_b of request b (ell_b verified positions, then the row of
+ * the bonus or residual draw), and dspark_verify / dspark_verify_rnn read no
+ * other row.  This call enqueues one kernel that copies exactly those rows
+ * from page-locked host memory into the device buffer of the same layout,
+ * reading ell on the device (e.g. dspark_schedule's ell_out, earlier on the
+ * same stream), so a round fed from the host needs no host round trip
+ * between scheduling and verification and stays graph-capturable.  The other
+ * rows of the device buffer are left as they are.  Nothing is allocated or
+ * synchronised.
+ * Inputs:  Tlog_host [B,G+1,V] dtype in page-locked host memory that the
+ *          device can address (cudaHostAlloc / cudaMallocHost memory under
+ *          unified addressing); ell [B] int32 (device), each clamped to
+ *          [0, G] when read.
+ * Outputs: Tlog_dev [B,G+1,V] dtype (device memory).
+ * Errors:  DSPARK_ERR_UNSUPPORTED_DTYPE; DSPARK_ERR_INVALID_ARG for a null
+ *          pointer, B outside [1, 4096], G outside [1, 16], V outside
+ *          [1, 2^24], a source that is not device-addressable page-locked host
+ *          memory or a destination that is not device memory (nothing is
+ *          enqueued); DSPARK_ERR_CUDA if the launch fails.  The caller
+ *          guarantees that both buffers hold B*(G+1)*V elements. */
+dspark_status dspark_gather_admitted_targets(const void *Tlog_host, void *Tlog_dev, const int32_t *ell, int B,
+                                             int G, int V, int dtype, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Drafting without a workspace, for callers that cannot allocate device
  * memory when they draft: e.g. a plugin of an inference engine that receives
  * only its inputs and outputs at enqueue time (the engine planned all memory

@@ -33,7 +33,7 @@ EXPORTS = ("dspark_version", "dspark_draft_workspace_size", "dspark_draft_markov
            "dspark_draft_noalloc_max_scratch", "dspark_draft_markov_noalloc", "dspark_schedule_threshold",
            "dspark_sts_workspace_size", "dspark_sts_fit", "dspark_survival_auc", "dspark_schedule_topk",
            "dspark_draft_noalloc_device_status", "dspark_draft_rnn", "dspark_verify_rnn", "dspark_get_near_ties",
-           "dspark_exp2_fma")
+           "dspark_exp2_fma", "dspark_gather_admitted_targets")
 
 
 class DsparkError(RuntimeError):
@@ -98,6 +98,8 @@ def load() -> ctypes.CDLL:
     lib.dspark_sts_fit.argtypes = [_vp] * 3 + [_i] * 4 + [_vp, _sz] + [_vp] * 6
     lib.dspark_survival_auc.restype = _i
     lib.dspark_survival_auc.argtypes = [_vp, _vp, _i, _i, _vp, _vp, _vp]
+    lib.dspark_gather_admitted_targets.restype = _i
+    lib.dspark_gather_admitted_targets.argtypes = [_vp, _vp, _vp, _i, _i, _i, _i, _vp]
     _lib = lib
     return lib
 
@@ -273,6 +275,19 @@ def dspark_get_near_ties(ws, stream=None):
     d, v = ctypes.c_uint32(0), ctypes.c_uint32(0)
     _call("dspark_get_near_ties", _ptr(ws), _stream(stream), ctypes.byref(d), ctypes.byref(v))
     return int(d.value), int(v.value)
+
+
+def dspark_gather_admitted_targets(Tlog_host, Tlog_dev, ell, stream=None):
+    """Enqueue one kernel that copies rows 0..ell[b] of every request of the
+    pinned host target logits [B, G+1, V] into the device buffer of the same
+    layout; ell: the device int32 [B] of admitted lengths."""
+    if Tlog_host.is_cuda or not Tlog_host.is_pinned() or not Tlog_host.is_contiguous():
+        raise ValueError("Tlog_host must be a contiguous pinned host tensor")
+    if Tlog_host.shape != Tlog_dev.shape or Tlog_host.dtype != Tlog_dev.dtype or ell.dtype != torch.int32:
+        raise ValueError("Tlog_host and Tlog_dev differ in shape or dtype, or ell is not int32")
+    B, G1, V = Tlog_dev.shape
+    _call("dspark_gather_admitted_targets", ctypes.c_void_p(Tlog_host.data_ptr()), _ptr(Tlog_dev), _ptr(ell), B,
+          G1 - 1, V, _dtype(Tlog_dev), _stream(stream))
 
 
 def dspark_exp2_fma(x, y, stream=None):

@@ -148,6 +148,26 @@ dspark_status dspark_verify(const void *Tlog, const void *L, const void *U, cons
     return cuda_status(launch_verify(a, ws, static_cast<cudaStream_t>(stream)));
 }
 
+dspark_status dspark_gather_admitted_targets(const void *Tlog_host, void *Tlog_dev, const int32_t *ell, int B,
+                                             int G, int V, int dtype, void *stream) {
+    if (dspark_status s = injected("dspark_gather_admitted_targets")) return s;
+    if (!dtype_ok(dtype)) return DSPARK_ERR_UNSUPPORTED_DTYPE;
+    if (!Tlog_host || !Tlog_dev || !ell || B < 1 || B > 4096 || G < 1 || G > 16 || V < 1 || V > (1 << 24))
+        return DSPARK_ERR_INVALID_ARG;
+    // The source must be page-locked host memory that the device can address,
+    // the destination device memory: anything else is refused before launch.
+    cudaPointerAttributes hs{}, dd{};
+    if (cudaPointerGetAttributes(&hs, Tlog_host) != cudaSuccess ||
+        cudaPointerGetAttributes(&dd, Tlog_dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return DSPARK_ERR_INVALID_ARG;
+    }
+    if (hs.type != cudaMemoryTypeHost || hs.devicePointer == nullptr) return DSPARK_ERR_INVALID_ARG;
+    if (dd.type != cudaMemoryTypeDevice && dd.type != cudaMemoryTypeManaged) return DSPARK_ERR_INVALID_ARG;
+    return cuda_status(launch_gather_admitted(hs.devicePointer, Tlog_dev, ell, B, G, V,
+                                              dtype == DSPARK_BF16 ? 2 : 4, static_cast<cudaStream_t>(stream)));
+}
+
 dspark_status dspark_draft_rnn(const void *L, const void *U, const void *Arec, const void *Wt, const int32_t *x0,
                                const float *temp, const float *u_draft, int B, int G, int V, int r, int dtype,
                                void *ws, size_t ws_bytes, int32_t *x_out, float *pd_x_out, float *rowmax_out,

@@ -101,5 +101,9 @@ cudaError_t launch_residual_tile_tc(const ResidualTcArgs &a, cudaStream_t st);
 cudaError_t launch_verify(const VerifyArgs &a, void *ws, cudaStream_t st);
 // y = 2^x by the FMA-pipe polynomial of common.cuh (diagnostics).
 cudaError_t launch_exp2_fma(const float *x, float *y, int n, cudaStream_t st);
+// Rows 0..ell[b] of each request of a [B, G+1, V] array from host memory
+// mapped into the device's address space (src: its device address).
+cudaError_t launch_gather_admitted(const void *src, void *dst, const int32_t *ell, int B, int G, int V,
+                                   int elem_bytes, cudaStream_t st);
 
 }  // namespace dspark

@@ -83,12 +83,12 @@ class DeviceRound:
                              for k, v in self.o.items() if k in ("tokens", "nout", "ell")}
 
     # -------------------------------------------------------------- running
-    def run(self, stream=None, overlap_confidence: bool = True):
+    def run(self, stream=None, overlap_confidence: bool = True, verify: bool = True):
         """Enqueue one round on `stream` (default: the current stream).  The
         confidence stage does not depend on the drafted tokens, so by default
         it runs on a side stream forked from `stream` at the start of the
         round and joined before the scheduler (a fork and a join when the
-        round is captured in a graph)."""
+        round is captured in a graph).  verify=False stops after scheduling."""
         t, o = self.t, self.o
         main = torch.cuda.current_stream(self.device) if stream is None else stream
         conf = lambda st: _lib.dspark_confidence(t["h"], t["w"], float(self.inp.bias), t["tau"], o["c"], o["S"], st)
@@ -108,7 +108,42 @@ class DeviceRound:
             conf(main)
         _lib.dspark_schedule(o["S"], t["knots_n"], t["knots_t"], self.budget, self.mode, self.ws, o["ell"],
                              o["n_adm"], o["theta"], o["order"], main)
-        self.verify(main)
+        if verify:
+            self.verify(main)
+
+    # Inputs that change every round and feed drafting, confidence and the
+    # draws; the target logits follow once the admitted lengths are known.
+    ROUND_INPUTS = ("L", "h", "x0", "temp", "u_draft", "u_accept", "u_final")
+
+    def run_from_host(self, stream=None, overlap_confidence: bool = True):
+        """Enqueue one round fed from pinned host memory, the way a serving
+        loop drives it: the round's draft-side inputs are copied in, drafting,
+        confidence and scheduling run, one kernel pulls in the target rows
+        that verification reads -- rows 0..ell_b of request b, what a target
+        forward over the admitted tokens produces -- reading ell on the
+        device, verification runs, and the emitted tokens, counts and lengths
+        go to pinned host memory (``host_out``).  Nothing waits on the host;
+        synchronise `stream` before reading ``host_out`` or calling
+        ``host_round_bytes``."""
+        if self.host is None:
+            raise RuntimeError("run_from_host needs DeviceRound(..., pinned_host=True)")
+        main = torch.cuda.current_stream(self.device) if stream is None else stream
+        with torch.cuda.stream(main):
+            for k in self.ROUND_INPUTS:
+                self.t[k].copy_(self.host[k], non_blocking=True)
+            self.run(main, overlap_confidence, verify=False)
+            _lib.dspark_gather_admitted_targets(self.host["Tlog"], self.t["Tlog"], self.o["ell"], main)
+            self.verify(main)
+        self.download(main)
+
+    def host_round_bytes(self):
+        """(host-to-device, device-to-host) bytes of the last run_from_host,
+        from the admitted lengths it brought back (synchronise first)."""
+        ell = self.host_out["ell"].numpy().astype(np.int64)
+        tl = self.host["Tlog"]
+        h2d = sum(self.host[k].numel() * self.host[k].element_size() for k in self.ROUND_INPUTS)
+        h2d += int((ell + 1).sum()) * tl.shape[2] * tl.element_size()
+        return h2d, self.d2h_bytes()
 
     def draft(self, stream=None):
         """The drafting stage alone (Markov or RNN head)."""

@@ -249,3 +249,23 @@ def test_rnn_entry_point_checks(lib, monkeypatch):
     assert d(*ok7, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, FAKE, FAKE, None) == 4
     monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_verify_rnn=5")
     assert v(*ok12, 4, 5, 1024, 16, 1, FAKE_WS, 1 << 30, FAKE, FAKE, FAKE, None, None) == 5
+
+
+def test_gather_admitted_targets_checks(lib, monkeypatch):
+    """The admitted target rows from host memory: the host checks reject an
+    unknown dtype, bad sizes and a null pointer before any CUDA call (the
+    pointer checks that follow need a GPU); host-side injection."""
+    f = lib.dspark_gather_admitted_targets
+    assert f(FAKE, FAKE, FAKE, 4, 5, 1024, 7, None) == 2
+    assert f(FAKE, FAKE, FAKE, 0, 5, 1024, 1, None) == 1
+    assert f(FAKE, FAKE, FAKE, 4097, 5, 1024, 1, None) == 1
+    assert f(FAKE, FAKE, FAKE, 4, 0, 1024, 1, None) == 1
+    assert f(FAKE, FAKE, FAKE, 4, 17, 1024, 1, None) == 1
+    assert f(FAKE, FAKE, FAKE, 4, 5, 0, 1, None) == 1
+    assert f(FAKE, FAKE, FAKE, 4, 5, (1 << 24) + 1, 1, None) == 1
+    for k in range(3):
+        args = [FAKE, FAKE, FAKE]
+        args[k] = None
+        assert f(*args, 4, 5, 1024, 1, None) == 1
+    monkeypatch.setenv("DSPARK_INJECT_ERROR", "dspark_gather_admitted_targets=4")
+    assert f(FAKE, FAKE, FAKE, 4, 5, 1024, 1, None) == 4

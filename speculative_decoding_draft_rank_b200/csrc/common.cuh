@@ -31,6 +31,7 @@ __device__ __forceinline__ void flag_status(WsHeader *h, uint32_t bit) {
 constexpr int kPadDraftTies = 8;
 constexpr int kPadVerifyTies = 9;
 constexpr int kPadSchedArrive = 4;   // the scheduler's arrival counter
+constexpr int kPadRowItems = 5;     // the verification row pass's item counter
 constexpr float kNearTie = 1e-5f;
 __device__ __forceinline__ void count_near_tie(WsHeader *h, int slot) { atomicAdd(&h->pad[slot], 1u); }
 

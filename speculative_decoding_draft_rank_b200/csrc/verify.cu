@@ -114,7 +114,7 @@ __global__ void verify_plan(const int32_t *__restrict__ ell, int B, int G, Verif
     __shared__ int tot[33];
     __shared__ int carry;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    if (tid == 0) { carry = 0; w.hdr->pad[1] = 0; }
+    if (tid == 0) { carry = 0; w.hdr->pad[1] = 0; w.hdr->pad[kPadRowItems] = 0; }
     __syncthreads();
     for (int b0 = 0; b0 < B; b0 += blockDim.x) {
         const int b = b0 + tid;
@@ -283,7 +283,6 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
     const int nrows = *reinterpret_cast<volatile uint32_t *>(&w.hdr->pad[0]);
     const int nwork = nrows * w.nChunks;
     if ((int)blockIdx.x >= nwork) return;
-    const int nmine = (nwork - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     if (threadIdx.x == 0) {
         for (int q = 0; q < kVrWarps * 2; ++q) tc::mbar_init(&full[q], 1);
         abort_s = 0;
@@ -294,64 +293,82 @@ __global__ void __launch_bounds__(kVrThreads, 1) verify_rows_bulk(const __nv_bfl
     volatile int *abort_flag = &abort_s;
     unsigned char *stage0 = vr_smem + warp * 2 * kVrStageBytes;
     uint64_t *myfull = full + warp * 2;
-    const int nk = (nmine - warp + kVrWarps - 1) / kVrWarps;   // this warp's items: k = 0..nk-1
-    auto item_of = [&](int k) { return (int)blockIdx.x + (warp + kVrWarps * k) * (int)gridDim.x; };
-    auto load_rk = [&](int k) { return k < nk ? w.rows[item_of(k) / w.nChunks] : 0; };
-    // Row ids of items base .. base + 63: lane l holds items base + l (cur) and base + 32 + l (nxt).
-    int base = 0, cur = load_rk(lane), nxt = load_rk(32 + lane);
-    auto rk_of = [&](int k) {
-        const int a = __shfl_sync(0xffffffffu, cur, (k - base) & 31);
-        const int b2 = __shfl_sync(0xffffffffu, nxt, (k - base) & 31);
-        return (k - base) < 32 ? a : b2;
-    };
+    // Items: a warp's first two are fixed (g and g + NW, g its index over the
+    // grid's NW warps); after that each warp claims one item at a time from
+    // the counter that verify_plan zeroed (claimed items are numbered from
+    // 2 NW), so the warps finish together instead of some taking one item
+    // more.  Lane 0 fires a claim and the claimed item's row-id load one
+    // iteration before the item is issued, so both latencies pass while the
+    // warp computes.  A warp's claims increase, so the first out-of-range item
+    // it meets ends its work with nothing claimed left over.
+    const int NW = (int)gridDim.x * kVrWarps;
+    uint32_t *claim_ctr = &w.hdr->pad[kPadRowItems];
+    int itA = warp * (int)gridDim.x + (int)blockIdx.x, itB = itA + NW;   // the items in stages 0 and 1
+    int rkA = 0, rkB = 0, nxt_it = nwork, nxt_rk = 0, pend = nwork;
+    if (lane == 0) {
+        pend = 2 * NW + (int)atomicAdd(claim_ctr, 1u);
+        if (itA < nwork) rkA = w.rows[itA / w.nChunks];
+        if (itB < nwork) rkB = w.rows[itB / w.nChunks];
+    }
+    rkA = __shfl_sync(0xffffffffu, rkA, 0);
+    rkB = __shfl_sync(0xffffffffu, rkB, 0);
     const uint64_t pol = tc::policy_evict_first();
-    auto issue = [&](int k) {
-        const int rk = rk_of(k);
-        if (lane == 0) {
-            const int item = item_of(k);
-            const int c = item % w.nChunks;
-            const int c0 = c * kChunk, ncols = min(kChunk, V - c0);
-            const __nv_bfloat16 *src = Tlog + ((size_t)(rk >> 5) * (G + 1) + (rk & 31)) * V + c0;
-            tc::mbar_arrive_expect_tx(&myfull[k & 1], (uint32_t)ncols * 2);
-            tc::bulk_load(stage0 + (k & 1) * kVrStageBytes, src, (uint32_t)ncols * 2, &myfull[k & 1], pol);
-        }
+    auto issue = [&](int item, int rk, int s) {   // lane 0
+        const int c = item % w.nChunks;
+        const int c0 = c * kChunk, ncols = min(kChunk, V - c0);
+        const __nv_bfloat16 *src = Tlog + ((size_t)(rk >> 5) * (G + 1) + (rk & 31)) * V + c0;
+        tc::mbar_arrive_expect_tx(&myfull[s], (uint32_t)ncols * 2);
+        tc::bulk_load(stage0 + s * kVrStageBytes, src, (uint32_t)ncols * 2, &myfull[s], pol);
     };
-    if (nk > 0) issue(0);
-    if (nk > 1) issue(1);
-    int issued = min(nk, 2);
-    for (int k = 0; k < nk; ++k) {
-        if (k - base == 32) {   // slide the row-id window by 32 items
-            cur = nxt;
-            base += 32;
-            nxt = load_rk(base + 32 + lane);
+    if (lane == 0) {
+        if (itA < nwork) issue(itA, rkA, 0);
+        if (itB < nwork) issue(itB, rkB, 1);
+        nxt_it = pend;   // waits for the first claim while the copies fly
+        if (nxt_it < nwork) {
+            nxt_rk = w.rows[nxt_it / w.nChunks];
+            pend = 2 * NW + (int)atomicAdd(claim_ctr, 1u);
         }
-        const bool ok = tc::mbar_wait_bounded(&myfull[k & 1], (k >> 1) & 1, abort_flag, budget);
+    }
+    for (int k = 0;; ++k) {
+        const int s = k & 1;
+        const int item = s ? itB : itA;
+        if (item >= nwork) break;
+        const bool ok = tc::mbar_wait_bounded(&myfull[s], (k >> 1) & 1, abort_flag, budget);
         if (!__all_sync(0xffffffffu, ok)) {
             // Give up: wait (bounded, ignoring the abort flag) for this warp's
-            // copies in flight so that none lands after the CTA exits.
+            // copies in flight (this stage's, and the other's if it holds an
+            // item) so that none lands after the CTA exits.
             if (lane == 0) {
                 int dummy = 0;
-                for (int kk = k; kk < issued; ++kk)
-                    tc::mbar_wait_bounded(&myfull[kk & 1], (kk >> 1) & 1, &dummy, kVrWaitBudget / 4);
+                tc::mbar_wait_bounded(&myfull[s], (k >> 1) & 1, &dummy, kVrWaitBudget / 4);
+                if ((s ? itA : itB) < nwork)
+                    tc::mbar_wait_bounded(&myfull[s ^ 1], ((k + 1) >> 1) & 1, &dummy, kVrWaitBudget / 4);
                 *abort_flag = 1;
                 flag_status(w.hdr, DSPARK_DEV_TIMEOUT);
             }
             break;
         }
         uint4 v[kVrPieces];
-        const unsigned char *src = stage0 + (k & 1) * kVrStageBytes + lane * 16;
+        const unsigned char *src = stage0 + s * kVrStageBytes + lane * 16;
 #pragma unroll
         for (int i = 0; i < kVrPieces; ++i) v[i] = *reinterpret_cast<const uint4 *>(src + i * 512);
-        const int rk = rk_of(k);
+        const int rk = s ? rkB : rkA;
         // The stage is free once every lane's reads are done: the next copy may
         // land in it (generic reads, then async-proxy writes).
         tc::fence_proxy_async_smem();
         __syncwarp();
-        if (k + 2 < nk) {
-            issue(k + 2);
-            issued = k + 3;
+        // Refill this stage with the claimed item; claim the next one.
+        const int nit = __shfl_sync(0xffffffffu, nxt_it, 0);
+        const int nrk = __shfl_sync(0xffffffffu, nxt_rk, 0);
+        if (lane == 0 && nit < nwork) {
+            issue(nit, nrk, s);
+            nxt_it = pend;
+            if (nxt_it < nwork) {
+                nxt_rk = w.rows[nxt_it / w.nChunks];
+                pend = 2 * NW + (int)atomicAdd(claim_ctr, 1u);
+            }
         }
-        const int item = item_of(k);
+        if (s) { itB = nit; rkB = nrk; } else { itA = nit; rkA = nrk; }
         const int jrow = item / w.nChunks, ch = item - jrow * w.nChunks;
         const int ncols = min(kChunk, V - ch * kChunk);
         float T = temp_s[rk >> 5];

@@ -250,18 +250,18 @@ __global__ void __launch_bounds__(kRowThreads) verify_rows(const T *__restrict__
 }
 
 // bf16 rows: persistent CTAs (one per SM) over the (row, 4096-column chunk)
-// work items, item q of CTA c being item c + q * grid.  Warp w of the CTA
-// takes items q = w, w + 12, ... and streams them itself: it owns two
-// shared-memory stages and keeps a bulk copy in flight into one while it
-// reduces the other (evict-first: every target row is read once, so the
-// transition factor that drafting left in L2 stays there for the residual
+// work items.  Each warp streams its items itself: its first two are fixed,
+// the rest it claims one at a time from a counter in the workspace header.
+// It owns two shared-memory stages and keeps a bulk copy in flight into one
+// while it reduces the other (evict-first: every target row is read once, so
+// the transition factor that drafting left in L2 stays there for the residual
 // pass).  As soon as a chunk's values are in registers the warp issues the
-// copy two items ahead into the stage it just read, reduces its 4096 columns
-// to (max, sum of exp((t - max) / T), lowest argmax) and writes the chunk
-// partial -- no block barrier, no producer to wait for.  The row of an item
-// comes from the compacted row list, read 32 items ahead; temperatures are
-// staged in shared memory.  Lane l reads the 16-byte pieces l, l + 32, ...
-// of the chunk (bank-conflict free).
+// next claimed item's copy into the stage it just read, reduces its 4096
+// columns to (max, sum of exp((t - max) / T), lowest argmax) and writes the
+// chunk partial -- no block barrier, no producer to wait for.  The row of an
+// item comes from the compacted row list; temperatures are staged in shared
+// memory.  Lane l reads the 16-byte pieces l, l + 32, ... of the chunk
+// (bank-conflict free).
 constexpr int kVrWarps = 12;
 constexpr int kVrThreads = kVrWarps * 32;
 constexpr int kVrStageBytes = kChunk * 2;            // 8 KB
